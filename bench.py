@@ -1,0 +1,361 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the quantized KV cache (libkvq.so, one process per GPU).
+
+A step is one decode step of the whole batch: kvq_append_token (the new
+token enters the residual window; a flush quantizes G tokens when due) and
+kvq_decode_attention over the packed cache.  Metric: packed-KV bytes read by
+the decode attention per second (GB/s), with tokens/s alongside.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 8b2] [--impl kivi|reference]
+
+Timing: CUDA events on the launching stream around exactly K steps, bracketed
+by a barrier and torch.cuda.synchronize(); the max over ranks is reported.
+Each step targets the next of several identical cache replicas whose total
+size is over 3x the L2, so every step streams its cache from HBM.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-KV decode attn: packed-KV GB/s (% of HBM peak), tokens/s"
+HBM_FALLBACK_GBS = 6650.0
+NORTH_STAR_HBM_GBS = 8000.0
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return HBM_FALLBACK_GBS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- inputs on the device
+def device_inputs(w, device, steps_total):
+    """Seeded synthetic inputs with the workload's recipe, drawn on the GPU
+    (standard normal, K outlier channels x20, 2% of V tokens per batch row x10)."""
+    import torch
+    from quantized_kv_cache_18_b200 import workloads as W
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+    g = torch.Generator(device=device)
+    g.manual_seed(1000 + w.seed)
+    shape = (w.batch, w.num_kv_heads, w.seq_len, w.head_dim)
+    ch = torch.as_tensor(W.k_outlier_channels(w), device=device)
+    K = torch.randn(shape, generator=g, device=device)
+    K[..., ch] *= w.k_outlier_scale
+    K = K.to(dt)
+    V = torch.randn(shape, generator=g, device=device)
+    if w.v_channel_outliers:
+        V[..., ch] *= w.k_outlier_scale
+    for b in range(w.batch):
+        vt = torch.as_tensor(W.v_outlier_tokens(w, b), device=device)
+        if vt.numel():
+            V[b, :, vt, :] *= w.v_outlier_scale
+    V = V.to(dt)
+    q = torch.randn((steps_total, w.batch, w.num_q_heads, w.head_dim), generator=g, device=device).to(dt)
+    kn = torch.randn((steps_total, w.batch, w.num_kv_heads, w.head_dim), generator=g, device=device)
+    kn[..., ch] *= w.k_outlier_scale
+    vn = torch.randn((steps_total, w.batch, w.num_kv_heads, w.head_dim), generator=g, device=device)
+    hit = torch.rand((steps_total, w.batch), generator=g, device=device) < w.v_outlier_frac
+    vn[hit] *= w.v_outlier_scale
+    return K, V, q, kn.to(dt), vn.to(dt)
+
+
+def step_bytes(cache) -> int:
+    """Packed bytes one decode attention reads: every group record and every
+    window token (16-bit key and value)."""
+    c, lay = cache.cfg, cache.layout
+    rows = c.batch * c.num_kv_heads
+    return rows * (cache.quantized_len // c.group * lay.record_bytes + cache.window_len * 2 * c.head_dim * 2)
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_gpu(args, w, rank, world):
+    import torch
+    from quantized_kv_cache_18_b200 import build as kbuild
+    from quantized_kv_cache_18_b200 import _lib as L
+    from quantized_kv_cache_18_b200.cache import QuantizedKVCache, config_from_workload, launch_count
+
+    kbuild.build()
+    device = torch.device("cuda", torch.cuda.current_device())
+    steps_total = args.warmup + args.steps
+    max_seq = w.seq_len + steps_total + 1
+    cfg = config_from_workload(w, max_seq)
+    K, V, q, kn, vn = device_inputs(w, device, steps_total)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    probe = QuantizedKVCache(cfg, device=device)
+    n_rep = max(2, math.ceil(3 * l2 / probe.nbytes) + 1)
+    caches = [probe] + [QuantizedKVCache(cfg, device=device) for _ in range(n_rep - 1)]
+    for c in caches:
+        c.prefill(K, V)
+    del K, V
+    torch.cuda.synchronize()
+    out = torch.empty((w.batch, w.num_q_heads, w.head_dim), dtype=torch.float32, device=device)
+    lib = L.load()
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    scale = ctypes.c_float(w.scale)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    qp = [ptr(q[i]) for i in range(steps_total)]
+    knp = [ptr(kn[i]) for i in range(steps_total)]
+    vnp = [ptr(vn[i]) for i in range(steps_total)]
+    outp = ptr(out)
+
+    def one_step(i, ev=None):
+        c = caches[i % n_rep]
+        L.check(lib.kvq_append_token(c.handle, knp[i], vnp[i], sp), "append")
+        if ev is not None:
+            ev[0].record(stream)
+        L.check(lib.kvq_decode_attention(c.handle, qp[i], outp, scale, ptr(c.ws), c.ws.numel(), sp), "attention")
+        if ev is not None:
+            ev[1].record(stream)
+        return step_bytes(c)
+
+    for i in range(args.warmup):
+        one_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = launch_count()
+    total_bytes = 0
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t0.record(stream)
+        for j in range(args.steps):
+            total_bytes += one_step(args.warmup + j, attn_ev[j])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    launches = launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
+    for c in caches:
+        if c.status():
+            raise RuntimeError("device status word set during the bench")
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end-to-end through the public API with host buffers: H2D of the step's
+    # inputs from pinned memory, append + attention, D2H of the output
+    h_q = q[args.warmup:].cpu().pin_memory()
+    h_kn = kn[args.warmup:].cpu().pin_memory()
+    h_vn = vn[args.warmup:].cpu().pin_memory()
+    h_out = torch.empty((args.steps,) + tuple(out.shape), dtype=torch.float32).pin_memory()
+    d_q, d_kn, d_vn = torch.empty_like(q[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
+    e_caches = [QuantizedKVCache(cfg, device=device) for _ in range(n_rep)]
+    K, V, _, _, _ = device_inputs(w, device, 1)
+    for c in e_caches:
+        c.prefill(K, V)
+    del K, V
+    torch.cuda.synchronize()
+    e_bytes = 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for j in range(args.steps):
+        c = e_caches[j % n_rep]
+        d_q.copy_(h_q[j], non_blocking=True)
+        d_kn.copy_(h_kn[j], non_blocking=True)
+        d_vn.copy_(h_vn[j], non_blocking=True)
+        c.append(d_kn, d_vn)
+        c.attention(d_q, out=out)
+        h_out[j].copy_(out, non_blocking=True)
+        e_bytes += step_bytes(c)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e_ms = float(t.item())
+
+    res = dict(ms=ms, bytes=total_bytes, attn_ms=attn_ms, launches=launches, clocks=clk.summary(),
+               e2e_ms=e_ms, e2e_bytes=e_bytes, n_rep=n_rep, splits=caches[0].decode_splits,
+               h2d=int(q[0].numel() * 2 + kn[0].numel() * 2 + vn[0].numel() * 2), d2h=int(out.numel() * 4),
+               step_bytes_last=step_bytes(caches[0]))
+    return res
+
+
+# ---------------------------------------------------------------- oracle (CPU) timing
+def oracle_sample(w, budget_s: float, steps: int = 1):
+    """Times the float64 oracle's decode step (append + attention over the
+    dequantized cache) on a bounded sample of (batch, kv-head) rows."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+    from oracle import attention as oatt
+    from oracle.cache import KiviRow
+    from oracle.numerics import decode16
+    from quantized_kv_cache_18_b200 import workloads as W
+
+    t_total, bytes_total, rows = 0.0, 0, 0
+    g = w.gqa
+    b, h = 0, 0
+    wall0 = time.time()
+    while t_total < budget_s and time.time() - wall0 < 3 * budget_s + 15:
+        k, v = W.prefill_row(w, b, h)
+        row = KiviRow(w.head_dim, w.bits, w.group, w.residual, w.dtype)
+        row.prefill(k, v)
+        for s in range(1, steps + 1):
+            kn, vn = W.decode_token(w, s)
+            q = W.query(w, s)[b, h * g:(h + 1) * g]
+            t = time.perf_counter()
+            row.append(kn[b, h], vn[b, h])
+            Kd, Vd = row.dequantized()
+            oatt.attention(decode16(q, w.dtype), Kd, Vd, w.scale)
+            t_total += time.perf_counter() - t
+            bytes_total += (row.tq // w.group) * (w.group * w.head_dim * w.bits // 4 + 4 * w.head_dim + 4 * w.group) \
+                + row.r * 4 * w.head_dim
+        rows += 1
+        h += 1
+        if h == w.num_kv_heads:
+            h, b = 0, (b + 1) % w.batch
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return dict(value=bytes_total / t_total / 1e9, seconds=t_total, rows=rows, steps=steps, cores=threads)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="8b2")
+    ap.add_argument("--impl", default="kivi", choices=["kivi", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    from quantized_kv_cache_18_b200 import workloads as W
+    w = W.WORKLOADS[args.config]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    cfg_desc = {"workload": f"{w.name}: B{w.batch} Hkv{w.num_kv_heads} Hq{w.num_q_heads} d{w.head_dim} "
+                            f"S{w.seq_len} {w.scheme} {w.bits}-bit G{w.group} R{w.residual}",
+                "global_batch": w.batch * world, "seq_len": w.seq_len, "parallelism": f"dp{world}",
+                "l2": "cache replicas > 3x L2, rotated per step"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        samp = oracle_sample(w, args.cpu_budget, steps=max(1, args.steps // 10))
+        line = {"impl": "reference", "metric": METRIC, "value": samp["value"], "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg_desc,
+                "cpu_baseline": {"value": samp["value"], "unit": "GB/s", "cores": samp["cores"], "kind": "oracle",
+                                 "sample": f"{samp['rows']} (batch, kv-head) rows x {samp['steps']} steps"},
+                "e2e": {"value": samp["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_gpu(args, w, rank, world)
+    hbm, peak_kind = _peaks()
+    value = res["bytes"] * world / (res["ms"] * 1e-3) / 1e9
+    attn_mean = statistics.mean(res["attn_ms"])
+    achieved = res["step_bytes_last"] / (attn_mean * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(res["ms"] / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16 mma (fp32 accumulate) over int2/int4 codes",
+        "data": "synthetic", "config": cfg_desc,
+        "tokens_per_s": round(w.batch * world * args.steps / (res["ms"] * 1e-3), 1),
+        "pct_of_north_star_hbm": round(100 * value / world / NORTH_STAR_HBM_GBS, 2),
+        "roofline": {"bound": "hbm", "kernel": "kivi_attn_kernel + lse_merge_kernel (one decode attention)",
+                     "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": None,
+                     "bytes_per_launch": res["step_bytes_last"], "mean_launch_us": round(attn_mean * 1e3, 2)},
+        "e2e": {"value": round(res["e2e_bytes"] * world / (res["e2e_ms"] * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["launches"], "clocks": res["clocks"], "replicas": res["n_rep"],
+        "decode_splits": res["splits"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        samp = oracle_sample(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(samp["value"], 4), "unit": "GB/s", "cores": samp["cores"],
+                                "kind": "oracle", "sample": f"{samp['rows']} (batch, kv-head) rows of {w.name}, "
+                                                            f"one append + attention each, {samp['seconds']:.1f} s"}
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

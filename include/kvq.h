@@ -1,0 +1,229 @@
+/*
+ * kvq.h -- C ABI of the quantized KV-cache library (libkvq.so, sm_100a).
+ *
+ * What the library computes comes from these web pages on KV-cache
+ * quantization (cited by title and section):
+ *   [KIVI]  "Quantification du KV-Cache : TurboQuant et l'etat de l'art en
+ *           2026", section "KIVI (2024) -- la quantification asymetrique par
+ *           canal"; zubnet.ai survey of KV-cache compression techniques,
+ *           paragraph "Famille deux, c'est la quantification".
+ *   [TQ]    same survey paragraph; "La compression du cache KV est une decision
+ *           d'infrastructure, pas un debat sur les modeles", section
+ *           "TurboQuant est le choix de portabilite, pas le gagnant universel";
+ *           "Quantification du KV-Cache ...", "TurboQuant : les cinq
+ *           innovations" items 1-4.
+ *   [DEC]   "La compression du cache KV ...", section "... quand la HBM, pas
+ *           les FLOPs, est votre plafond" (every decoded token reads the whole
+ *           cache); "Quantification du KV-Cache ...", "Le probleme" (the cache
+ *           lets each new token look back without recomputation).
+ *   [MERGE] "KV-cache compresse et modeles 4-bit : la compression s'impose
+ *           comme le premier levier d'inference", section "Minima-KV : la
+ *           compression sans eviction" (partial attention states merged by a
+ *           globally normalised online softmax).
+ *
+ * Conventions for every call:
+ *   - Ownership: the caller allocates and frees all device memory (cache
+ *     buffer, inputs, outputs, workspace).  The library keeps only a small
+ *     host-side handle; it never allocates device memory.
+ *   - Pointers marked "device" must point to memory of the current CUDA device
+ *     and be 16-byte aligned; 16-bit inputs are bf16 or fp16 bit patterns as
+ *     the config says.  `stream` is a cudaStream_t (NULL = legacy default).
+ *   - Asynchrony: every call only enqueues kernels on `stream` and returns.
+ *     Argument errors are detected on the host and returned before anything is
+ *     launched.  Conditions found on the device (non-finite input, a quantizer
+ *     parameter that overflows fp16, a bounded wait that ran out) set bits of a
+ *     status word inside the cache buffer; kvq_get_status reads it.
+ *   - One handle must not be used from two streams at the same time.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer   */
+  KVQ_ERR_UNSUPPORTED = 2,   /* config outside the supported shapes         */
+  KVQ_ERR_CAPACITY = 3,      /* sequence would exceed max_seq                */
+  KVQ_ERR_CUDA = 4,          /* a CUDA runtime call failed                   */
+  KVQ_ERR_DEVICE_STATUS = 5  /* kvq_get_status: the device status word is set */
+} kvq_status;
+
+enum { KVQ_KIVI = 0, KVQ_TURBO = 1 };
+enum { KVQ_BF16 = 0, KVQ_FP16 = 1 };
+
+/* Device status bits (kvq_get_status). */
+enum {
+  KVQ_DEV_NONFINITE_INPUT = 1u << 0, /* a quantized input was inf or nan       */
+  KVQ_DEV_PARAM_OVERFLOW = 1u << 1,  /* a scale or zero-point overflowed fp16  */
+  KVQ_DEV_WAIT_TIMEOUT = 1u << 2     /* a bounded pipeline wait gave up        */
+};
+
+/*
+ * Cache configuration.
+ *   scheme        KVQ_KIVI (int2/int4 asymmetric, [KIVI]) or KVQ_TURBO ([TQ]).
+ *   bits          KIVI: 2 or 4.  TURBO: 3 (codes per rotated coordinate).
+ *   group         KIVI: G, tokens per key quantization group (32 or 64).
+ *                 TURBO: tokens flushed from the window at a time (32).
+ *   residual      R, tokens always kept unquantized (a multiple of group).
+ *   head_dim      d: 64 or 128 (TURBO: 128).
+ *   num_kv_heads, num_q_heads  Hkv and Hq; Hq / Hkv in {1, 2, 4, 8}; query
+ *                 head h reads kv head h / (Hq / Hkv).
+ *   batch         B sequences; all of them have the same length.
+ *   max_seq       capacity in tokens per sequence.
+ *   dtype         KVQ_BF16 or KVQ_FP16: the 16-bit format of k, v and q.
+ *   qjl_dim       TURBO: m, rows of the 1-bit QJL sketch of the key residual
+ *                 (128).  KIVI: 0.
+ */
+typedef struct {
+  int32_t scheme;
+  int32_t bits;
+  int32_t group;
+  int32_t residual;
+  int32_t head_dim;
+  int32_t num_kv_heads;
+  int32_t num_q_heads;
+  int32_t batch;
+  int32_t max_seq;
+  int32_t dtype;
+  int32_t qjl_dim;
+  int32_t reserved;
+} kvq_config;
+
+/*
+ * Where things live inside the caller's cache buffer (byte offsets from its
+ * start).  For KIVI every (batch, kv head) row holds `groups_per_row` group
+ * records of `record_bytes` each; a record packs G tokens: the key codes and
+ * value codes of its 32-token blocks (16 INT2 or 8 INT4 codes per 32-bit word,
+ * in the fragment order of the decode kernel), the fp16 (scale, zero) of each
+ * key channel, and the fp16 (scale, zero) of each value token.  Each row also
+ * owns a ring of `ring_tokens` 16-bit key rows and one of value rows (the
+ * residual window).
+ */
+typedef struct {
+  uint64_t total_bytes;      /* == kvq_cache_bytes                           */
+  uint64_t records_offset;   /* [B][Hkv][groups_per_row][record_bytes]       */
+  uint64_t record_bytes;     /* bytes of one group record (KIVI) or token    */
+                             /* record (TURBO)                               */
+  uint64_t groups_per_row;   /* record capacity of one row                   */
+  uint64_t window_offset;    /* [B][Hkv][2 (k, v)][ring_tokens][d] 16-bit    */
+  uint64_t ring_tokens;      /* R + group                                    */
+  uint64_t params_offset;    /* TURBO: rotation, sketch and codebook         */
+  uint64_t params_bytes;
+  uint64_t status_offset;    /* uint32 device status word                    */
+} kvq_layout;
+
+typedef struct kvq_cache kvq_cache; /* opaque host handle */
+
+/* Device bytes the caller must allocate for a cache of this config; 0 if the
+ * config is invalid or unsupported. */
+size_t kvq_cache_bytes(const kvq_config* cfg);
+
+/* Device scratch bytes kvq_decode_attention needs (split-K partial states);
+ * 0 if the config is invalid. */
+size_t kvq_workspace_bytes(const kvq_config* cfg);
+
+/* Fills *out with the buffer layout of a config. */
+kvq_status kvq_get_layout(const kvq_config* cfg, kvq_layout* out);
+
+/*
+ * Creates a host handle over the caller's device buffer `dev_buf` (at least
+ * kvq_cache_bytes(cfg) bytes, 256-byte aligned) and enqueues the clearing of
+ * its status word on `stream`.  The cache starts empty.  On success *out owns
+ * only host memory; release it with kvq_cache_destroy.
+ */
+kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes,
+                          void* stream, kvq_cache** out);
+
+/*
+ * TURBO only, once after kvq_cache_init and before any prefill.  Derives the
+ * deployment constants of [TQ] on the device and stores them in the cache
+ * buffer:
+ *   rot_gauss  device float32 [d][d]: a seeded N(0,1) draw; the rotation is
+ *              the Q factor of its QR decomposition with diag(R) > 0
+ *              ("rotation orthogonale aleatoire").
+ *   qjl_gauss  device float32 [m][d]: the N(0,1) QJL projection S, used as is.
+ * The 8-level Lloyd-Max codebook for N(0, 1/d) ("TurboQuant : les cinq
+ * innovations", item 2) is computed on the device as well.
+ */
+kvq_status kvq_turbo_setup(kvq_cache* cache, const float* rot_gauss, const float* qjl_gauss,
+                           void* stream);
+
+/*
+ * Prefill ([KIVI] / [TQ]).  k, v: device [B][Hkv][seq_len][d], 16-bit.
+ * The cache must be empty.  Quantizes T_q = G * floor(max(0, seq_len - R) / G)
+ * tokens per row and keeps the other seq_len - T_q tokens, unchanged, in the
+ * residual window ("TurboQuant : les cinq innovations", item 4).
+ * Errors: KVQ_ERR_CAPACITY if seq_len > max_seq; KVQ_ERR_INVALID_ARG for a
+ * null or misaligned pointer, a negative length or a non-empty cache.
+ */
+kvq_status kvq_quantize_prefill(kvq_cache* cache, const void* k, const void* v, int32_t seq_len,
+                                void* stream);
+
+/*
+ * One decode step's new token per row.  k_new, v_new: device [B][Hkv][d],
+ * 16-bit.  The token enters the residual window; when the window then holds
+ * R + G tokens, its oldest G tokens are quantized (one new key group and G
+ * value tokens) and leave it.
+ * Errors: KVQ_ERR_CAPACITY if the sequence would exceed max_seq.
+ */
+kvq_status kvq_append_token(kvq_cache* cache, const void* k_new, const void* v_new, void* stream);
+
+/*
+ * Single-token decode attention over the whole cache ([DEC], [MERGE]).
+ *   q          device [B][Hq][d], 16-bit.
+ *   out        device float32 [B][Hq][d]: softmax(scale * q.k_t) v_t summed
+ *              over every cached token t, quantized tokens dequantized on the
+ *              fly and window tokens exact.
+ *   softmax_scale  usually 1/sqrt(d).
+ *   workspace  device scratch of at least kvq_workspace_bytes(cfg) bytes; its
+ *              contents need no initialisation and are overwritten.
+ * Errors: KVQ_ERR_INVALID_ARG on an empty cache, null pointers or a short
+ * workspace.
+ */
+kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, float* out, float softmax_scale,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, reads the device status word into *bits (may be
+ * NULL) and returns KVQ_ERR_DEVICE_STATUS if any bit is set, else KVQ_OK.
+ * `clear` != 0 also zeroes the word.
+ */
+kvq_status kvq_get_status(kvq_cache* cache, uint32_t* bits, int32_t clear, void* stream);
+
+/* Host-side counters (no device access). */
+int32_t kvq_seq_len(const kvq_cache* cache);        /* tokens per sequence   */
+int32_t kvq_quantized_len(const kvq_cache* cache);  /* T_q                   */
+int32_t kvq_window_len(const kvq_cache* cache);     /* r = seq_len - T_q     */
+int32_t kvq_window_head(const kvq_cache* cache);    /* ring slot of the oldest window token */
+
+/*
+ * Checkpoint / resume: sets the counters of a handle whose buffer already
+ * holds a cache in the documented layout (e.g. restored by the caller).
+ * Requires quantized_len % G == 0, window_head % G == 0, and
+ * 0 <= seq_len - quantized_len < R + G.
+ */
+kvq_status kvq_cache_set_state(kvq_cache* cache, int32_t seq_len, int32_t quantized_len,
+                               int32_t window_head);
+
+void kvq_cache_destroy(kvq_cache* cache);
+
+const char* kvq_status_string(kvq_status s);
+
+/* Kernels this library has launched since it was loaded (all handles). */
+uint64_t kvq_launch_count(void);
+
+/* Decode-attention split count the library picks for the current state. */
+int32_t kvq_decode_splits(const kvq_cache* cache);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

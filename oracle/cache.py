@@ -6,7 +6,7 @@ Residual window ("Quantification du KV-Cache : TurboQuant et l'etat de l'art en
 section "KIVI (2024)", "un residu FP16 pour les derniers tokens"): the most
 recent tokens stay unquantized and the attention kernel sees the hybrid cache
 as one sequence.  The pages give the window size (128) but not how tokens move
-out of it.  Reading used here (the design doc lists it):
+out of it.  Reading used here:
 
 * prefill of S tokens quantizes T_q = G * floor(max(0, S - R) / G) tokens and
   keeps r = S - T_q in the window (R <= r < R + G once S >= R);
@@ -71,12 +71,11 @@ class KiviRow:
         G, bits = self.G, self.bits
         k = decode16(kb, self.dtype)
         v = decode16(vb, self.dtype)
-        for g0 in range(0, k.shape[0], G):
-            c, s, z = kivi.quantize_keys(k[g0:g0 + G], bits)
-            self.ok &= kivi.in_range(k[g0:g0 + G], s, z)
-            self.kc = np.concatenate([self.kc, c])
-            self.ks = np.concatenate([self.ks, s[None]])
-            self.kz = np.concatenate([self.kz, z[None]])
+        c, s, z = kivi.quantize_key_groups(k, bits, G)
+        self.ok &= kivi.in_range(k, s, z)
+        self.kc = np.concatenate([self.kc, c])
+        self.ks = np.concatenate([self.ks, s])
+        self.kz = np.concatenate([self.kz, z])
         c, s, z = kivi.quantize_values(v, bits)
         self.ok &= kivi.in_range(v, s, z)
         self.vc = np.concatenate([self.vc, c])

@@ -7,7 +7,7 @@ per channel and values per token, each with its own min/max parameters, at
 2 bits (the 4-bit width follows the same recipe), with the most recent tokens
 kept unquantized.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 * asymmetric parameters: s = (max - min) / (2^b - 1) rounded to fp16 (ties to
   even), z = min rounded to fp16;
 * code = clamp(round_half_even((x - z) / s), 0, 2^b - 1), decided exactly by
@@ -68,6 +68,17 @@ def quantize_keys(kg: np.ndarray, bits: int):
     kg = np.asarray(kg, np.float64)
     s, z = params(kg.min(axis=0), kg.max(axis=0), bits)
     return codes(kg, s[None, :], z[None, :], bits), s, z
+
+
+def quantize_key_groups(k: np.ndarray, bits: int, G: int):
+    """Consecutive key groups [n*G][d] -> (codes [n*G][d], scale [n][d],
+    zero [n][d]); the same per-channel arithmetic as quantize_keys, for every
+    group at once."""
+    k = np.asarray(k, np.float64)
+    n, d = k.shape[0] // G, k.shape[1]
+    kg = k.reshape(n, G, d)
+    s, z = params(kg.min(axis=1), kg.max(axis=1), bits)
+    return codes(kg, s[:, None, :], z[:, None, :], bits).reshape(n * G, d), s, z
 
 
 def quantize_values(v: np.ndarray, bits: int):

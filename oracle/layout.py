@@ -6,7 +6,7 @@ dequantized in registers ("Quantification du KV-Cache : TurboQuant et l'etat de
 l'art en 2026", "TurboQuant : les cinq innovations", item 3 "Bit-packing
 dense") -- but not the order of codes inside the words.  Format v1 orders them
 for the decode kernel's tensor-core fragments; the order is a bijection, so it
-changes no value, only where a code sits.  the design doc carries the same table.
+changes no value, only where a code sits.
 
 Notation: a token block (TB) is 32 consecutive tokens; lane L in [0, 32) has
 gr = L >> 2 and tc = L & 3; every lane owns P = d*b/32 words of a TB's key

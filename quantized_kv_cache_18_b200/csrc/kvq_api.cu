@@ -1,0 +1,325 @@
+// Host side of the C ABI declared in include/kvq.h: argument validation, the
+// cache-buffer layout, host-side length counters, split planning and launches.
+// No call here allocates device memory; every computation runs in the kernels.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "kvq_internal.cuh"
+
+struct kvq_cache {
+  kvq_config cfg;
+  kvq_layout lay;
+  char* base;
+  int32_t seq_len;
+  int32_t tq;
+  int32_t r;
+  int32_t head;
+};
+
+namespace kvq {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+static uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+static bool config_ok(const kvq_config* c) {
+  if (!c) return false;
+  if (c->scheme != KVQ_KIVI) return false;   // the TurboQuant scheme is declared, built separately
+  if (!(c->bits == 2 || c->bits == 4)) return false;
+  if (!(c->group == 32 || c->group == 64)) return false;
+  if (!(c->head_dim == 64 || c->head_dim == 128)) return false;
+  if (c->residual < 0 || c->residual % c->group != 0) return false;
+  if (c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->num_q_heads % c->num_kv_heads != 0) return false;
+  const int g = c->num_q_heads / c->num_kv_heads;
+  if (!(g == 1 || g == 2 || g == 4 || g == 8)) return false;
+  if (c->batch <= 0 || c->max_seq <= 0) return false;
+  if ((int64_t)c->batch * c->num_kv_heads > 65535) return false;
+  if (!(c->dtype == KVQ_BF16 || c->dtype == KVQ_FP16)) return false;
+  return true;
+}
+
+static kvq_layout make_layout(const kvq_config* c) {
+  kvq_layout L;
+  std::memset(&L, 0, sizeof(L));
+  const uint64_t rows = (uint64_t)c->batch * c->num_kv_heads;
+  const uint64_t d = c->head_dim, G = c->group;
+  L.record_bytes = G * d * c->bits / 4 + 4 * d + 4 * G;
+  L.groups_per_row = c->max_seq > c->residual ? (uint64_t)(c->max_seq - c->residual) / G : 0;
+  L.ring_tokens = (uint64_t)c->residual + G;
+  L.records_offset = 0;
+  uint64_t off = align_up(rows * L.groups_per_row * L.record_bytes, 256);
+  L.window_offset = off;
+  off = align_up(off + rows * 2 * L.ring_tokens * d * 2, 256);
+  L.params_offset = off;
+  L.params_bytes = 0;
+  L.status_offset = off;
+  L.total_bytes = align_up(off + 16, 256);
+  return L;
+}
+
+static Geom make_geom(const kvq_cache* h) {
+  Geom g;
+  const kvq_config& c = h->cfg;
+  g.d = c.head_dim;
+  g.bits = c.bits;
+  g.G = c.group;
+  g.R = c.residual;
+  g.cap = c.residual + c.group;
+  g.B = c.batch;
+  g.Hkv = c.num_kv_heads;
+  g.Hq = c.num_q_heads;
+  g.g = c.num_q_heads / c.num_kv_heads;
+  g.dtype = c.dtype;
+  g.groups_per_row = (int64_t)h->lay.groups_per_row;
+  g.rec_bytes = (int64_t)h->lay.record_bytes;
+  g.tb_code_bytes = (int64_t)kTB * c.head_dim * c.bits / 8;
+  g.records = h->base + h->lay.records_offset;
+  g.window = reinterpret_cast<uint16_t*>(h->base + h->lay.window_offset);
+  g.status = reinterpret_cast<uint32_t*>(h->base + h->lay.status_offset);
+  return g;
+}
+
+// Split plan of a decode step: quantized groups in nq splits of gps groups,
+// window tokens in nw splits of kWindowChunk tokens.
+struct Plan {
+  int nq, gps, nw;
+};
+
+static Plan plan_decode(const kvq_config& c, int64_t n_groups, int r) {
+  Plan p{0, 1, 0};
+  const int64_t rows = (int64_t)c.batch * c.num_kv_heads;
+  const int64_t target = 4 * (int64_t)num_sms();
+  if (n_groups > 0) {
+    int64_t nq = (target + rows - 1) / rows;
+    if (nq < 1) nq = 1;
+    if (nq > n_groups) nq = n_groups;
+    const int64_t gps = (n_groups + nq - 1) / nq;
+    p.gps = (int)gps;
+    p.nq = (int)((n_groups + gps - 1) / gps);
+  }
+  p.nw = (r + kWindowChunk - 1) / kWindowChunk;
+  return p;
+}
+
+static int max_splits(const kvq_config& c, const kvq_layout& L) {
+  const int64_t rows = (int64_t)c.batch * c.num_kv_heads;
+  const int64_t target = 4 * (int64_t)num_sms();
+  int64_t nq = (target + rows - 1) / rows;
+  if (nq > (int64_t)L.groups_per_row) nq = (int64_t)L.groups_per_row;
+  const int64_t nw = ((int64_t)c.residual + c.group - 1 + kWindowChunk - 1) / kWindowChunk;
+  return (int)(nq + nw);
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+size_t kvq_cache_bytes(const kvq_config* cfg) {
+  if (!config_ok(cfg)) return 0;
+  return (size_t)make_layout(cfg).total_bytes;
+}
+
+size_t kvq_workspace_bytes(const kvq_config* cfg) {
+  if (!config_ok(cfg)) return 0;
+  const kvq_layout L = make_layout(cfg);
+  const int64_t rows = (int64_t)cfg->batch * cfg->num_kv_heads;
+  const int g = cfg->num_q_heads / cfg->num_kv_heads;
+  return (size_t)(rows * max_splits(*cfg, L) * g * (cfg->head_dim + 2) * sizeof(float));
+}
+
+kvq_status kvq_get_layout(const kvq_config* cfg, kvq_layout* out) {
+  if (!out) return KVQ_ERR_INVALID_ARG;
+  if (!config_ok(cfg)) return KVQ_ERR_UNSUPPORTED;
+  *out = make_layout(cfg);
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes, void* stream, kvq_cache** out) {
+  if (!cfg || !dev_buf || !out) return KVQ_ERR_INVALID_ARG;
+  if (!config_ok(cfg)) return KVQ_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(dev_buf) & 255u) != 0) return KVQ_ERR_INVALID_ARG;
+  const kvq_layout L = make_layout(cfg);
+  if (bytes < L.total_bytes) return KVQ_ERR_INVALID_ARG;
+  kvq_cache* h = new (std::nothrow) kvq_cache;
+  if (!h) return KVQ_ERR_INVALID_ARG;
+  h->cfg = *cfg;
+  h->lay = L;
+  h->base = static_cast<char*>(dev_buf);
+  h->seq_len = h->tq = h->r = h->head = 0;
+  launch_clear_status(reinterpret_cast<uint32_t*>(h->base + L.status_offset), (cudaStream_t)stream);
+  if (cudaGetLastError() != cudaSuccess) {
+    delete h;
+    return KVQ_ERR_CUDA;
+  }
+  *out = h;
+  return KVQ_OK;
+}
+
+kvq_status kvq_turbo_setup(kvq_cache* cache, const float* rot_gauss, const float* qjl_gauss, void* stream) {
+  (void)rot_gauss;
+  (void)qjl_gauss;
+  (void)stream;
+  if (!cache) return KVQ_ERR_INVALID_ARG;
+  return KVQ_ERR_UNSUPPORTED;
+}
+
+kvq_status kvq_quantize_prefill(kvq_cache* h, const void* k, const void* v, int32_t seq_len, void* stream) {
+  if (!h || !k || !v || seq_len < 0) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_INVALID_ARG;
+  if (h->seq_len != 0) return KVQ_ERR_INVALID_ARG;
+  if (seq_len > h->cfg.max_seq) return KVQ_ERR_CAPACITY;
+  const kvq_config& c = h->cfg;
+  const int32_t G = c.group, R = c.residual;
+  const int32_t tq = seq_len > R ? G * ((seq_len - R) / G) : 0;
+  const Geom g = make_geom(h);
+  cudaStream_t st = (cudaStream_t)stream;
+  QuantArgs a;
+  a.geom = g;
+  a.src_k = static_cast<const uint16_t*>(k);
+  a.src_v = static_cast<const uint16_t*>(v);
+  a.src_row_stride = (int64_t)seq_len * c.head_dim;
+  a.dst_group0 = 0;
+  a.n_groups = tq / G;
+  launch_kivi_quantize(a, st);
+  launch_window_copy(g, a.src_k, a.src_v, seq_len, tq, seq_len - tq, st);
+  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  h->seq_len = seq_len;
+  h->tq = tq;
+  h->r = seq_len - tq;
+  h->head = 0;
+  return KVQ_OK;
+}
+
+kvq_status kvq_append_token(kvq_cache* h, const void* k_new, const void* v_new, void* stream) {
+  if (!h || !k_new || !v_new) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
+  if (h->seq_len + 1 > h->cfg.max_seq) return KVQ_ERR_CAPACITY;
+  const kvq_config& c = h->cfg;
+  const int32_t G = c.group, R = c.residual, cap = R + G;
+  const Geom g = make_geom(h);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int slot = (h->head + h->r) % cap;
+  int32_t r = h->r + 1, head = h->head, tq = h->tq;
+  if (r == R + G && (uint64_t)(tq / G) >= h->lay.groups_per_row) return KVQ_ERR_CAPACITY;
+  launch_append(g, static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), slot, st);
+  if (r == R + G) {
+    QuantArgs a;
+    a.geom = g;
+    a.src_k = g.window + (int64_t)head * c.head_dim;
+    a.src_v = g.window + ((int64_t)cap + head) * c.head_dim;
+    a.src_row_stride = (int64_t)2 * cap * c.head_dim;
+    a.dst_group0 = tq / G;
+    a.n_groups = 1;
+    launch_kivi_quantize(a, st);
+    head = (head + G) % cap;
+    r -= G;
+    tq += G;
+  }
+  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  h->r = r;
+  h->head = head;
+  h->tq = tq;
+  h->seq_len += 1;
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention(const kvq_cache* h, const void* q, float* out, float softmax_scale, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!h || !q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
+  if (h->seq_len <= 0) return KVQ_ERR_INVALID_ARG;
+  if (!(std::isfinite(softmax_scale))) return KVQ_ERR_INVALID_ARG;
+  const kvq_config& c = h->cfg;
+  if (workspace_bytes < kvq_workspace_bytes(&c)) return KVQ_ERR_INVALID_ARG;
+  const Plan p = plan_decode(c, h->tq / c.group, h->r);
+  AttnArgs a;
+  a.geom = make_geom(h);
+  a.q = static_cast<const uint16_t*>(q);
+  a.out = out;
+  a.ws = static_cast<float*>(workspace);
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.n_groups = h->tq / c.group;
+  a.gps = p.gps;
+  a.nq = p.nq;
+  a.nw = p.nw;
+  a.r = h->r;
+  a.head = h->head;
+  launch_kivi_attention(a, (cudaStream_t)stream);
+  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
+kvq_status kvq_get_status(kvq_cache* h, uint32_t* bits, int32_t clear, void* stream) {
+  if (!h) return KVQ_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t v = 0;
+  uint32_t* dev = reinterpret_cast<uint32_t*>(h->base + h->lay.status_offset);
+  if (cudaMemcpyAsync(&v, dev, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (clear) launch_clear_status(dev, st);
+  if (bits) *bits = v;
+  return v ? KVQ_ERR_DEVICE_STATUS : KVQ_OK;
+}
+
+int32_t kvq_seq_len(const kvq_cache* h) { return h ? h->seq_len : -1; }
+int32_t kvq_quantized_len(const kvq_cache* h) { return h ? h->tq : -1; }
+int32_t kvq_window_len(const kvq_cache* h) { return h ? h->r : -1; }
+int32_t kvq_window_head(const kvq_cache* h) { return h ? h->head : -1; }
+
+kvq_status kvq_cache_set_state(kvq_cache* h, int32_t seq_len, int32_t quantized_len, int32_t window_head) {
+  if (!h) return KVQ_ERR_INVALID_ARG;
+  const kvq_config& c = h->cfg;
+  const int32_t G = c.group, cap = c.residual + c.group;
+  if (seq_len < 0 || quantized_len < 0 || quantized_len % G != 0 || window_head < 0 || window_head >= cap ||
+      window_head % G != 0)
+    return KVQ_ERR_INVALID_ARG;
+  const int32_t r = seq_len - quantized_len;
+  if (r < 0 || r >= cap) return KVQ_ERR_INVALID_ARG;
+  if (seq_len > c.max_seq || (uint64_t)(quantized_len / G) > h->lay.groups_per_row) return KVQ_ERR_CAPACITY;
+  h->seq_len = seq_len;
+  h->tq = quantized_len;
+  h->r = r;
+  h->head = window_head;
+  return KVQ_OK;
+}
+
+void kvq_cache_destroy(kvq_cache* h) { delete h; }
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "capacity exceeded";
+    case KVQ_ERR_CUDA: return "CUDA runtime error";
+    case KVQ_ERR_DEVICE_STATUS: return "device status word set";
+  }
+  return "unknown status";
+}
+
+uint64_t kvq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int32_t kvq_decode_splits(const kvq_cache* h) {
+  if (!h) return -1;
+  const Plan p = plan_decode(h->cfg, h->tq / h->cfg.group, h->r);
+  return p.nq + p.nw;
+}
+
+}  // extern "C"

@@ -1,0 +1,167 @@
+// Internal declarations shared by the libkvq CUDA sources (sm_100a only).
+//
+// Packed KIVI format v1 (one "group record" per G tokens of a (batch, kv head)
+// row).  A token block (TB) is 32 tokens; lane L of a warp has gr = L >> 2 and
+// tc = L & 3, the coordinates of the m16n8k16 mma.sync fragments.
+//
+//  key codes of a TB    pair (nt, kt, rho) of lane (gr, tc) = token 8nt+gr,
+//                       channels 16kt+8rho+2tc (+0 low half, +1 high half);
+//                       u = 2kt + rho
+//                       2-bit: j'=u&3, slot=nt*(d/32)+(u>>2), word=slot>>1, j=4(slot&1)+j'
+//                       4-bit: j'=u&1, slot=nt*(d/16)+(u>>1), word=slot>>1, j=2(slot&1)+j'
+//  value codes of a TB  pair (kt, nt, rho) of lane (gr, tc) = channel 8nt+gr,
+//                       tokens 16kt+8rho+2tc (+0 low, +1 high); u = 2kt + rho
+//                       2-bit: j'=u,   slot=nt,          word=slot>>1, j=4(slot&1)+j'
+//                       4-bit: j'=u&1, slot=2nt+(u>>1),  word=slot>>1, j=2(slot&1)+j'
+//  low code of pair j at bit b*j, high code at bit 16+b*j; word w of lane L at
+//  byte 16*(32*(w>>2)+L) + 4*(w&3) of the TB's code block.
+//  key meta   d fp16 scales, then d fp16 zeros; channel 16kt+8rho+2tc+e at
+//             position tc*(d/4)+4kt+2rho+e.
+//  value meta per TB, 32 x {fp16 scale, fp16 zero}; token 16kt+8rho+2tc+e at
+//             entry 8tc+4kt+2rho+e.
+//  record     [key TBs][value TBs][key scales][key zeros][value meta TBs]
+//
+// The format puts every pair a lane needs for one mma.sync B operand inside one
+// 32-bit word at the bit positions (b*j, 16+b*j), so a single LOP3 turns two
+// codes into the mantissas of an fp16x2 and one HFMA2 makes them exact small
+// integers.  A warp reads a TB's codes as 16-byte pieces, one per lane.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+constexpr int kTB = 32;         // tokens per token block
+constexpr int kWarpsAttn = 4;   // warps per decode-attention CTA
+constexpr int kWindowChunk = 128;  // window tokens per window CTA
+
+struct Geom {
+  int d, bits, G, R, cap, B, Hkv, Hq, g, dtype;
+  int64_t groups_per_row;   // record capacity of a row
+  int64_t rec_bytes;        // bytes of one group record
+  int64_t tb_code_bytes;    // bytes of one TB's key (or value) codes
+  char* records;            // [B][Hkv][groups_per_row][rec_bytes]
+  uint16_t* window;         // [B][Hkv][2][cap][d]
+  uint32_t* status;         // device status word
+};
+
+__host__ __device__ inline int64_t rec_kscale_off(const Geom& g) { return (int64_t)g.G * g.d * g.bits / 4; }
+__host__ __device__ inline int64_t rec_kzero_off(const Geom& g) { return rec_kscale_off(g) + 2 * g.d; }
+__host__ __device__ inline int64_t rec_vmeta_off(const Geom& g) { return rec_kscale_off(g) + 4 * g.d; }
+
+__host__ __device__ inline char* record_ptr(const Geom& g, int row, int64_t group) {
+  return g.records + ((int64_t)row * g.groups_per_row + group) * g.rec_bytes;
+}
+__host__ __device__ inline uint16_t* ring_ptr(const Geom& g, int row, int kv) {
+  return g.window + ((int64_t)row * 2 + kv) * g.cap * g.d;
+}
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// 16-bit input pattern -> float (exact).
+__device__ __forceinline__ float in16_to_float(uint16_t bits, int dtype) {
+  if (dtype == KVQ_BF16) return __uint_as_float((uint32_t)bits << 16);
+  return __half2float(__ushort_as_half(bits));
+}
+
+// Exact code decision: q = clamp(round_half_even((x - z) / s), 0, levels), by
+// comparing t = 2(x - z), carried as an error-free double sum hi + lo, with the
+// exact thresholds (2k + 1) s.  A double-precision estimate is corrected by
+// exact comparisons (at most a couple of steps each way).
+__device__ __forceinline__ bool t_above(double hi, double lo, double T) {
+  return hi > T || (hi == T && lo > 0.0);
+}
+__device__ __forceinline__ int exact_code(double x, double z, double s, double inv_s, int levels) {
+  if (!(s > 0.0)) return 0;
+  double hi = x - z;
+  double bb = hi - x;
+  double lo = (x - (hi - bb)) + (-z - bb);
+  hi *= 2.0;
+  lo *= 2.0;
+  double est = ceil((hi * inv_s - 1.0) * 0.5);
+  int k = est < 0.0 ? 0 : (est > (double)levels ? levels : (int)est);
+  // k must count the thresholds strictly below t
+  for (int it = 0; it < 4 && k > 0 && !t_above(hi, lo, (2.0 * k - 1.0) * s); ++it) --k;
+  for (int it = 0; it < 4 && k < levels && t_above(hi, lo, (2.0 * k + 1.0) * s); ++it) ++k;
+  if (k < levels && hi == (2.0 * k + 1.0) * s && lo == 0.0 && (k & 1)) ++k;
+  return k;
+}
+
+// Unpack one 32-bit code word into exact fp16x2 code values.
+// 2-bit: 8 pairs, pair j at bits (2j, 16+2j); 4-bit: 4 pairs at (4j, 16+4j).
+// (w & field) | 0x6400 is the fp16 1024 + code * 2^(b*j'), and one HFMA2
+// (x * 2^(-b*j') - 1024 * 2^(-b*j')) leaves the code, exactly.
+template <int BITS>
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t* out) {
+  constexpr int J = BITS == 2 ? 4 : 2;  // pairs per half word
+  constexpr uint32_t M = BITS == 2 ? 0x00030003u : 0x000F000Fu;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint32_t x = half ? (w >> 8) : w;
+#pragma unroll
+    for (int jp = 0; jp < J; ++jp) {
+      const uint32_t f = (x & (M << (BITS * jp))) | 0x64006400u;
+      const float sc = 1.0f / (float)(1u << (BITS * jp));
+      const __half2 s2 = __float2half2_rn(sc);
+      const __half2 c2 = __float2half2_rn(-1024.0f * sc);
+      out[half * J + jp] = h2_as_u32(__hfma2(u32_as_h2(f), s2, c2));
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernels (launchers in kvq_api.cu)
+struct QuantArgs {
+  Geom geom;
+  const uint16_t* src_k;   // token 0 of group `src_group0` of row 0
+  const uint16_t* src_v;
+  int64_t src_row_stride;  // elements between rows
+  int64_t dst_group0;      // first record index written
+  int n_groups;            // groups per row handled by this launch
+};
+
+struct AttnArgs {
+  Geom geom;
+  const uint16_t* q;       // [B][Hq][d]
+  float* out;              // [B][Hq][d]
+  float* ws;               // partials [rows][n_split][g][d + 2]
+  float scale_log2;        // softmax scale * log2(e)
+  int64_t n_groups;        // quantized groups per row (T_q / G)
+  int gps;                 // groups per quantized split
+  int nq;                  // quantized splits per row
+  int nw;                  // window splits per row
+  int r;                   // window tokens
+  int head;                // ring slot of the oldest window token
+};
+
+void launch_kivi_quantize(const QuantArgs& a, cudaStream_t st);
+void launch_window_copy(const Geom& g, const uint16_t* k, const uint16_t* v, int64_t seq_len, int64_t t0,
+                        int n, cudaStream_t st);
+void launch_append(const Geom& g, const uint16_t* k, const uint16_t* v, int slot, cudaStream_t st);
+void launch_kivi_attention(const AttnArgs& a, cudaStream_t st);
+void launch_clear_status(uint32_t* status, cudaStream_t st);
+
+int num_sms();
+void count_launch(int n = 1);
+
+}  // namespace kvq

@@ -219,6 +219,15 @@ def test_constant_group_gives_zero_codes():
     assert np.array_equal(kivi.dequant(c, s[None], z[None]), g)
 
 
+def test_group_batch_equals_single_groups():
+    rng = np.random.default_rng(12)
+    k = _rand_groups(rng, 5, 32, 16, "bf16").reshape(160, 16)
+    c, s, z = kivi.quantize_key_groups(k, 2, 32)
+    for i in range(5):
+        c1, s1, z1 = kivi.quantize_keys(k[32 * i:32 * (i + 1)], 2)
+        assert np.array_equal(c[32 * i:32 * (i + 1)], c1) and np.array_equal(s[i], s1) and np.array_equal(z[i], z1)
+
+
 def test_keys_per_channel_values_per_token():
     """Channel outliers blow up a per-token scale but not a per-channel one, and
     token outliers the reverse: the reason the pages give for the K/V split."""
