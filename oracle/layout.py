@@ -27,7 +27,9 @@ In a word, the low code of pair j sits at bit b*j and the high code at bit
 of the TB's code block, so a warp reads a block as 16-byte pieces, one per lane.
 
 Key metadata of a group: d fp16 scales then d fp16 zeros, channel
-c = 16 kt + 8 rho + 2 tc + e stored at position tc*(d/4) + 4 kt + 2 rho + e.
+c = 16 kt + 8 rho + 2 tc + e stored at position
+8 (4 (kt >> 1) + tc) + 4 (kt & 1) + 2 rho + e, so the lanes of one tc read 16
+consecutive bytes per k-tile pair and the four tc read adjacent chunks.
 Value metadata of a TB: 32 entries of 4 bytes (fp16 scale in the low half,
 fp16 zero in the high half); token t = 16 kt + 8 rho + 2 tc + e stored at
 entry 8 tc + 4 kt + 2 rho + e.
@@ -120,7 +122,7 @@ def key_meta_perm(d: int) -> np.ndarray:
         for kt in range(d // 16):
             for rho in range(2):
                 for e in range(2):
-                    pos[16 * kt + 8 * rho + 2 * tc + e] = tc * (d // 4) + 4 * kt + 2 * rho + e
+                    pos[16 * kt + 8 * rho + 2 * tc + e] = 8 * (4 * (kt >> 1) + tc) + 4 * (kt & 1) + 2 * rho + e
     assert sorted(pos.tolist()) == list(range(d))
     return pos
 

@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
   uint16_t* kzr = reinterpret_cast<uint16_t*>(rec + rec_kzero_off(gm));
   for (int c = tid; c < D; c += kQuantThreads) {
     const int kt = c >> 4, rho = (c >> 3) & 1, tc = (c >> 1) & 3, e = c & 1;
-    const int pos = tc * (D / 4) + 4 * kt + 2 * rho + e;
+    const int pos = 8 * (4 * (kt >> 1) + tc) + 4 * (kt & 1) + 2 * rho + e;
     ksc[pos] = k_sb[c];
     kzr[pos] = k_zb[c];
   }
@@ -225,7 +225,9 @@ __global__ void append_kernel(Geom g, const uint16_t* k, const uint16_t* v, int 
   }
 }
 
-__global__ void clear_status_kernel(uint32_t* status) { *status = 0; }
+__global__ void clear_words_kernel(uint32_t* words, int n) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) words[i] = 0u;
+}
 
 template <int BITS, int D, int G>
 void launch_q(const QuantArgs& a, cudaStream_t st) {
@@ -271,8 +273,8 @@ void launch_append(const Geom& g, const uint16_t* k, const uint16_t* v, int slot
   count_launch();
 }
 
-void launch_clear_status(uint32_t* status, cudaStream_t st) {
-  clear_status_kernel<<<1, 1, 0, st>>>(status);
+void launch_clear_words(uint32_t* words, int n, cudaStream_t st) {
+  clear_words_kernel<<<1, 256, 0, st>>>(words, n);
   count_launch();
 }
 

@@ -65,8 +65,8 @@ static kvq_layout make_layout(const kvq_config* c) {
   off = align_up(off + rows * 2 * L.ring_tokens * d * 2, 256);
   L.params_offset = off;
   L.params_bytes = 0;
-  L.status_offset = off;
-  L.total_bytes = align_up(off + 16, 256);
+  L.status_offset = off;               // status word, then one counter per row
+  L.total_bytes = align_up(off + 4 + 4 * rows, 256);
   return L;
 }
 
@@ -92,35 +92,21 @@ static Geom make_geom(const kvq_cache* h) {
   return g;
 }
 
-// Split plan of a decode step: quantized groups in nq splits of gps groups,
-// window tokens in nw splits of kWindowChunk tokens.
-struct Plan {
-  int nq, gps, nw;
-};
-
-static Plan plan_decode(const kvq_config& c, int64_t n_groups, int r) {
-  Plan p{0, 1, 0};
+// Decode launch size: one CTA per SM at most, and few enough that every CTA's
+// byte range holds at least one whole item (a group record or a window chunk
+// of 32 tokens), so each CTA between a row's first and last contributor has
+// work in that row.
+static int plan_ctas(const kvq_config& c, int64_t n_groups, int r) {
   const int64_t rows = (int64_t)c.batch * c.num_kv_heads;
-  const int64_t target = 4 * (int64_t)num_sms();
-  if (n_groups > 0) {
-    int64_t nq = (target + rows - 1) / rows;
-    if (nq < 1) nq = 1;
-    if (nq > n_groups) nq = n_groups;
-    const int64_t gps = (n_groups + nq - 1) / nq;
-    p.gps = (int)gps;
-    p.nq = (int)((n_groups + gps - 1) / gps);
-  }
-  p.nw = (r + kWindowChunk - 1) / kWindowChunk;
-  return p;
-}
-
-static int max_splits(const kvq_config& c, const kvq_layout& L) {
-  const int64_t rows = (int64_t)c.batch * c.num_kv_heads;
-  const int64_t target = 4 * (int64_t)num_sms();
-  int64_t nq = (target + rows - 1) / rows;
-  if (nq > (int64_t)L.groups_per_row) nq = (int64_t)L.groups_per_row;
-  const int64_t nw = ((int64_t)c.residual + c.group - 1 + kWindowChunk - 1) / kWindowChunk;
-  return (int)(nq + nw);
+  const int64_t rec = (int64_t)c.group * c.head_dim * c.bits / 4 + 4 * c.head_dim + 4 * c.group;
+  const int64_t tokb = 4 * (int64_t)c.head_dim;
+  const int64_t w_tot = rows * (n_groups * rec + (int64_t)r * tokb);
+  const int64_t w_max = r > 0 ? (rec > 32 * tokb ? rec : 32 * tokb) : rec;
+  int64_t n = w_tot / w_max;
+  const int64_t sms = num_sms();
+  if (n > sms) n = sms;
+  if (n < 1) n = 1;
+  return (int)n;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -138,10 +124,9 @@ size_t kvq_cache_bytes(const kvq_config* cfg) {
 
 size_t kvq_workspace_bytes(const kvq_config* cfg) {
   if (!config_ok(cfg)) return 0;
-  const kvq_layout L = make_layout(cfg);
   const int64_t rows = (int64_t)cfg->batch * cfg->num_kv_heads;
   const int g = cfg->num_q_heads / cfg->num_kv_heads;
-  return (size_t)(rows * max_splits(*cfg, L) * g * (cfg->head_dim + 2) * sizeof(float));
+  return (size_t)((rows + num_sms()) * g * (cfg->head_dim + 2) * sizeof(float));
 }
 
 kvq_status kvq_get_layout(const kvq_config* cfg, kvq_layout* out) {
@@ -163,7 +148,8 @@ kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes, vo
   h->lay = L;
   h->base = static_cast<char*>(dev_buf);
   h->seq_len = h->tq = h->r = h->head = 0;
-  launch_clear_status(reinterpret_cast<uint32_t*>(h->base + L.status_offset), (cudaStream_t)stream);
+  launch_clear_words(reinterpret_cast<uint32_t*>(h->base + L.status_offset),
+                     1 + cfg->batch * cfg->num_kv_heads, (cudaStream_t)stream);
   if (cudaGetLastError() != cudaSuccess) {
     delete h;
     return KVQ_ERR_CUDA;
@@ -248,17 +234,15 @@ kvq_status kvq_decode_attention(const kvq_cache* h, const void* q, float* out, f
   if (!(std::isfinite(softmax_scale))) return KVQ_ERR_INVALID_ARG;
   const kvq_config& c = h->cfg;
   if (workspace_bytes < kvq_workspace_bytes(&c)) return KVQ_ERR_INVALID_ARG;
-  const Plan p = plan_decode(c, h->tq / c.group, h->r);
   AttnArgs a;
   a.geom = make_geom(h);
   a.q = static_cast<const uint16_t*>(q);
   a.out = out;
   a.ws = static_cast<float*>(workspace);
+  a.counters = reinterpret_cast<unsigned*>(h->base + h->lay.status_offset) + 1;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.n_groups = h->tq / c.group;
-  a.gps = p.gps;
-  a.nq = p.nq;
-  a.nw = p.nw;
+  a.n_cta = plan_ctas(c, a.n_groups, h->r);
   a.r = h->r;
   a.head = h->head;
   launch_kivi_attention(a, (cudaStream_t)stream);
@@ -273,7 +257,7 @@ kvq_status kvq_get_status(kvq_cache* h, uint32_t* bits, int32_t clear, void* str
   uint32_t* dev = reinterpret_cast<uint32_t*>(h->base + h->lay.status_offset);
   if (cudaMemcpyAsync(&v, dev, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return KVQ_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return KVQ_ERR_CUDA;
-  if (clear) launch_clear_status(dev, st);
+  if (clear) launch_clear_words(dev, 1, st);
   if (bits) *bits = v;
   return v ? KVQ_ERR_DEVICE_STATUS : KVQ_OK;
 }
@@ -318,8 +302,7 @@ uint64_t kvq_launch_count(void) { return g_launches.load(std::memory_order_relax
 
 int32_t kvq_decode_splits(const kvq_cache* h) {
   if (!h) return -1;
-  const Plan p = plan_decode(h->cfg, h->tq / h->cfg.group, h->r);
-  return p.nq + p.nw;
+  return plan_ctas(h->cfg, h->tq / h->cfg.group, h->r);
 }
 
 }  // extern "C"

@@ -16,7 +16,8 @@
 //  low code of pair j at bit b*j, high code at bit 16+b*j; word w of lane L at
 //  byte 16*(32*(w>>2)+L) + 4*(w&3) of the TB's code block.
 //  key meta   d fp16 scales, then d fp16 zeros; channel 16kt+8rho+2tc+e at
-//             position tc*(d/4)+4kt+2rho+e.
+//             position 8(4(kt>>1)+tc) + 4(kt&1) + 2rho + e (one 16-byte chunk
+//             per (k-tile pair, tc), adjacent across tc).
 //  value meta per TB, 32 x {fp16 scale, fp16 zero}; token 16kt+8rho+2tc+e at
 //             entry 8tc+4kt+2rho+e.
 //  record     [key TBs][value TBs][key scales][key zeros][value meta TBs]
@@ -30,13 +31,11 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include "../../include/kvq.h"
+#include "kvq.h"
 
 namespace kvq {
 
 constexpr int kTB = 32;         // tokens per token block
-constexpr int kWarpsAttn = 4;   // warps per decode-attention CTA
-constexpr int kWindowChunk = 128;  // window tokens per window CTA
 
 struct Geom {
   int d, bits, G, R, cap, B, Hkv, Hq, g, dtype;
@@ -108,26 +107,54 @@ __device__ __forceinline__ int exact_code(double x, double z, double s, double i
   return k;
 }
 
-// Unpack one 32-bit code word into exact fp16x2 code values.
-// 2-bit: 8 pairs, pair j at bits (2j, 16+2j); 4-bit: 4 pairs at (4j, 16+4j).
-// (w & field) | 0x6400 is the fp16 1024 + code * 2^(b*j'), and one HFMA2
-// (x * 2^(-b*j') - 1024 * 2^(-b*j')) leaves the code, exactly.
+// Unpack one 32-bit code word into exact fp16x2 values.
+// 2-bit: 8 pairs, pair j at bits (2j, 16+2j); 4-bit: 4 pairs at (4j, 16+4j);
+// the upper four (two) pairs are read after shifting the word down by 8, so a
+// pair sits at position j' (0..3 for 2-bit, 0..1 for 4-bit) of its half word.
+// (w & field) | 0x6400 is the fp16 1024 + code * 2^(b*j'); subtracting 1024
+// leaves code * 2^(b*j'), an exact normal fp16 (at most 3*64 or 15*16).  The
+// factor 2^(b*j') is undone on the other mma operand, where it is an exact
+// power-of-two rescale (pos_comp).
+constexpr uint32_t kMagic = 0x64006400u;   // fp16x2 (1024, 1024)
+
+template <int BITS, int JP>
+__device__ __forceinline__ uint32_t unpack_pair(uint32_t x, uint32_t magic) {
+  constexpr uint32_t M = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << (BITS * JP);
+  uint32_t f, d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(f) : "r"(x), "n"(M), "r"(magic));   // (x & M) | magic
+  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(f), "r"(magic));
+  return d;
+}
+// One half word (already shifted down for the upper half): J pairs.
 template <int BITS>
-__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t* out) {
-  constexpr int J = BITS == 2 ? 4 : 2;  // pairs per half word
-  constexpr uint32_t M = BITS == 2 ? 0x00030003u : 0x000F000Fu;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const uint32_t x = half ? (w >> 8) : w;
-#pragma unroll
-    for (int jp = 0; jp < J; ++jp) {
-      const uint32_t f = (x & (M << (BITS * jp))) | 0x64006400u;
-      const float sc = 1.0f / (float)(1u << (BITS * jp));
-      const __half2 s2 = __float2half2_rn(sc);
-      const __half2 c2 = __float2half2_rn(-1024.0f * sc);
-      out[half * J + jp] = h2_as_u32(__hfma2(u32_as_h2(f), s2, c2));
-    }
+__device__ __forceinline__ void unpack_half(uint32_t x, uint32_t* out, uint32_t magic) {
+  out[0] = unpack_pair<BITS, 0>(x, magic);
+  out[1] = unpack_pair<BITS, 1>(x, magic);
+  if (BITS == 2) {
+    out[2] = unpack_pair<BITS, 2>(x, magic);
+    out[3] = unpack_pair<BITS, 3>(x, magic);
   }
+}
+template <int BITS>
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t* out, uint32_t magic) {
+  constexpr int J = BITS == 2 ? 4 : 2;
+  unpack_half<BITS>(w, out, magic);
+  unpack_half<BITS>(w >> 8, out + J, magic);
+}
+// 2^(-b*j'): the compensation of pair position j', as fp16x2 and as float
+__host__ __device__ constexpr uint32_t pos_comp(int bits, int jp) {
+  return bits == 2 ? (jp == 0 ? 0x3C003C00u : jp == 1 ? 0x34003400u : jp == 2 ? 0x2C002C00u : 0x24002400u)
+                   : (jp == 0 ? 0x3C003C00u : 0x2C002C00u);
+}
+__host__ __device__ constexpr float pos_comp_f(int bits, int jp) {
+  return bits == 2 ? (jp == 0 ? 1.f : jp == 1 ? 0.25f : jp == 2 ? 0.0625f : 0.015625f) : (jp == 0 ? 1.f : 0.0625f);
+}
+
+// 2^x with the MUFU instruction (inputs are <= 0 here; ftz is harmless)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ------------------------------------------------------------------ kernels (launchers in kvq_api.cu)
@@ -144,12 +171,11 @@ struct AttnArgs {
   Geom geom;
   const uint16_t* q;       // [B][Hq][d]
   float* out;              // [B][Hq][d]
-  float* ws;               // partials [rows][n_split][g][d + 2]
+  float* ws;               // partials [n_cta + rows][g][d + 2] (o[d], m, l)
+  unsigned* counters;      // [rows] arrival counters, zero between launches
   float scale_log2;        // softmax scale * log2(e)
   int64_t n_groups;        // quantized groups per row (T_q / G)
-  int gps;                 // groups per quantized split
-  int nq;                  // quantized splits per row
-  int nw;                  // window splits per row
+  int n_cta;               // CTAs of the launch (one per SM at most)
   int r;                   // window tokens
   int head;                // ring slot of the oldest window token
 };
@@ -159,7 +185,8 @@ void launch_window_copy(const Geom& g, const uint16_t* k, const uint16_t* v, int
                         int n, cudaStream_t st);
 void launch_append(const Geom& g, const uint16_t* k, const uint16_t* v, int slot, cudaStream_t st);
 void launch_kivi_attention(const AttnArgs& a, cudaStream_t st);
-void launch_clear_status(uint32_t* status, cudaStream_t st);
+void launch_clear_words(uint32_t* words, int n, cudaStream_t st);
+int decode_stage_bytes(int bits, int d, int G);
 
 int num_sms();
 void count_launch(int n = 1);

@@ -274,8 +274,11 @@ def test_layout_hand_worked_positions():
     # u 5 -> j' 1, slot 2, word 1, j 1 -> bit 4, byte 4
     off, bit = layout.key_code_map(128, 4)
     assert (off[0, 40], bit[0, 40]) == (4, 4)
-    # key meta: channel 19 = 16*1 + 0 + 2*1 + 1 -> tc 1 -> 32 + 4 + 0 + 1 = 37
-    assert layout.key_meta_perm(128)[19] == 37
+    # key meta: channel 19 = 16*1 + 0 + 2*1 + 1 -> kt 1, rho 0, tc 1, e 1
+    #   -> 8*(4*0 + 1) + 4*1 + 0 + 1 = 13
+    assert layout.key_meta_perm(128)[19] == 13
+    # channel 125 = 16*7 + 8 + 2*2 + 1 -> kt 7, rho 1, tc 2, e 1 -> 8*(12 + 2) + 4 + 2 + 1 = 119
+    assert layout.key_meta_perm(128)[125] == 119
     # value meta: token 27 = 16 + 8 + 2*1 + 1 -> tc 1 -> 8 + 4 + 2 + 1 = 15
     assert layout.value_meta_perm()[27] == 15
 
