@@ -191,6 +191,32 @@ kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, float* ou
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Decode attention that allocates nothing and needs no workspace argument.
+ * The pages have no counterpart for this call: it exists for callers that
+ * cannot allocate device memory -- for example a plugin running inside a
+ * serving engine that owns every device allocation and gives its plugins no
+ * allocator, or a serving loop that forbids allocator calls once it is
+ * running -- and so cannot provide the scratch space kvq_decode_attention
+ * takes.  It computes the same result as kvq_decode_attention, using a
+ * scratch array of KVQ_STATIC_WORKSPACE_BYTES compiled into this library
+ * (every GPU that loads the library holds that array until the process exits).
+ *   q, out, softmax_scale, stream  as for kvq_decode_attention.
+ * Errors: KVQ_ERR_CAPACITY, before anything is launched, if this cache's
+ * configuration needs more scratch than KVQ_STATIC_WORKSPACE_BYTES
+ * (kvq_workspace_bytes(cfg) > KVQ_STATIC_WORKSPACE_BYTES); otherwise the
+ * errors of kvq_decode_attention.
+ * The first call on a device looks up the array's device address for that
+ * device (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  All calls share the one array and it keeps
+ * the last call's contents (nothing in it needs to start at zero), so calls
+ * whose GPU work overlaps -- on two streams, or on two caches at once -- race
+ * and must be serialised by the caller.  No call allocates or frees memory.
+ */
+#define KVQ_STATIC_WORKSPACE_BYTES ((size_t)4 * 1024 * 1024)
+kvq_status kvq_decode_attention_static(const kvq_cache* cache, const void* q, float* out, float softmax_scale,
+                                       void* stream);
+
+/*
  * Synchronises `stream`, reads the device status word into *bits (may be
  * NULL) and returns KVQ_ERR_DEVICE_STATUS if any bit is set, else KVQ_OK.
  * `clear` != 0 also zeroes the word.

@@ -31,6 +31,8 @@
 // copies in flight before the CTA exits.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include <cuda_bf16.h>
 
 #include "kvq_internal.cuh"
@@ -806,3 +808,47 @@ void launch_kivi_attention(const AttnArgs& a, cudaStream_t st) {
 }
 
 }  // namespace kvq
+
+// ------------------------------------------------------------------ decode attention without caller scratch
+// For callers that cannot allocate device memory (see kvq_decode_attention_static
+// in kvq.h): the split-K partial states go to this fixed array instead of a
+// caller workspace.  The counters the kernel needs are in the cache buffer, so
+// nothing here has to start at zero.
+namespace kvq {
+static __device__ __align__(256) unsigned char g_static_ws[KVQ_STATIC_WORKSPACE_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mutex;
+void* g_static_ws_addr[kMaxDevices] = {};
+
+// Device address of g_static_ws on the current device.  The host-side name
+// g_static_ws is only a stand-in; the address is looked up once per device,
+// with that device current.
+kvq_status static_ws_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (g_static_ws_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress((void**)&ptr, g_static_ws) != cudaSuccess || ptr == nullptr) return KVQ_ERR_CUDA;
+    g_static_ws_addr[dev] = ptr;
+  }
+  *out = g_static_ws_addr[dev];
+  return KVQ_OK;
+}
+}  // namespace
+}  // namespace kvq
+
+extern "C" kvq_status kvq_decode_attention_static(const kvq_cache* cache, const void* q, float* out,
+                                                  float softmax_scale, void* stream) {
+  if (!cache) return KVQ_ERR_INVALID_ARG;
+  const size_t need = kvq::cache_workspace_bytes(cache);
+  if (need == 0) return KVQ_ERR_INVALID_ARG;
+  if (need > KVQ_STATIC_WORKSPACE_BYTES) return KVQ_ERR_CAPACITY;
+  void* ws = nullptr;
+  const kvq_status st = kvq::static_ws_address(&ws);
+  if (st != KVQ_OK) return st;
+  return kvq_decode_attention(cache, q, out, softmax_scale, ws, KVQ_STATIC_WORKSPACE_BYTES, stream);
+}

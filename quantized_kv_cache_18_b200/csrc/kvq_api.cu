@@ -113,6 +113,8 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 }  // namespace kvq
 
+size_t kvq::cache_workspace_bytes(const kvq_cache* h) { return h ? kvq_workspace_bytes(&h->cfg) : 0; }
+
 using namespace kvq;
 
 extern "C" {

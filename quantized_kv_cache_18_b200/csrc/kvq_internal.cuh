@@ -187,6 +187,7 @@ void launch_append(const Geom& g, const uint16_t* k, const uint16_t* v, int slot
 void launch_kivi_attention(const AttnArgs& a, cudaStream_t st);
 void launch_clear_words(uint32_t* words, int n, cudaStream_t st);
 int decode_stage_bytes(int bits, int d, int G);
+size_t cache_workspace_bytes(const kvq_cache* cache);   // kvq_workspace_bytes of the cache's config
 
 int num_sms();
 void count_launch(int n = 1);
