@@ -23,6 +23,7 @@ import ctypes
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -35,6 +36,21 @@ sys.path.insert(0, ROOT)
 METRIC = "quantized-KV decode attn: packed-KV GB/s (% of HBM peak), tokens/s"
 HBM_FALLBACK_GBS = 6650.0
 NORTH_STAR_HBM_GBS = 8000.0
+
+
+def _profiled_traffic(kernel: str, source: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when there is none or the kernel source has changed
+    since the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.md")
+    if not os.path.exists(p):
+        return None
+    m = re.search(r"traffic_bytes_per_launch=(\d+) source_sha256_16=([0-9a-f]+)", open(p).read())
+    if not m:
+        return None
+    src = open(os.path.join(ROOT, "quantized_kv_cache_18_b200", "csrc", source), "rb").read()
+    return int(m.group(1)) if hashlib.sha256(src).hexdigest()[:16] == m.group(2) else None
 
 
 def _peaks():
@@ -378,7 +394,8 @@ def main():
         "pct_of_north_star_hbm": round(100 * value / world / NORTH_STAR_HBM_GBS, 2),
         "roofline": {"bound": "hbm", "kernel": "kivi_decode_kernel (one launch per decode attention)",
                      "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": None,
+                     "frac": round(achieved / hbm, 4),
+                     "traffic": _profiled_traffic("kivi_decode_kernel", "kivi_attn.cu", w.name),
                      "bytes_per_launch": res["step_bytes_last"], "mean_launch_us": round(attn_mean * 1e3, 2)},
         "e2e": {"value": round(res["e2e_bytes"] * world / (res["e2e_ms"] * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
