@@ -172,7 +172,14 @@ def run_gpu(args, w, rank, world):
     probe = QuantizedKVCache(cfg, device=device)
     n_rep = max(2, math.ceil(3 * l2 / probe.nbytes) + 1)
     caches = [probe] + [QuantizedKVCache(cfg, device=device) for _ in range(n_rep - 1)]
+    turbo = None
+    if w.scheme == "turbo":
+        from quantized_kv_cache_18_b200 import workloads as W
+        turbo = (torch.from_numpy(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)).to(device),
+                 torch.from_numpy(W.gaussian_matrix(w, "qjl", w.qjl_dim, w.head_dim)).to(device))
     for c in caches:
+        if turbo is not None:
+            c.turbo_setup(*turbo)
         c.prefill(K, V)
     del K, V
     torch.cuda.synchronize()
@@ -274,6 +281,8 @@ def run_gpu(args, w, rank, world):
     e_caches = [QuantizedKVCache(cfg, device=device) for _ in range(n_rep)]
     K, V, _, _, _ = device_inputs(w, device, 1)
     for c in e_caches:
+        if turbo is not None:
+            c.turbo_setup(*turbo)
         c.prefill(K, V)
     del K, V
     torch.cuda.synchronize()
@@ -311,9 +320,15 @@ def oracle_sample(w, budget_s: float, steps: int = 1):
     import numpy as np
     from threadpoolctl import threadpool_info
     from oracle import attention as oatt
+    from oracle import turbo, turbo_cache
     from oracle.cache import KiviRow
     from oracle.numerics import decode16
     from quantized_kv_cache_18_b200 import workloads as W
+
+    if w.scheme == "turbo":
+        tq_params = (turbo.rotation(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)),
+                     W.gaussian_matrix(w, "qjl", w.qjl_dim, w.head_dim).astype(np.float64),
+                     *turbo.deployed_codebook(w.head_dim))
 
     t_total, bytes_total, rows = 0.0, 0, 0
     g = w.gqa
@@ -321,18 +336,25 @@ def oracle_sample(w, budget_s: float, steps: int = 1):
     wall0 = time.time()
     while t_total < budget_s and time.time() - wall0 < 3 * budget_s + 15:
         k, v = W.prefill_row(w, b, h)
-        row = KiviRow(w.head_dim, w.bits, w.group, w.residual, w.dtype)
+        if w.scheme == "turbo":
+            row = turbo_cache.TurboRow(w.head_dim, w.residual, w.dtype, *tq_params, G=w.group)
+            rec_bytes = turbo_cache.TB_BYTES
+        else:
+            row = KiviRow(w.head_dim, w.bits, w.group, w.residual, w.dtype)
+            rec_bytes = w.group * w.head_dim * w.bits // 4 + 4 * w.head_dim + 4 * w.group
         row.prefill(k, v)
         for s in range(1, steps + 1):
             kn, vn = W.decode_token(w, s)
             q = W.query(w, s)[b, h * g:(h + 1) * g]
             t = time.perf_counter()
             row.append(kn[b, h], vn[b, h])
-            Kd, Vd = row.dequantized()
-            oatt.attention(decode16(q, w.dtype), Kd, Vd, w.scale)
+            if w.scheme == "turbo":
+                row.attention(q, w.scale)
+            else:
+                Kd, Vd = row.dequantized()
+                oatt.attention(decode16(q, w.dtype), Kd, Vd, w.scale)
             t_total += time.perf_counter() - t
-            bytes_total += (row.tq // w.group) * (w.group * w.head_dim * w.bits // 4 + 4 * w.head_dim + 4 * w.group) \
-                + row.r * 4 * w.head_dim
+            bytes_total += (row.tq // w.group) * rec_bytes + row.r * 4 * w.head_dim
         rows += 1
         h += 1
         if h == w.num_kv_heads:
@@ -384,18 +406,26 @@ def main():
     hbm, peak_kind = _peaks()
     value = res["bytes"] * world / (res["ms"] * 1e-3) / 1e9
     attn_mean = statistics.mean(res["attn_ms"])
+    if w.scheme == "turbo":
+        kern, kern_src = "tq_decode_kernel", "tq_attn.cu"
+        kern_desc = "tq_decode_kernel (after tq_query_prep_kernel; both inside the timed attention call)"
+    else:
+        kern, kern_src = "kivi_decode_kernel", "kivi_attn.cu"
+        kern_desc = "kivi_decode_kernel (one launch per decode attention)"
     achieved = res["step_bytes_last"] / (attn_mean * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(res["ms"] / args.steps, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16 mma (fp32 accumulate) over int2/int4 codes",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": ("f16 mma (fp32 accumulate) over 3-bit codes + 1-bit sketch" if w.scheme == "turbo"
+                  else "f16 mma (fp32 accumulate) over int2/int4 codes"),
         "data": "synthetic", "config": cfg_desc,
         "tokens_per_s": round(w.batch * world * args.steps / (res["ms"] * 1e-3), 1),
         "pct_of_north_star_hbm": round(100 * value / world / NORTH_STAR_HBM_GBS, 2),
-        "roofline": {"bound": "hbm", "kernel": "kivi_decode_kernel (one launch per decode attention)",
+        "roofline": {"bound": "hbm", "kernel": kern_desc,
                      "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4),
-                     "traffic": _profiled_traffic("kivi_decode_kernel", "kivi_attn.cu", w.name),
+                     "traffic": _profiled_traffic(kern, kern_src, w.name),
                      "bytes_per_launch": res["step_bytes_last"], "mean_launch_us": round(attn_mean * 1e3, 2)},
         "e2e": {"value": round(res["e2e_bytes"] * world / (res["e2e_ms"] * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},

@@ -103,6 +103,19 @@ class QuantizedKVCache:
     def set_state(self, seq_len: int, quantized_len: int, window_head: int):
         L.check(self.lib.kvq_cache_set_state(self.handle, seq_len, quantized_len, window_head), "kvq_cache_set_state")
 
+    def turbo_setup(self, rot_gauss: torch.Tensor, qjl_gauss: torch.Tensor, stream=None):
+        """TurboQuant scheme: derive the rotation, codebook and sketch tables on
+        the device from two float32 N(0, 1) draws, [d][d] and [m][d]."""
+        c = self.cfg
+        for t, shape, what in ((rot_gauss, (c.head_dim, c.head_dim), "rot_gauss"),
+                               (qjl_gauss, (c.qjl_dim, c.head_dim), "qjl_gauss")):
+            if t.device != self.buf.device or t.dtype != torch.float32 or not t.is_contiguous():
+                raise ValueError(f"{what}: needs a contiguous float32 tensor on {self.buf.device}")
+            if tuple(t.shape) != shape:
+                raise ValueError(f"{what}: shape {tuple(t.shape)} != {shape}")
+        L.check(self.lib.kvq_turbo_setup(self.handle, _ptr(rot_gauss), _ptr(qjl_gauss), _stream_ptr(stream)),
+                "kvq_turbo_setup")
+
     # ------------------------------------------------------------------ the three calls
     def _check_16(self, t: torch.Tensor, shape, what: str):
         if t.device != self.buf.device or not t.is_contiguous() or t.element_size() != 2:
@@ -151,6 +164,11 @@ class QuantizedKVCache:
         n = c.batch * c.num_kv_heads * lay.groups_per_row * lay.record_bytes
         return self.buf[lay.records_offset:lay.records_offset + n].view(
             c.batch * c.num_kv_heads, lay.groups_per_row, lay.record_bytes)
+
+    def params_view(self) -> torch.Tensor:
+        """uint8 view of the TurboQuant parameter block (empty for KIVI)."""
+        lay = self.layout
+        return self.buf[lay.params_offset:lay.params_offset + lay.params_bytes]
 
     def ring_view(self) -> torch.Tensor:
         """[B*Hkv][2][ring_tokens][d] 16-bit patterns (as int16) of the residual rings."""

@@ -19,6 +19,7 @@ struct kvq_cache {
   int32_t tq;
   int32_t r;
   int32_t head;
+  bool tq_ready;   // TURBO: the parameter block holds the deployment constants
 };
 
 namespace kvq {
@@ -37,10 +38,15 @@ static uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
 static bool config_ok(const kvq_config* c) {
   if (!c) return false;
-  if (c->scheme != KVQ_KIVI) return false;   // the TurboQuant scheme is declared, built separately
-  if (!(c->bits == 2 || c->bits == 4)) return false;
-  if (!(c->group == 32 || c->group == 64)) return false;
-  if (!(c->head_dim == 64 || c->head_dim == 128)) return false;
+  if (c->scheme == KVQ_KIVI) {
+    if (!(c->bits == 2 || c->bits == 4)) return false;
+    if (!(c->group == 32 || c->group == 64)) return false;
+    if (!(c->head_dim == 64 || c->head_dim == 128)) return false;
+  } else if (c->scheme == KVQ_TURBO) {
+    if (c->bits != 3 || c->group != kTB || c->head_dim != kTqD || c->qjl_dim != kTqM) return false;
+  } else {
+    return false;
+  }
   if (c->residual < 0 || c->residual % c->group != 0) return false;
   if (c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->num_q_heads % c->num_kv_heads != 0) return false;
   const int g = c->num_q_heads / c->num_kv_heads;
@@ -56,7 +62,7 @@ static kvq_layout make_layout(const kvq_config* c) {
   std::memset(&L, 0, sizeof(L));
   const uint64_t rows = (uint64_t)c->batch * c->num_kv_heads;
   const uint64_t d = c->head_dim, G = c->group;
-  L.record_bytes = G * d * c->bits / 4 + 4 * d + 4 * G;
+  L.record_bytes = c->scheme == KVQ_TURBO ? (uint64_t)kTqTbBytes : G * d * c->bits / 4 + 4 * d + 4 * G;
   L.groups_per_row = c->max_seq > c->residual ? (uint64_t)(c->max_seq - c->residual) / G : 0;
   L.ring_tokens = (uint64_t)c->residual + G;
   L.records_offset = 0;
@@ -64,7 +70,8 @@ static kvq_layout make_layout(const kvq_config* c) {
   L.window_offset = off;
   off = align_up(off + rows * 2 * L.ring_tokens * d * 2, 256);
   L.params_offset = off;
-  L.params_bytes = 0;
+  L.params_bytes = c->scheme == KVQ_TURBO ? (uint64_t)kTqParamBytes : 0;
+  off = align_up(off + L.params_bytes, 256);
   L.status_offset = off;               // status word, then one counter per row
   L.total_bytes = align_up(off + 4 + 4 * rows, 256);
   return L;
@@ -73,6 +80,7 @@ static kvq_layout make_layout(const kvq_config* c) {
 static Geom make_geom(const kvq_cache* h) {
   Geom g;
   const kvq_config& c = h->cfg;
+  g.scheme = c.scheme;
   g.d = c.head_dim;
   g.bits = c.bits;
   g.G = c.group;
@@ -85,10 +93,11 @@ static Geom make_geom(const kvq_cache* h) {
   g.dtype = c.dtype;
   g.groups_per_row = (int64_t)h->lay.groups_per_row;
   g.rec_bytes = (int64_t)h->lay.record_bytes;
-  g.tb_code_bytes = (int64_t)kTB * c.head_dim * c.bits / 8;
+  g.tb_code_bytes = c.scheme == KVQ_TURBO ? (int64_t)(kTqVCodes - kTqKCodes) : (int64_t)kTB * c.head_dim * c.bits / 8;
   g.records = h->base + h->lay.records_offset;
   g.window = reinterpret_cast<uint16_t*>(h->base + h->lay.window_offset);
   g.status = reinterpret_cast<uint32_t*>(h->base + h->lay.status_offset);
+  g.params = reinterpret_cast<unsigned char*>(h->base + h->lay.params_offset);
   return g;
 }
 
@@ -98,7 +107,8 @@ static Geom make_geom(const kvq_cache* h) {
 // work in that row.
 static int plan_ctas(const kvq_config& c, int64_t n_groups, int r) {
   const int64_t rows = (int64_t)c.batch * c.num_kv_heads;
-  const int64_t rec = (int64_t)c.group * c.head_dim * c.bits / 4 + 4 * c.head_dim + 4 * c.group;
+  const int64_t rec = c.scheme == KVQ_TURBO ? (int64_t)kTqTbBytes
+                                             : (int64_t)c.group * c.head_dim * c.bits / 4 + 4 * c.head_dim + 4 * c.group;
   const int64_t tokb = 4 * (int64_t)c.head_dim;
   const int64_t w_tot = rows * (n_groups * rec + (int64_t)r * tokb);
   const int64_t w_max = r > 0 ? (rec > 32 * tokb ? rec : 32 * tokb) : rec;
@@ -124,10 +134,18 @@ size_t kvq_cache_bytes(const kvq_config* cfg) {
   return (size_t)make_layout(cfg).total_bytes;
 }
 
+// KIVI: partial states, (rows + SMs) slots of g x (d + 2) floats.  TURBO: the
+// rotated query fragments of every row, then (2 rows + SMs) partial slots (a
+// row's token blocks and window chunks give separate partials).
+static size_t tq_qprep_bytes(const kvq_config* cfg) {
+  return (size_t)cfg->batch * cfg->num_kv_heads * kTqQPrepBytes;
+}
 size_t kvq_workspace_bytes(const kvq_config* cfg) {
   if (!config_ok(cfg)) return 0;
   const int64_t rows = (int64_t)cfg->batch * cfg->num_kv_heads;
   const int g = cfg->num_q_heads / cfg->num_kv_heads;
+  if (cfg->scheme == KVQ_TURBO)
+    return tq_qprep_bytes(cfg) + (size_t)((2 * rows + num_sms()) * g * (cfg->head_dim + 2) * sizeof(float));
   return (size_t)((rows + num_sms()) * g * (cfg->head_dim + 2) * sizeof(float));
 }
 
@@ -150,6 +168,7 @@ kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes, vo
   h->lay = L;
   h->base = static_cast<char*>(dev_buf);
   h->seq_len = h->tq = h->r = h->head = 0;
+  h->tq_ready = false;
   launch_clear_words(reinterpret_cast<uint32_t*>(h->base + L.status_offset),
                      1 + cfg->batch * cfg->num_kv_heads, (cudaStream_t)stream);
   if (cudaGetLastError() != cudaSuccess) {
@@ -160,18 +179,22 @@ kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes, vo
   return KVQ_OK;
 }
 
-kvq_status kvq_turbo_setup(kvq_cache* cache, const float* rot_gauss, const float* qjl_gauss, void* stream) {
-  (void)rot_gauss;
-  (void)qjl_gauss;
-  (void)stream;
-  if (!cache) return KVQ_ERR_INVALID_ARG;
-  return KVQ_ERR_UNSUPPORTED;
+kvq_status kvq_turbo_setup(kvq_cache* h, const float* rot_gauss, const float* qjl_gauss, void* stream) {
+  if (!h || !rot_gauss || !qjl_gauss) return KVQ_ERR_INVALID_ARG;
+  if (h->cfg.scheme != KVQ_TURBO) return KVQ_ERR_UNSUPPORTED;
+  if (!aligned16(rot_gauss) || !aligned16(qjl_gauss)) return KVQ_ERR_INVALID_ARG;
+  if (h->seq_len != 0) return KVQ_ERR_INVALID_ARG;
+  launch_turbo_setup(make_geom(h), rot_gauss, qjl_gauss, (cudaStream_t)stream);
+  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  h->tq_ready = true;
+  return KVQ_OK;
 }
 
 kvq_status kvq_quantize_prefill(kvq_cache* h, const void* k, const void* v, int32_t seq_len, void* stream) {
   if (!h || !k || !v || seq_len < 0) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_INVALID_ARG;
   if (h->seq_len != 0) return KVQ_ERR_INVALID_ARG;
+  if (h->cfg.scheme == KVQ_TURBO && !h->tq_ready) return KVQ_ERR_INVALID_ARG;
   if (seq_len > h->cfg.max_seq) return KVQ_ERR_CAPACITY;
   const kvq_config& c = h->cfg;
   const int32_t G = c.group, R = c.residual;
@@ -185,7 +208,8 @@ kvq_status kvq_quantize_prefill(kvq_cache* h, const void* k, const void* v, int3
   a.src_row_stride = (int64_t)seq_len * c.head_dim;
   a.dst_group0 = 0;
   a.n_groups = tq / G;
-  launch_kivi_quantize(a, st);
+  if (c.scheme == KVQ_TURBO) launch_tq_quantize(a, st);
+  else launch_kivi_quantize(a, st);
   launch_window_copy(g, a.src_k, a.src_v, seq_len, tq, seq_len - tq, st);
   if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
   h->seq_len = seq_len;
@@ -199,6 +223,7 @@ kvq_status kvq_append_token(kvq_cache* h, const void* k_new, const void* v_new, 
   if (!h || !k_new || !v_new) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
   if (h->seq_len + 1 > h->cfg.max_seq) return KVQ_ERR_CAPACITY;
+  if (h->cfg.scheme == KVQ_TURBO && !h->tq_ready) return KVQ_ERR_INVALID_ARG;
   const kvq_config& c = h->cfg;
   const int32_t G = c.group, R = c.residual, cap = R + G;
   const Geom g = make_geom(h);
@@ -215,7 +240,8 @@ kvq_status kvq_append_token(kvq_cache* h, const void* k_new, const void* v_new, 
     a.src_row_stride = (int64_t)2 * cap * c.head_dim;
     a.dst_group0 = tq / G;
     a.n_groups = 1;
-    launch_kivi_quantize(a, st);
+    if (c.scheme == KVQ_TURBO) launch_tq_quantize(a, st);
+    else launch_kivi_quantize(a, st);
     head = (head + G) % cap;
     r -= G;
     tq += G;
@@ -236,18 +262,32 @@ kvq_status kvq_decode_attention(const kvq_cache* h, const void* q, float* out, f
   if (!(std::isfinite(softmax_scale))) return KVQ_ERR_INVALID_ARG;
   const kvq_config& c = h->cfg;
   if (workspace_bytes < kvq_workspace_bytes(&c)) return KVQ_ERR_INVALID_ARG;
+  if (c.scheme == KVQ_TURBO && !h->tq_ready) return KVQ_ERR_INVALID_ARG;
   AttnArgs a;
   a.geom = make_geom(h);
   a.q = static_cast<const uint16_t*>(q);
   a.out = out;
   a.ws = static_cast<float*>(workspace);
+  a.qprep = nullptr;
+  a.qjl_c = 0.f;
+  if (c.scheme == KVQ_TURBO) {
+    unsigned char* qp = static_cast<unsigned char*>(workspace);
+    a.qprep = qp;
+    a.ws = reinterpret_cast<float*>(qp + tq_qprep_bytes(&c));
+    a.qjl_c = (float)(std::sqrt(3.14159265358979323846 / 2.0) / c.qjl_dim);
+  }
   a.counters = reinterpret_cast<unsigned*>(h->base + h->lay.status_offset) + 1;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.n_groups = h->tq / c.group;
   a.n_cta = plan_ctas(c, a.n_groups, h->r);
   a.r = h->r;
   a.head = h->head;
-  launch_kivi_attention(a, (cudaStream_t)stream);
+  if (c.scheme == KVQ_TURBO) {
+    launch_tq_query_prep(a.geom, a.q, const_cast<unsigned char*>(a.qprep), (cudaStream_t)stream);
+    launch_tq_attention(a, (cudaStream_t)stream);
+  } else {
+    launch_kivi_attention(a, (cudaStream_t)stream);
+  }
   if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
   return KVQ_OK;
 }
@@ -283,6 +323,7 @@ kvq_status kvq_cache_set_state(kvq_cache* h, int32_t seq_len, int32_t quantized_
   h->tq = quantized_len;
   h->r = r;
   h->head = window_head;
+  h->tq_ready = true;   // TURBO: the restored buffer carries its parameter block
   return KVQ_OK;
 }
 

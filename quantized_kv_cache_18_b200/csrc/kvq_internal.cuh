@@ -38,14 +38,51 @@ namespace kvq {
 constexpr int kTB = 32;         // tokens per token block
 
 struct Geom {
-  int d, bits, G, R, cap, B, Hkv, Hq, g, dtype;
+  int scheme, d, bits, G, R, cap, B, Hkv, Hq, g, dtype;
   int64_t groups_per_row;   // record capacity of a row
   int64_t rec_bytes;        // bytes of one group record
   int64_t tb_code_bytes;    // bytes of one TB's key (or value) codes
   char* records;            // [B][Hkv][groups_per_row][rec_bytes]
   uint16_t* window;         // [B][Hkv][2][cap][d]
   uint32_t* status;         // device status word
+  unsigned char* params;    // TURBO: deployment constants (kTq* offsets)
 };
+
+// ------------------------------------------------------------------ TurboQuant-style format (head_dim = m = 128)
+// Token block (32 tokens of one row), kTqTbBytes bytes:
+//   [key codes 1664][value codes 1664][key sign bits 512][key meta 128][value meta 64]
+// Codes: the two 3-bit codes of a fragment pair form the 6-bit index lo + 8 hi;
+// five indices fill a 32-bit word (bits 6f..6f+5).  Lane L owns 64 pairs per
+// code block, slot s in word s / 5, field s % 5; words 0..11 of lane L sit at
+// byte 16 (32 (w >> 2) + L) + 4 (w & 3) and word 12 at 1536 + 4 L, so word q of
+// the block (in that order) is at byte 4 q.
+//   key pair   (nt, kt, rho), slot 16 nt + 2 kt + rho: token 8 nt + gr,
+//              coordinates 16 kt + 8 rho + 2 tc (lo) and + 1 (hi)
+//   value pair (kt, nt, rho), slot 32 kt + 2 nt + rho: coordinate 8 nt + gr,
+//              tokens 16 kt + 8 rho + 2 tc (lo) and + 1 (hi)
+// Sign bits of the key sketch: pair (nt, kt, rho) of lane L (token 8 nt + gr,
+// sketch rows 16 kt + 8 rho + 2 tc and + 1) in word nt of the lane's 16-byte
+// piece at byte 16 L, bits 2 kt + rho (lo) and 16 + 2 kt + rho (hi).
+// Meta: token 16 kt + 8 rho + 2 tc + e at entry 8 tc + 4 kt + 2 rho + e; keys
+// as (fp16 norm, fp16 gamma) words, values as fp16 norms.
+constexpr int kTqD = 128;
+constexpr int kTqM = 128;
+constexpr int kTqTbBytes = 4032;
+constexpr int kTqKCodes = 0;
+constexpr int kTqVCodes = 1664;
+constexpr int kTqSigns = 3328;
+constexpr int kTqKMeta = 3840;
+constexpr int kTqVMeta = 3968;
+// Parameter block (inside the cache buffer, written by kvq_turbo_setup):
+constexpr int kTqPi = 0;                      // float [d][d], Pi[i][j] (y = Pi u)
+constexpr int kTqPiT = kTqPi + kTqD * kTqD * 4;    // float [d][d], transpose of Pi
+constexpr int kTqST = kTqPiT + kTqD * kTqD * 4;    // float [d][m], transpose of S
+constexpr int kTqLevels = kTqST + kTqD * kTqM * 4; // float [8] codebook levels
+constexpr int kTqThr = kTqLevels + 32;             // float [8] thresholds (7 used, [7] = +inf)
+constexpr int kTqLevels16 = kTqThr + 32;           // fp16 [8] levels
+constexpr int kTqLut = kTqLevels + 128;            // uint32 [64]: fp16x2 (level[lo], level[hi]) of index lo + 8 hi
+constexpr int kTqParamBytes = kTqLut + 256;
+constexpr int kTqQPrepBytes = 2 * (kTqD / 16) * 32 * 16;   // rotated query fragments of one row
 
 __host__ __device__ inline int64_t rec_kscale_off(const Geom& g) { return (int64_t)g.G * g.d * g.bits / 4; }
 __host__ __device__ inline int64_t rec_kzero_off(const Geom& g) { return rec_kscale_off(g) + 2 * g.d; }
@@ -169,6 +206,8 @@ struct QuantArgs {
 
 struct AttnArgs {
   Geom geom;
+  const unsigned char* qprep;   // TURBO: [rows][kTqQPrepBytes] query fragments
+  float qjl_c;                  // TURBO: sqrt(pi / 2) / m
   const uint16_t* q;       // [B][Hq][d]
   float* out;              // [B][Hq][d]
   float* ws;               // partials [n_cta + rows][g][d + 2] (o[d], m, l)
@@ -186,6 +225,10 @@ void launch_window_copy(const Geom& g, const uint16_t* k, const uint16_t* v, int
 void launch_append(const Geom& g, const uint16_t* k, const uint16_t* v, int slot, cudaStream_t st);
 void launch_kivi_attention(const AttnArgs& a, cudaStream_t st);
 void launch_clear_words(uint32_t* words, int n, cudaStream_t st);
+void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_gauss, cudaStream_t st);
+void launch_tq_quantize(const QuantArgs& a, cudaStream_t st);
+void launch_tq_query_prep(const Geom& g, const uint16_t* q, unsigned char* qprep, cudaStream_t st);
+void launch_tq_attention(const AttnArgs& a, cudaStream_t st);
 int decode_stage_bytes(int bits, int d, int G);
 size_t cache_workspace_bytes(const kvq_cache* cache);   // kvq_workspace_bytes of the cache's config
 

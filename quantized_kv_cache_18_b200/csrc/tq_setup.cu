@@ -1,0 +1,271 @@
+// TurboQuant-style deployment constants and the per-step query rotation.
+//
+// The rotation Pi is a random orthogonal matrix: the Q factor of the QR
+// decomposition of a seeded N(0, 1) draw, with the sign of each column fixed so
+// that diag(R) > 0 ("Quantification du KV-Cache : TurboQuant et l'etat de l'art
+// en 2026", "TurboQuant : les cinq innovations", item 1; zubnet.ai survey,
+// "Famille deux ...").  Each rotated coordinate then has the law N(0, 1/d), and
+// the scalar quantizer is the 8-level Lloyd-Max quantizer of that law, fixed at
+// deployment (same page, item 2): levels are the Lloyd-Max levels of N(0, 1)
+// scaled by 1/sqrt(d) and stored in fp16, thresholds are the midpoints of
+// adjacent levels.  The QJL projection S is the caller's N(0, 1) draw as is.
+//
+// turbo_setup_kernel   one CTA: Householder QR in fp64 in shared memory, the
+//                      Lloyd-Max fixed point in fp64, then the fp32 tables.
+// tq_query_prep_kernel one CTA per (batch, kv head): q' = Pi q and q'' = S q'
+//                      for the row's query heads, split into fp16 hi + lo and
+//                      stored in the A-fragment order of the decode kernel.
+#include <cuda_runtime.h>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+namespace {
+
+constexpr int kSetupThreads = 256;
+
+__device__ __forceinline__ double warp_sum_d(double x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// A (column-major, A[j * D + i] = element (i, j)) is factored in place: column
+// k keeps the Householder vector v_k on rows k..D-1 (v_k[k] included), tau[k] =
+// 2 / (v_k . v_k) (0 for an identity step) and rdiag[k] = R[k][k].
+__global__ void __launch_bounds__(kSetupThreads, 1)
+    turbo_setup_kernel(const float* __restrict__ rot_gauss, const float* __restrict__ qjl_gauss,
+                       unsigned char* __restrict__ params, uint32_t* status) {
+  constexpr int D = kTqD, M = kTqM;
+  extern __shared__ __align__(16) double A[];   // [D][D]
+  __shared__ double tau[D], rdiag[D];
+  __shared__ uint32_t s_flags;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int NW = kSetupThreads / 32;
+  if (tid == 0) s_flags = 0;
+  __syncthreads();
+
+  uint32_t flags = 0;
+  for (int e = tid; e < D * D; e += kSetupThreads) {
+    const int i = e / D, j = e - i * D;
+    const float g = rot_gauss[e];   // row-major [i][j]
+    if (!isfinite(g)) flags |= KVQ_DEV_NONFINITE_INPUT;
+    A[j * D + i] = (double)g;
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- Householder QR
+  for (int k = 0; k < D; ++k) {
+    if (warp == 0) {
+      double s = 0.0;
+      for (int i = k + lane; i < D; i += 32) s += A[k * D + i] * A[k * D + i];
+      s = warp_sum_d(s);
+      if (lane == 0) {
+        const double x0 = A[k * D + k];
+        const double nrm = sqrt(s);
+        if (nrm == 0.0) {
+          tau[k] = 0.0;
+          rdiag[k] = 0.0;
+        } else {
+          const double alpha = x0 >= 0.0 ? -nrm : nrm;   // reflect x onto alpha e_1, away from x
+          A[k * D + k] = x0 - alpha;                      // v = x - alpha e_1
+          tau[k] = 1.0 / (nrm * (nrm + fabs(x0)));        // 2 / (v . v)
+          rdiag[k] = alpha;
+        }
+      }
+    }
+    __syncthreads();
+    const double tk = tau[k];
+    if (tk != 0.0) {
+      for (int j = k + 1 + warp; j < D; j += NW) {
+        double dot = 0.0;
+        for (int i = k + lane; i < D; i += 32) dot += A[k * D + i] * A[j * D + i];
+        const double f = tk * warp_sum_d(dot);
+        for (int i = k + lane; i < D; i += 32) A[j * D + i] -= f * A[k * D + i];
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---------------------------------------------------------------- Q = H_0 H_1 ... H_{D-1}, column by column
+  float* Pi = reinterpret_cast<float*>(params + kTqPi);
+  float* PiT = reinterpret_cast<float*>(params + kTqPiT);
+  for (int j = warp; j < D; j += NW) {
+    double x[D / 32];
+#pragma unroll
+    for (int r = 0; r < D / 32; ++r) x[r] = (lane + 32 * r == j) ? 1.0 : 0.0;
+    // H_k e_j = e_j for k > j (v_k vanishes above row k)
+    for (int k = j; k >= 0; --k) {
+      const double tk = tau[k];
+      if (tk == 0.0) continue;
+      double dot = 0.0;
+#pragma unroll
+      for (int r = 0; r < D / 32; ++r) {
+        const int i = lane + 32 * r;
+        if (i >= k) dot += A[k * D + i] * x[r];
+      }
+      const double f = tk * warp_sum_d(dot);
+#pragma unroll
+      for (int r = 0; r < D / 32; ++r) {
+        const int i = lane + 32 * r;
+        if (i >= k) x[r] -= f * A[k * D + i];
+      }
+    }
+    const double sg = rdiag[j] < 0.0 ? -1.0 : 1.0;   // diag(R) > 0 after the sign fix (0 counts as +)
+#pragma unroll
+    for (int r = 0; r < D / 32; ++r) {
+      const int i = lane + 32 * r;
+      const float v = (float)(sg * x[r]);
+      Pi[i * D + j] = v;
+      PiT[j * D + i] = v;
+    }
+  }
+
+  // ---------------------------------------------------------------- S^T
+  float* ST = reinterpret_cast<float*>(params + kTqST);
+  for (int e = tid; e < M * D; e += kSetupThreads) {
+    const int i = e / D, j = e - i * D;   // S row-major [i][j]
+    const float g = qjl_gauss[e];
+    if (!isfinite(g)) flags |= KVQ_DEV_NONFINITE_INPUT;
+    ST[j * M + i] = g;
+  }
+
+  // ---------------------------------------------------------------- Lloyd-Max for N(0, 1), 8 levels
+  // Alternate: thresholds = midpoints of the levels, levels = conditional
+  // means of their cells, E[X | a < X < b] = (phi(a) - phi(b)) / (Phi(b) - Phi(a)),
+  // from levels evenly spaced on [-2, 2] until no level moves by 1e-15.
+  if (warp == 0) {
+    const double inv_sqrt_2pi = 1.0 / sqrt(2.0 * 3.14159265358979323846);
+    const int l = lane & 7;
+    double c = l == 7 ? 2.0 : -2.0 + (double)l * (4.0 / 7.0);
+    for (int it = 0; it < 10000; ++it) {
+      const double cm = __shfl_up_sync(0xffffffffu, c, 1, 8);
+      const double cp = __shfl_down_sync(0xffffffffu, c, 1, 8);
+      const double lo = l == 0 ? -INFINITY : 0.5 * (c + cm);
+      const double hi = l == 7 ? INFINITY : 0.5 * (cp + c);
+      const double plo = l == 0 ? 0.0 : exp(-0.5 * lo * lo) * inv_sqrt_2pi;
+      const double phi_hi = l == 7 ? 0.0 : exp(-0.5 * hi * hi) * inv_sqrt_2pi;
+      const double mass = normcdf(hi) - normcdf(lo);
+      const double nc = (plo - phi_hi) / mass;
+      double diff = fabs(nc - c);
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) diff = fmax(diff, __shfl_xor_sync(0xffffffffu, diff, o, 8));
+      c = nc;
+      if (diff < 1e-15) break;
+    }
+    // deployed: fp16 levels of N(0, 1/d); midpoints are exact in fp32
+    const __half h = __double2half(c / sqrt((double)D));
+    const float lv = __half2float(h);
+    const float lv_next = __shfl_down_sync(0xffffffffu, lv, 1, 8);
+    float* levels = reinterpret_cast<float*>(params + kTqLevels);
+    float* thr = reinterpret_cast<float*>(params + kTqThr);
+    uint16_t* lv16 = reinterpret_cast<uint16_t*>(params + kTqLevels16);
+    if (lane < 8) {
+      levels[l] = lv;
+      lv16[l] = __half_as_ushort(h);
+      thr[l] = l < 7 ? 0.5f * (lv + lv_next) : INFINITY;
+    }
+    const uint16_t h_lo = __shfl_sync(0xffffffffu, __half_as_ushort(h), lane & 7);
+    const uint16_t h_hi = __shfl_sync(0xffffffffu, __half_as_ushort(h), (lane >> 3) & 7);
+    uint32_t* lut = reinterpret_cast<uint32_t*>(params + kTqLut);
+    // lanes 0..31 write indices 0..31 (hi = lane >> 3 in 0..3), then 32..63
+    lut[lane] = (uint32_t)h_lo | ((uint32_t)h_hi << 16);
+    const uint16_t h_hi2 = __shfl_sync(0xffffffffu, __half_as_ushort(h), 4 + ((lane >> 3) & 3));
+    lut[32 + lane] = (uint32_t)h_lo | ((uint32_t)h_hi2 << 16);
+  }
+  if (flags) atomicOr(&s_flags, flags);
+  __syncthreads();
+  if (tid == 0 && s_flags) atomicOr(status, s_flags);
+}
+
+// ---------------------------------------------------------------- query rotation
+constexpr int kPrepThreads = 256;
+
+__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
+  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+__global__ void __launch_bounds__(kPrepThreads)
+    tq_query_prep_kernel(Geom gm, const uint16_t* __restrict__ q, unsigned char* __restrict__ qprep) {
+  constexpr int D = kTqD, M = kTqM;
+  __shared__ float qf[8][D];    // raw q of the row's heads
+  __shared__ float qr[8][D];    // Pi q
+  __shared__ float qs[8][M];    // S Pi q
+  const int row = blockIdx.x;
+  const int b = row / gm.Hkv, hkv = row - b * gm.Hkv;
+  const int g = gm.g;
+  const int tid = threadIdx.x;
+  const uint16_t* qrow = q + ((int64_t)b * gm.Hq + (int64_t)hkv * g) * D;
+  for (int e = tid; e < 8 * D; e += kPrepThreads) {
+    const int h = e / D;
+    qf[h][e - h * D] = h < g ? in16_to_float(qrow[e], gm.dtype) : 0.f;
+  }
+  __syncthreads();
+  const float* PiT = reinterpret_cast<const float*>(gm.params + kTqPiT);
+  const float* ST = reinterpret_cast<const float*>(gm.params + kTqST);
+  const int i = tid & (D - 1), h0 = tid / D;   // two head slots per column
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < D; ++j) {
+      const float w = __ldg(PiT + j * D + i);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = fmaf(w, qf[h0 + 2 * u][j], acc[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) qr[h0 + 2 * u][i] = acc[u];
+  }
+  __syncthreads();
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < D; ++j) {
+      const float w = __ldg(ST + j * M + i);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = fmaf(w, qr[h0 + 2 * u][j], acc[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) qs[h0 + 2 * u][i] = acc[u];
+  }
+  __syncthreads();
+  // fragments: [vector (q', q'')][kt][lane] uint4 =
+  //   {hi(gr, c0..c0+1), lo(gr, c0..c0+1), hi(gr, c0+8..c0+9), lo(gr, c0+8..c0+9)}, c0 = 16 kt + 2 tc
+  uint4* out = reinterpret_cast<uint4*>(qprep + (int64_t)row * kTqQPrepBytes);
+  for (int e = tid; e < 2 * (D / 16) * 32; e += kPrepThreads) {
+    const int vec = e / ((D / 16) * 32);
+    const int kt = (e / 32) % (D / 16);
+    const int lane = e & 31;
+    const int gr = lane >> 2, tc = lane & 3;
+    const float* src = vec == 0 ? qr[gr] : qs[gr];
+    uint32_t w[4];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int c = 16 * kt + 8 * half + 2 * tc;
+      const float x0 = src[c], x1 = src[c + 1];
+      const __half h0v = __float2half_rn(x0), h1v = __float2half_rn(x1);
+      const __half l0 = __float2half_rn(x0 - __half2float(h0v)), l1 = __float2half_rn(x1 - __half2float(h1v));
+      w[2 * half] = pack_h2(h0v, h1v);
+      w[2 * half + 1] = pack_h2(l0, l1);
+    }
+    out[e] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+}  // namespace
+
+void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_gauss, cudaStream_t st) {
+  const int smem = kTqD * kTqD * (int)sizeof(double);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(turbo_setup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    attr_set = true;
+  }
+  turbo_setup_kernel<<<1, kSetupThreads, smem, st>>>(rot_gauss, qjl_gauss, g.params, g.status);
+  count_launch(1);
+}
+
+void launch_tq_query_prep(const Geom& g, const uint16_t* q, unsigned char* qprep, cudaStream_t st) {
+  tq_query_prep_kernel<<<g.B * g.Hkv, kPrepThreads, 0, st>>>(g, q, qprep);
+  count_launch(1);
+}
+
+}  // namespace kvq

@@ -103,3 +103,31 @@ def test_status_strings(lib):
 
 def test_launch_counter_starts_without_device_work(lib):
     assert lib.kvq_launch_count() >= 0
+
+
+def test_turbo_layout(lib):
+    """TurboQuant-style cache: 4032-byte token blocks (3-bit codes of keys and
+    values, 128 sketch bits, fp16 norms and gammas), a parameter block for the
+    rotation, its transpose, the sketch and the codebook."""
+    w = WORKLOADS["tq"]
+    cfg = config_from_workload(w)
+    lay = L.KvqLayout()
+    assert lib.kvq_get_layout(ctypes.byref(cfg), ctypes.byref(lay)) == L.KVQ_OK
+    rows = w.batch * w.num_kv_heads
+    assert lay.record_bytes == 4032 == 2 * 1664 + 512 + 128 + 64
+    assert lay.groups_per_row == (w.max_seq - w.residual) // 32
+    assert lay.params_bytes == 3 * 128 * 128 * 4 + 128 + 256
+    assert lay.params_offset % 256 == 0 and lay.params_offset >= lay.window_offset + rows * 2 * lay.ring_tokens * 256
+    assert lay.status_offset >= lay.params_offset + lay.params_bytes
+    assert lib.kvq_cache_bytes(ctypes.byref(cfg)) == lay.total_bytes
+    # rotated query fragments (8 KiB per row) + (2 rows + SMs) partial slots
+    ws = lib.kvq_workspace_bytes(ctypes.byref(cfg))
+    g = w.gqa
+    assert ws >= rows * 8192 + 2 * rows * g * 130 * 4
+
+
+@pytest.mark.parametrize("field,value", [("bits", 2), ("group", 64), ("head_dim", 64), ("qjl_dim", 64)])
+def test_unsupported_turbo_configs_are_rejected(lib, field, value):
+    cfg = config_from_workload(WORKLOADS["tq"])
+    setattr(cfg, field, value)
+    assert lib.kvq_cache_bytes(ctypes.byref(cfg)) == 0
