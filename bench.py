@@ -116,15 +116,37 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- ranks
+# Weak scaling: every rank owns an independent batch of sequences (its own
+# seeded inputs and caches); there is no exchange on the data path.  The only
+# collectives are the barriers around the timed region and these reductions.
+def rank_seed(w, rank: int) -> int:
+    return 1000 + w.seed + 7919 * rank
+
+
+def combine_ranks(ms: float, units: float, world: int, device) -> tuple:
+    """(max of ms over ranks, sum of units over ranks)."""
+    if world == 1:
+        return ms, units
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
 # ---------------------------------------------------------------- inputs on the device
-def device_inputs(w, device, steps_total):
-    """Seeded synthetic inputs with the workload's recipe, drawn on the GPU
-    (standard normal, K outlier channels x20, 2% of V tokens per batch row x10)."""
+def device_inputs(w, device, steps_total, rank: int = 0):
+    """Seeded synthetic inputs with the workload's recipe, drawn on the device
+    (standard normal, K outlier channels x20, 2% of V tokens per batch row x10);
+    each rank draws its own batch."""
     import torch
     from quantized_kv_cache_18_b200 import workloads as W
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
     g = torch.Generator(device=device)
-    g.manual_seed(1000 + w.seed)
+    g.manual_seed(rank_seed(w, rank))
     shape = (w.batch, w.num_kv_heads, w.seq_len, w.head_dim)
     ch = torch.as_tensor(W.k_outlier_channels(w), device=device)
     K = torch.randn(shape, generator=g, device=device)
@@ -167,7 +189,7 @@ def run_gpu(args, w, rank, world):
     steps_total = args.warmup + args.steps
     max_seq = w.seq_len + steps_total + 1
     cfg = config_from_workload(w, max_seq)
-    K, V, q, kn, vn = device_inputs(w, device, steps_total)
+    K, V, q, kn, vn = device_inputs(w, device, steps_total, rank)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     probe = QuantizedKVCache(cfg, device=device)
     n_rep = max(2, math.ceil(3 * l2 / probe.nbytes) + 1)
@@ -266,10 +288,7 @@ def run_gpu(args, w, rank, world):
     for c in caches:
         if c.status():
             raise RuntimeError("device status word set during the bench")
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms, total_bytes = combine_ranks(ms, total_bytes, world, device)
 
     # end-to-end through the public API with host buffers: H2D of the step's
     # inputs from pinned memory, append + attention, D2H of the output
@@ -279,7 +298,7 @@ def run_gpu(args, w, rank, world):
     h_out = torch.empty((args.steps,) + tuple(out.shape), dtype=torch.float32).pin_memory()
     d_q, d_kn, d_vn = torch.empty_like(q[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
     e_caches = [QuantizedKVCache(cfg, device=device) for _ in range(n_rep)]
-    K, V, _, _, _ = device_inputs(w, device, 1)
+    K, V, _, _, _ = device_inputs(w, device, 1, rank)
     for c in e_caches:
         if turbo is not None:
             c.turbo_setup(*turbo)
@@ -301,10 +320,7 @@ def run_gpu(args, w, rank, world):
     e1.record(stream)
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms, e_bytes = combine_ranks(e_ms, e_bytes, world, device)
 
     res = dict(ms=ms, bytes=total_bytes, attn_ms=attn_ms, launches=launches, clocks=clk.summary(),
                e2e_ms=e_ms, e2e_bytes=e_bytes, n_rep=n_rep, splits=caches[0].decode_splits,
@@ -404,7 +420,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_gpu(args, w, rank, world)
     hbm, peak_kind = _peaks()
-    value = res["bytes"] * world / (res["ms"] * 1e-3) / 1e9
+    value = res["bytes"] / (res["ms"] * 1e-3) / 1e9          # all ranks' bytes / max time
     attn_mean = statistics.mean(res["attn_ms"])
     if w.scheme == "turbo":
         kern, kern_src = "tq_decode_kernel", "tq_attn.cu"
@@ -427,7 +443,7 @@ def main():
                      "frac": round(achieved / hbm, 4),
                      "traffic": _profiled_traffic(kern, kern_src, w.name),
                      "bytes_per_launch": res["step_bytes_last"], "mean_launch_us": round(attn_mean * 1e3, 2)},
-        "e2e": {"value": round(res["e2e_bytes"] * world / (res["e2e_ms"] * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "e2e": {"value": round(res["e2e_bytes"] / (res["e2e_ms"] * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
         "gpu_launches": res["launches"], "clocks": res["clocks"], "replicas": res["n_rep"],
         "decode_splits": res["splits"],

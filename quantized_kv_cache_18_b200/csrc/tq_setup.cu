@@ -189,6 +189,7 @@ __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
 __global__ void __launch_bounds__(kPrepThreads)
     tq_query_prep_kernel(Geom gm, const uint16_t* __restrict__ q, unsigned char* __restrict__ qprep) {
   constexpr int D = kTqD, M = kTqM;
+  extern __shared__ __align__(16) float sW[];   // [D][D]: Pi^T, then S^T
   __shared__ float qf[8][D];    // raw q of the row's heads
   __shared__ float qr[8][D];    // Pi q
   __shared__ float qs[8][M];    // S Pi q
@@ -197,18 +198,28 @@ __global__ void __launch_bounds__(kPrepThreads)
   const int g = gm.g;
   const int tid = threadIdx.x;
   const uint16_t* qrow = q + ((int64_t)b * gm.Hq + (int64_t)hkv * g) * D;
+  // the whole matrix is requested at once (16 x 16-byte loads per thread), so
+  // its latency is paid once rather than once per row of the product
+  auto stage = [&](int off) {
+    const uint4* src = reinterpret_cast<const uint4*>(gm.params + off);
+    uint4 v[D * D / 4 / kPrepThreads];
+#pragma unroll
+    for (int k = 0; k < D * D / 4 / kPrepThreads; ++k) v[k] = __ldg(src + tid + k * kPrepThreads);
+#pragma unroll
+    for (int k = 0; k < D * D / 4 / kPrepThreads; ++k) reinterpret_cast<uint4*>(sW)[tid + k * kPrepThreads] = v[k];
+  };
+  stage(kTqPiT);
   for (int e = tid; e < 8 * D; e += kPrepThreads) {
     const int h = e / D;
     qf[h][e - h * D] = h < g ? in16_to_float(qrow[e], gm.dtype) : 0.f;
   }
   __syncthreads();
-  const float* PiT = reinterpret_cast<const float*>(gm.params + kTqPiT);
-  const float* ST = reinterpret_cast<const float*>(gm.params + kTqST);
   const int i = tid & (D - 1), h0 = tid / D;   // two head slots per column
   {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
     for (int j = 0; j < D; ++j) {
-      const float w = __ldg(PiT + j * D + i);
+      const float w = sW[j * D + i];
 #pragma unroll
       for (int u = 0; u < 4; ++u) acc[u] = fmaf(w, qf[h0 + 2 * u][j], acc[u]);
     }
@@ -216,10 +227,13 @@ __global__ void __launch_bounds__(kPrepThreads)
     for (int u = 0; u < 4; ++u) qr[h0 + 2 * u][i] = acc[u];
   }
   __syncthreads();
+  stage(kTqST);
+  __syncthreads();
   {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
     for (int j = 0; j < D; ++j) {
-      const float w = __ldg(ST + j * M + i);
+      const float w = sW[j * M + i];
 #pragma unroll
       for (int u = 0; u < 4; ++u) acc[u] = fmaf(w, qr[h0 + 2 * u][j], acc[u]);
     }
@@ -264,7 +278,13 @@ void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_
 }
 
 void launch_tq_query_prep(const Geom& g, const uint16_t* q, unsigned char* qprep, cudaStream_t st) {
-  tq_query_prep_kernel<<<g.B * g.Hkv, kPrepThreads, 0, st>>>(g, q, qprep);
+  const int smem = kTqD * kTqD * (int)sizeof(float);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(tq_query_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    attr_set = true;
+  }
+  tq_query_prep_kernel<<<g.B * g.Hkv, kPrepThreads, smem, st>>>(g, q, qprep);
   count_launch(1);
 }
 
