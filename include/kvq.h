@@ -242,6 +242,10 @@ void kvq_cache_destroy(kvq_cache* cache);
 
 const char* kvq_status_string(kvq_status s);
 
+/* Message of the CUDA error behind the calling thread's last KVQ_ERR_CUDA
+ * ("no error" if there was none); a static string, never freed. */
+const char* kvq_cuda_error_string(void);
+
 /* Kernels this library has launched since it was loaded (all handles). */
 uint64_t kvq_launch_count(void);
 

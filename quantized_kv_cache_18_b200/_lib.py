@@ -46,6 +46,7 @@ _SIGS = {
     "kvq_cache_destroy": (None, [_P]),
     "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvq_launch_count": (ctypes.c_uint64, []),
+    "kvq_cuda_error_string": (ctypes.c_char_p, []),
     "kvq_decode_splits": (ctypes.c_int32, [_P]),
 }
 
@@ -76,6 +77,8 @@ class KvqError(RuntimeError):
     def __init__(self, code: int, what: str = ""):
         self.code = code
         msg = load().kvq_status_string(code).decode()
+        if code == KVQ_ERR_CUDA:
+            msg += ": " + load().kvq_cuda_error_string().decode()
         super().__init__(f"{what}: {msg} (status {code})" if what else msg)
 
 

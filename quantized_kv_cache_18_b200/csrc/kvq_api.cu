@@ -25,6 +25,18 @@ struct kvq_cache {
 namespace kvq {
 
 static std::atomic<uint64_t> g_launches{0};
+static thread_local const char* g_cuda_error = "no error";
+
+// Records the failing CUDA call's message for kvq_cuda_error_string.
+static kvq_status cuda_failed(cudaError_t e) {
+  g_cuda_error = cudaGetErrorString(e);
+  return KVQ_ERR_CUDA;
+}
+// Checks the launches just enqueued (launch-configuration errors surface here).
+static kvq_status check_launch() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KVQ_OK : cuda_failed(e);
+}
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 int num_sms() {
@@ -171,7 +183,7 @@ kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes, vo
   h->tq_ready = false;
   launch_clear_words(reinterpret_cast<uint32_t*>(h->base + L.status_offset),
                      1 + cfg->batch * cfg->num_kv_heads, (cudaStream_t)stream);
-  if (cudaGetLastError() != cudaSuccess) {
+  if (check_launch() != KVQ_OK) {
     delete h;
     return KVQ_ERR_CUDA;
   }
@@ -185,7 +197,7 @@ kvq_status kvq_turbo_setup(kvq_cache* h, const float* rot_gauss, const float* qj
   if (!aligned16(rot_gauss) || !aligned16(qjl_gauss)) return KVQ_ERR_INVALID_ARG;
   if (h->seq_len != 0) return KVQ_ERR_INVALID_ARG;
   launch_turbo_setup(make_geom(h), rot_gauss, qjl_gauss, (cudaStream_t)stream);
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  if (check_launch() != KVQ_OK) return KVQ_ERR_CUDA;
   h->tq_ready = true;
   return KVQ_OK;
 }
@@ -211,7 +223,7 @@ kvq_status kvq_quantize_prefill(kvq_cache* h, const void* k, const void* v, int3
   if (c.scheme == KVQ_TURBO) launch_tq_quantize(a, st);
   else launch_kivi_quantize(a, st);
   launch_window_copy(g, a.src_k, a.src_v, seq_len, tq, seq_len - tq, st);
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  if (check_launch() != KVQ_OK) return KVQ_ERR_CUDA;
   h->seq_len = seq_len;
   h->tq = tq;
   h->r = seq_len - tq;
@@ -246,7 +258,7 @@ kvq_status kvq_append_token(kvq_cache* h, const void* k_new, const void* v_new, 
     r -= G;
     tq += G;
   }
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  if (check_launch() != KVQ_OK) return KVQ_ERR_CUDA;
   h->r = r;
   h->head = head;
   h->tq = tq;
@@ -288,7 +300,7 @@ kvq_status kvq_decode_attention(const kvq_cache* h, const void* q, float* out, f
   } else {
     launch_kivi_attention(a, (cudaStream_t)stream);
   }
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  if (check_launch() != KVQ_OK) return KVQ_ERR_CUDA;
   return KVQ_OK;
 }
 
@@ -297,8 +309,9 @@ kvq_status kvq_get_status(kvq_cache* h, uint32_t* bits, int32_t clear, void* str
   cudaStream_t st = (cudaStream_t)stream;
   uint32_t v = 0;
   uint32_t* dev = reinterpret_cast<uint32_t*>(h->base + h->lay.status_offset);
-  if (cudaMemcpyAsync(&v, dev, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return KVQ_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return KVQ_ERR_CUDA;
+  cudaError_t e = cudaMemcpyAsync(&v, dev, sizeof(v), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_failed(e);
   if (clear) launch_clear_words(dev, 1, st);
   if (bits) *bits = v;
   return v ? KVQ_ERR_DEVICE_STATUS : KVQ_OK;
@@ -342,6 +355,8 @@ const char* kvq_status_string(kvq_status s) {
 }
 
 uint64_t kvq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* kvq_cuda_error_string(void) { return g_cuda_error; }
 
 int32_t kvq_decode_splits(const kvq_cache* h) {
   if (!h) return -1;
