@@ -79,6 +79,11 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t* r, const void* row_addr) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(smem_u32(row_addr)));
 }
+__device__ __forceinline__ void ldsm_x2_t(uint32_t* r, const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(smem_u32(row_addr)));
+}
 // two floats -> packed pair in the input's 16-bit format
 __device__ __forceinline__ uint32_t pack2_in16(float lo, float hi, int dtype) {
   if (dtype == KVQ_FP16) return h2_as_u32(__floats2half2_rn(lo, hi));

@@ -7,16 +7,22 @@
 //   score_t = sum_c q_c (z_c + s_c code_tc) = beta + sum_c (q_c s_c) code_tc
 //   o_c     = sum_t p_t (zv_t + sv_t code_tc) = sum_t p_t zv_t + sum_t (p_t sv_t) code_tc
 // q~ = q (.) s (per group) and p~ = p (.) sv (per token) are split into fp16
-// hi + lo parts held in the two 8-row halves of the m16 A operand, so one GQA
-// group of up to 8 query heads runs both contractions on mma.sync with exact
-// small-integer fp16 codes as the B operand.
+// hi + lo parts, and both contractions run on mma.sync with the exact
+// small-integer fp16 codes as the other operand.  Two formulations:
+//   head-major (GQA groups of 5..8 heads): the heads' hi | lo parts are the
+//     two 8-row halves of the m16 A operand and the codes are the B operand;
+//   token-major (groups of 1..4 heads): the codes are the A operand (tokens,
+//     resp. channels, are M) and the heads' hi | lo parts are the 8 columns
+//     of B, which halves the mma count and the accumulators of the
+//     head-major form for such groups and leaves room for 12 consumer warps.
 //
 // Structure (one CTA per SM, one launch per decode step):
 //   warp 0      producer: 1-D bulk copies (cp.async.bulk, no multicast) of whole
 //               group records / window rows into a ring of shared-memory stages
 //   warp 1      prep: the zero-point term beta = q . z for every group of a stage
-//               in one batched mma (columns = groups)
-//   warps 2..9  consumers: one 32-token block per warp per stage, online softmax
+//               in batched mma's (columns = groups)
+//   warps 2..   consumers (8 head-major, 12 token-major): one 32-token block
+//               per warp per stage, online softmax
 // Work: the (row, item) sequence -- a row's groups then its 32-token window
 // chunks -- is cut into equal-byte ranges, one per CTA.  A CTA writes one
 // partial (m, l, o) per row it touches; the last CTA to finish a row (atomic
@@ -41,34 +47,46 @@ namespace kvq {
 
 namespace {
 
-constexpr int kConsumers = 8;
-constexpr int kThreads = (kConsumers + 2) * 32;
 constexpr int kWinTok = 32;                     // tokens per window item
 
-__device__ __forceinline__ void consumer_bar() { named_bar_sync<kConsumers * 32>(); }
+template <int NC>
+__device__ __forceinline__ void consumer_bar() { named_bar_sync<NC * 32>(); }
 
-template <int BITS, int D, int G>
+// NC consumer warps; TR selects the token-major formulation (GQA groups of up
+// to 4 heads, see the kernel comment), which runs 12 consumers.
+template <int BITS, int D, int G, bool TR>
 struct K {
+  static constexpr int NC = TR ? 12 : 8;                         // consumer warps
+  static constexpr int THREADS = (NC + 3) * 32;                  // + producer, prep, merge warps
+  static constexpr int HS = TR ? 4 : 8;                          // heads per warp state
+  static constexpr int DP = D + 4;                               // partial row (o[D], m, l, pad): 16-byte multiple
   static constexpr int NTB = G / kTB;
-  static constexpr int SG = kConsumers / NTB;                    // groups per stage
+  static constexpr int SG = NC / NTB;                            // groups per stage
   static constexpr int REC = G * D * BITS / 4 + 4 * D + 4 * G;   // record bytes
   static constexpr int TBC = kTB * D * BITS / 8;                 // TB code bytes
   static constexpr int WROW = D * 2;                             // window row in shared memory
   static constexpr int WINB = kWinTok * WROW * 2;                 // window item bytes in a stage (K + V)
   static constexpr int STAGE = ((SG * REC > WINB ? SG * REC : WINB) + 127) / 128 * 128;
-  static constexpr int NST = STAGE > 48 * 1024 ? 3 : 4;          // pipeline depth
+  // warp-state buffer (floats): m[NC][HS], l[NC][HS], a flag word and padding,
+  // then o[NC][HS][D]
+  static constexpr int SO = (2 * NC * HS + 1 + 3) / 4 * 4;
+  static constexpr int SBUF_F = SO + NC * HS * D;
+  static constexpr int FIXED = 2 * SBUF_F * 4 + (TR ? NC * 512 : 0) + 2 * 8 * D * 2 + 8 * 8 + 16;
+  static constexpr int NST_FIT = (227 * 1024 - FIXED) / (STAGE + SG * 8 * 4 + 3 * 8);
+  static constexpr int NST = (STAGE > 48 * 1024 ? 3 : 4) < NST_FIT ? (STAGE > 48 * 1024 ? 3 : 4) : NST_FIT;
   static constexpr int KSOFF = G * D * BITS / 4;
   static constexpr int KZOFF = KSOFF + 2 * D;
   static constexpr int VMOFF = KSOFF + 4 * D;
   // shared memory map (bytes)
   static constexpr int OFF_BETA = NST * STAGE;
-  static constexpr int OFF_M = OFF_BETA + NST * SG * 8 * 4;
-  static constexpr int OFF_L = OFF_M + kConsumers * 8 * 4;
-  static constexpr int OFF_O = OFF_L + kConsumers * 8 * 4;
-  static constexpr int OFF_Q = OFF_O + kConsumers * 8 * D * 4;   // q ring: 2 slots x raw 16-bit q of 8 heads
+  static constexpr int OFF_S = OFF_BETA + NST * SG * 8 * 4;      // two warp-state buffers
+  static constexpr int OFF_PW = OFF_S + 2 * SBUF_F * 4;          // per-warp P tile (TR): 32 tokens x 8 fp16
+  static constexpr int OFF_Q = OFF_PW + (TR ? NC * 512 : 0);     // q ring: 2 slots x raw 16-bit q of 8 heads
   static constexpr int OFF_BAR = OFF_Q + 2 * 8 * D * 2;
-  static constexpr int OFF_FLAG = OFF_BAR + (3 * NST + 4) * 8;
+  static constexpr int OFF_FLAG = OFF_BAR + (3 * NST + 8) * 8;
   static constexpr int SMEM = OFF_FLAG + 16;
+  static_assert(NST >= 2, "decode pipeline needs two stages");
+  static_assert(SMEM <= 227 * 1024, "decode kernel shared memory exceeds the per-block limit");
 };
 
 // ------------------------------------------------------------------ work partition
@@ -130,9 +148,12 @@ __device__ __forceinline__ void for_each_chunk(const Part& P, int64_t i0, int64_
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int BITS, int D, int G>
-__global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
-  using C = K<BITS, D, G>;
+// The token-major variant runs 15 warps, the head-major one 11.  Declaring
+// 512 (384) threads caps them at 128 (168) registers, so that the four (three)
+// warps one SM sub-partition holds fit its 16,384-entry register file.
+template <int BITS, int D, int G, bool TR>
+__global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs a) {
+  using C = K<BITS, D, G, TR>;
   constexpr int P = D * BITS / 32;
   constexpr int J = BITS == 2 ? 4 : 2;
   constexpr int NKT = D / 16;
@@ -141,17 +162,16 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
 
   extern __shared__ __align__(128) unsigned char smem[];
   float* sm_beta = reinterpret_cast<float*>(smem + C::OFF_BETA);
-  float* sm_m = reinterpret_cast<float*>(smem + C::OFF_M);
-  float* sm_l = reinterpret_cast<float*>(smem + C::OFF_L);
-  float* sm_o = reinterpret_cast<float*>(smem + C::OFF_O);
+  float* sm_state = reinterpret_cast<float*>(smem + C::OFF_S);   // [2][SBUF_F]
   uint16_t* sm_q = reinterpret_cast<uint16_t*>(smem + C::OFF_Q);
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_ready = bar_full + C::NST;
   uint64_t* bar_empty = bar_ready + C::NST;
   uint64_t* bar_qfull = bar_empty + C::NST;    // [2]
   uint64_t* bar_qempty = bar_qfull + 2;        // [2]
+  uint64_t* bar_sfull = bar_qempty + 2;        // [2] warp states of a segment written
+  uint64_t* bar_sfree = bar_sfull + 2;         // [2] merge warp done with a state buffer
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
-  volatile int* last_flag = abort_flag + 1;
 
   const Geom& gm = a.geom;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,11 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
     for (int i = 0; i < C::NST; ++i) {
       mbar_init(&bar_full[i], 1);
       mbar_init(&bar_ready[i], 1);
-      mbar_init(&bar_empty[i], kConsumers);
+      mbar_init(&bar_empty[i], C::NC);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_qfull[i], 1);
-      mbar_init(&bar_qempty[i], kConsumers + 1);
+      mbar_init(&bar_qempty[i], C::NC + 1);
+      mbar_init(&bar_sfull[i], C::NC);
+      mbar_init(&bar_sfree[i], 1);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -188,6 +210,144 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
   const int64_t i0 = Pt.first_item(Pt.lo(cta));
   const int64_t i1 = Pt.first_item(Pt.lo(cta + 1));
   auto nop_seg = [](int) {};
+  const int64_t last_row = i1 > i0 ? (i1 - 1) / Pt.n_items : -1;
+
+  // Merges the warp states of one segment (state buffer sb) and writes the
+  // row's output when this CTA covers the whole row, else the CTA's partial
+  // (o[D], m, l) of the row; the last CTA to finish a row then merges the row's
+  // partials with a log-sum-exp.  tid / nth: this thread's rank among the nth
+  // threads running it together; sync(): their barrier.  A thread handles four
+  // channels of one head at a time and derives that head's merge factors
+  // itself, so only the publication of a partial needs barriers.
+  auto merge_segment = [&](int row, float* sb, int tid, int nth, auto sync) {
+    constexpr int NC = C::NC, HS = C::HS, DP = C::DP;
+    const float* s_m = sb;
+    const float* s_l = sb + NC * HS;
+    volatile int* s_last = reinterpret_cast<volatile int*>(sb + 2 * NC * HS);
+    const float* s_o = sb + C::SO;
+    const int g = gm.g;
+    const int b = row / gm.Hkv, hkv = row - b * gm.Hkv;
+    const int64_t first_it = (int64_t)row * Pt.n_items;
+    const int c_first = Pt.cta_of(first_it), c_last = Pt.cta_of(first_it + Pt.n_items - 1);
+    const int np = c_last - c_first + 1;
+    float* out_row = a.out + ((int64_t)b * gm.Hq + (int64_t)hkv * g) * D;
+    float* part = a.ws + ((int64_t)(cta + row) * g) * DP;
+    // warp states -> this CTA's (o, M, L) of the row, four channels per step
+    for (int e4 = tid; e4 < g * D / 4; e4 += nth) {
+      const int h = e4 / (D / 4), c = 4 * (e4 - h * (D / 4));
+      float M = -INFINITY;
+      for (int w = 0; w < NC; ++w) M = fmaxf(M, s_m[w * HS + h]);
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      float L = 0.f;
+#pragma unroll 4
+      for (int w = 0; w < NC; ++w) {
+        const float f = M == -INFINITY ? 0.f : exp2f(s_m[w * HS + h] - M);
+        const float4 v = *reinterpret_cast<const float4*>(s_o + (w * HS + h) * D + c);
+        O.x = fmaf(v.x, f, O.x);
+        O.y = fmaf(v.y, f, O.y);
+        O.z = fmaf(v.z, f, O.z);
+        O.w = fmaf(v.w, f, O.w);
+        L = fmaf(s_l[w * HS + h], f, L);
+      }
+      if (np == 1) {
+        if (!*abort_flag) {
+          const float r = 1.f / L;
+          *reinterpret_cast<float4*>(out_row + h * D + c) = make_float4(O.x * r, O.y * r, O.z * r, O.w * r);
+        }
+      } else {
+        *reinterpret_cast<float4*>(part + h * DP + c) = O;
+        if (c == 0) *reinterpret_cast<float4*>(part + h * DP + D) = make_float4(M, L, 0.f, 0.f);
+      }
+    }
+    if (np == 1) return;
+    // The barrier orders every thread's partial stores before thread 0's
+    // gpu-scope acq_rel atomic (release is cumulative), so one fenced atomic
+    // publishes the whole partial; the last arriver's acquire plus the next
+    // barrier make every partial visible to all the merging threads.
+    sync();
+    if (tid == 0) {
+      int last = 0;
+      if (!*abort_flag) {
+        unsigned old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;\n" : "=r"(old) : "l"(a.counters + row) : "memory");
+        last = old == (unsigned)(np - 1);
+      }
+      *s_last = last;
+    }
+    sync();
+    if (!*s_last) return;
+    // Last CTA of the row: online log-sum-exp over the np partials, the loads
+    // of up to kMB partials (o, m, l) in flight together.
+    constexpr int kMB = 4;
+    const float* ws_row = a.ws + (int64_t)(c_first + row) * g * DP;
+    for (int e4 = tid; e4 < g * D / 4; e4 += nth) {
+      const int h = e4 / (D / 4), c = 4 * (e4 - h * (D / 4));
+      const float* col = ws_row + (int64_t)h * DP;
+      float M = -INFINITY, L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j0 = 0; j0 < np; j0 += kMB) {
+        const int nj = min(kMB, np - j0);
+        float4 v[kMB];
+        float2 ml[kMB];
+#pragma unroll
+        for (int u = 0; u < kMB; ++u) {
+          if (u < nj) {
+            const float* pj = col + (int64_t)(j0 + u) * g * DP;
+            v[u] = __ldcg(reinterpret_cast<const float4*>(pj + c));
+            ml[u] = __ldcg(reinterpret_cast<const float2*>(pj + D));
+          }
+        }
+        float Mb = M;
+#pragma unroll
+        for (int u = 0; u < kMB; ++u)
+          if (u < nj) Mb = fmaxf(Mb, ml[u].x);
+        const float r = M == -INFINITY ? 0.f : exp2f(M - Mb);
+        L *= r;
+        acc.x *= r;
+        acc.y *= r;
+        acc.z *= r;
+        acc.w *= r;
+#pragma unroll
+        for (int u = 0; u < kMB; ++u) {
+          if (u < nj) {
+            const float f = ml[u].x == -INFINITY ? 0.f : exp2f(ml[u].x - Mb);
+            L = fmaf(ml[u].y, f, L);
+            acc.x = fmaf(v[u].x, f, acc.x);
+            acc.y = fmaf(v[u].y, f, acc.y);
+            acc.z = fmaf(v[u].z, f, acc.z);
+            acc.w = fmaf(v[u].w, f, acc.w);
+          }
+        }
+        M = Mb;
+      }
+      const float r = 1.f / L;
+      *reinterpret_cast<float4*>(out_row + h * D + c) = make_float4(acc.x * r, acc.y * r, acc.z * r, acc.w * r);
+    }
+    if (tid == 0) a.counters[row] = 0u;
+  };
+
+  if (warp == 2) {
+    // ------------------------------------------------------------ merge: every segment but the CTA's last
+    int k = 0;
+    for_each_chunk<C::SG>(
+        Pt, i0, i1, [](int, int, bool, int64_t, int) {}, nop_seg,
+        [&](int row) {
+          const int sbi = k & 1;
+          const uint32_t par = (k >> 1) & 1;
+          ++k;
+          if (row == last_row) return;   // the consumer warps merge the CTA's last segment
+          const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[sbi], par, abort_flag));
+          if (!ok) {
+            if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
+            *abort_flag = 1;
+          } else {
+            merge_segment(row, sm_state + sbi * C::SBUF_F, lane, 32, [] { __syncwarp(); });
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_sfree[sbi]);
+        });
+    return;
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -266,21 +426,23 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
           if (ok && !win) {
             // columns of B = the stage's groups; rows of A = heads (q, exact in fp16)
             const unsigned char* st = smem + slot * C::STAGE;
-            float bacc[4] = {0.f, 0.f, 0.f, 0.f};
-            const int grp = gr < cnt ? gr : 0;
-            const unsigned char* pz = st + grp * C::REC + C::KZOFF + 16 * tc;
-#pragma unroll
-            for (int i = 0; i < D / 32; ++i) {
-              const uint4 z4 = lds128(pz + 64 * i);
-              const uint32_t a0[4] = {qh[2 * i][0], 0u, qh[2 * i][1], 0u};
-              const uint32_t a1[4] = {qh[2 * i + 1][0], 0u, qh[2 * i + 1][1], 0u};
-              mma_f16_16816(bacc, a0, z4.x, z4.y);
-              mma_f16_16816(bacc, a1, z4.z, z4.w);
-            }
             float* bt = sm_beta + (slot * C::SG) * 8;
-            // thread holds beta(head gr, groups 2tc, 2tc+1)
-            if (2 * tc < cnt) bt[(2 * tc) * 8 + gr] = bacc[0];
-            if (2 * tc + 1 < cnt) bt[(2 * tc + 1) * 8 + gr] = bacc[1];
+            for (int g0 = 0; g0 < cnt; g0 += 8) {   // columns: groups g0 .. g0 + 7
+              float bacc[4] = {0.f, 0.f, 0.f, 0.f};
+              const int grp = g0 + gr < cnt ? g0 + gr : g0;
+              const unsigned char* pz = st + grp * C::REC + C::KZOFF + 16 * tc;
+#pragma unroll
+              for (int i = 0; i < D / 32; ++i) {
+                const uint4 z4 = lds128(pz + 64 * i);
+                const uint32_t a0[4] = {qh[2 * i][0], 0u, qh[2 * i][1], 0u};
+                const uint32_t a1[4] = {qh[2 * i + 1][0], 0u, qh[2 * i + 1][1], 0u};
+                mma_f16_16816(bacc, a0, z4.x, z4.y);
+                mma_f16_16816(bacc, a1, z4.z, z4.w);
+              }
+              // thread holds beta(head gr, groups g0 + 2tc, g0 + 2tc + 1)
+              if (g0 + 2 * tc < cnt) bt[(g0 + 2 * tc) * 8 + gr] = bacc[0];
+              if (g0 + 2 * tc + 1 < cnt) bt[(g0 + 2 * tc + 1) * 8 + gr] = bacc[1];
+            }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar_ready[slot]);
@@ -311,13 +473,21 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
   }
 
   // ------------------------------------------------------------------ consumers
-  const int cw = warp - 2;
-  const bool head_ok = gr < gm.g;
+  const int cw = warp - 3;
+  // Head whose q this lane feeds to the score contraction: gr in the
+  // head-major formulation; gr >> 1 in the token-major one, where column gr of
+  // the q~ operand is the hi (even gr) or lo (odd gr) part of head gr >> 1.
+  const int qhead = TR ? gr >> 1 : gr;
+  const bool head_ok = qhead < gm.g;
   const uint32_t magic = kMagic;
   int qseg = 0;
   const uint16_t* sq = sm_q;   // ring slot of the current segment
-  uint32_t qh[NKT][2];   // q of head gr at channels 16kt + 8rho + 2tc + {0, 1}, fp16x2
-  float o[NNT][4];
+  uint32_t qh[NKT][2];   // q of head qhead at channels 16kt + 8rho + 2tc + {0, 1}, fp16x2
+  // Output accumulators.  Head-major: m16n8 tiles (rows = heads hi | lo,
+  // columns = 8 channels).  Token-major: m16n8 tiles (rows = 16 channels,
+  // columns = heads x {hi, lo}); this lane then holds head tc only.
+  constexpr int NO = TR ? D / 16 : NNT;
+  float o[NO][4];
   float m = -INFINITY, l = 0.f, wz = 0.f;
   int seg_row = 0;
 
@@ -331,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
       *abort_flag = 1;
     }
     sq = sm_q + qs * 8 * D;
-    const uint16_t* qrow = sq + gr * D;
+    const uint16_t* qrow = sq + qhead * D;
     // q, pre-scaled by the position compensation of the key codes it meets:
     // pair position j' = (2kt + rho) & 3 for 2-bit, rho for 4-bit
 #pragma unroll
@@ -346,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
         qh[kt][rho] = h2_as_u32(__hmul2(u32_as_h2(qv), u32_as_h2(pos_comp(BITS, jp))));
       }
 #pragma unroll
-    for (int i = 0; i < NNT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    for (int i = 0; i < NO; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     m = -INFINITY;
     l = 0.f;
     wz = 0.f;
@@ -362,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
       l *= alpha;
       wz *= alpha;
 #pragma unroll
-      for (int i = 0; i < NNT; ++i) {
+      for (int i = 0; i < NO; ++i) {
         o[i][0] *= alpha;
         o[i][1] *= alpha;
         o[i][2] *= alpha;
@@ -370,6 +540,194 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
       }
       m = mn;
     }
+  };
+
+  // ---------------------------------------------------------------- token-major formulation
+  // Tokens are the M dimension of both contractions, so the K and V codes are
+  // the A operand (one A fragment = the B fragments of two adjacent 8-token
+  // or 8-channel tiles of the packed format) and the N = 8 columns are the
+  // heads' hi and lo parts: column 2h + {0, 1} = head h, hi | lo.  A GQA group
+  // of up to 4 heads then fills the tile, with half the mma's of the
+  // head-major formulation and half its accumulators.  Lane (gr, tc) holds
+  // the scores of head tc for tokens gr + 8i and the output of head tc.
+  uint32_t* sm_pw = reinterpret_cast<uint32_t*>(smem + C::OFF_PW) + cw * 128;   // [32 tokens][4 words]
+  auto tr_head_max = [&](float x) {
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 8));
+    return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 16));
+  };
+  auto tr_block = [&](const unsigned char* st, int slot) {
+    const int grp = cw / C::NTB, tbg = cw - grp * C::NTB;
+    const unsigned char* rec = st + grp * C::REC;
+    uint4 kc[P / 4];
+#pragma unroll
+    for (int p = 0; p < P / 4; ++p) kc[p] = lds128(rec + tbg * C::TBC + 16 * (32 * p + lane));
+    const float beta = sm_beta[(slot * C::SG + grp) * 8 + tc];
+    const unsigned char* psc = rec + C::KSOFF + 16 * tc;
+    // fp16x2 (-1, -1) on lo lanes, (0, 0) on hi lanes: q~ column = fma(q, s, sel * round(q s))
+    const uint32_t sel = (gr & 1) ? 0xBC00BC00u : 0u;
+    float sc[2][2][4];   // [k-tile parity][token m-tile]
+#pragma unroll
+    for (int par = 0; par < 2; ++par)
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) sc[par][mt][0] = sc[par][mt][1] = sc[par][mt][2] = sc[par][mt][3] = 0.f;
+#pragma unroll
+    for (int wi = 0; wi < WPN; ++wi)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pr[4][J];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          const int w = nt * WPN + wi;
+          const uint4 pc = kc[w >> 2];
+          const uint32_t word = (w & 3) == 0 ? pc.x : (w & 3) == 1 ? pc.y : (w & 3) == 2 ? pc.z : pc.w;
+          unpack_half<BITS>(half ? word >> 8 : word, pr[nt], magic);
+        }
+#pragma unroll
+        for (int m2 = 0; m2 < J / 2; ++m2) {
+          const int kt = (J / 2) * (2 * wi + half) + m2;
+          const uint2 s2 = *reinterpret_cast<const uint2*>(psc + 64 * (kt >> 1) + 8 * (kt & 1));
+          const __half2 h0 = __hmul2(u32_as_h2(qh[kt][0]), u32_as_h2(s2.x));
+          const __half2 h1 = __hmul2(u32_as_h2(qh[kt][1]), u32_as_h2(s2.y));
+          const uint32_t b0 = h2_as_u32(__hfma2(u32_as_h2(qh[kt][0]), u32_as_h2(s2.x), __hmul2(h0, u32_as_h2(sel))));
+          const uint32_t b1 = h2_as_u32(__hfma2(u32_as_h2(qh[kt][1]), u32_as_h2(s2.y), __hmul2(h1, u32_as_h2(sel))));
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            const uint32_t ak[4] = {pr[2 * mt][2 * m2], pr[2 * mt + 1][2 * m2], pr[2 * mt][2 * m2 + 1],
+                                    pr[2 * mt + 1][2 * m2 + 1]};
+            mma_f16_16816(sc[kt & 1][mt], ak, b0, b1);
+          }
+        }
+      }
+    // scores of head tc, tokens gr + 8i (i = 2 mt + e2)
+    float x[4];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int e2 = 0; e2 < 2; ++e2) {
+        const int i = 2 * mt + e2;
+        x[i] = ((sc[0][mt][2 * e2] + sc[1][mt][2 * e2]) + (sc[0][mt][2 * e2 + 1] + sc[1][mt][2 * e2 + 1]) + beta) *
+               a.scale_log2;
+        mx = fmaxf(mx, x[i]);
+      }
+    rescale_to(tr_head_max(mx));
+    // value meta of token gr + 8i sits at entry 8 (gr >> 1) + 2i + (gr & 1) of the TB
+    const unsigned char* pvm = rec + C::VMOFF + 4 * (tbg * kTB + 8 * (gr >> 1) + (gr & 1));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float p = fast_exp2(x[i] - m);
+      const float2 sz = __half22float2(u32_as_h2(*reinterpret_cast<const uint32_t*>(pvm + 8 * i)));
+      l += p;
+      wz = fmaf(p, sz.y, wz);
+      // value pair position j' of token gr + 8i: i (2-bit), i & 1 (4-bit)
+      const float ps = p * (sz.x * pos_comp_f(BITS, BITS == 2 ? i : (i & 1)));
+      const __half hi = __float2half_rn(ps);
+      const __half lo = __float2half_rn(ps - __half2float(hi));
+      sm_pw[(gr + 8 * i) * 4 + tc] = h2_as_u32(__halves2half2(hi, lo));
+    }
+    __syncwarp();
+    uint32_t bp[4];   // k-tile kt: b0 = bp[2kt], b1 = bp[2kt + 1]
+    ldsm_x4_t(bp, sm_pw + 4 * lane);
+    uint4 vc[P / 4];
+#pragma unroll
+    for (int p = 0; p < P / 4; ++p) vc[p] = lds128(rec + (C::NTB + tbg) * C::TBC + 16 * (32 * p + lane));
+    auto vword = [&](int w) {
+      const uint4 pc = vc[w >> 2];
+      return (w & 3) == 0 ? pc.x : (w & 3) == 1 ? pc.y : (w & 3) == 2 ? pc.z : pc.w;
+    };
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        uint32_t av[4];
+        if (BITS == 2) {
+          // channels 16mt + gr (low byte of each half word) and 16mt + 8 + gr (high byte)
+          const uint32_t w = vword(mt);
+          av[0] = kt ? unpack_pair<2, 2>(w, magic) : unpack_pair<2, 0>(w, magic);
+          av[1] = kt ? unpack_pair<2, 2>(w >> 8, magic) : unpack_pair<2, 0>(w >> 8, magic);
+          av[2] = kt ? unpack_pair<2, 3>(w, magic) : unpack_pair<2, 1>(w, magic);
+          av[3] = kt ? unpack_pair<2, 3>(w >> 8, magic) : unpack_pair<2, 1>(w >> 8, magic);
+        } else {
+          // words 2mt (channel 16mt + gr) and 2mt + 1 (16mt + 8 + gr); half word = kt
+          const uint32_t w0 = kt ? vword(2 * mt) >> 8 : vword(2 * mt);
+          const uint32_t w1 = kt ? vword(2 * mt + 1) >> 8 : vword(2 * mt + 1);
+          av[0] = unpack_pair<4, 0>(w0, magic);
+          av[1] = unpack_pair<4, 0>(w1, magic);
+          av[2] = unpack_pair<4, 1>(w0, magic);
+          av[3] = unpack_pair<4, 1>(w1, magic);
+        }
+        mma_f16_16816(o[mt], av, bp[2 * kt], bp[2 * kt + 1]);
+      }
+    __syncwarp();   // the P tile is rewritten by this warp's next block
+  };
+  // Window chunk: warps 0 and 1 take tokens 16cw .. 16cw + 15 (exact 16-bit
+  // operands; p split hi + lo in the input's format).
+  auto tr_window = [&](const unsigned char* st, int64_t first) {
+    const int n_tok = min(kWinTok, a.r - (int)first * kWinTok);
+    const int t0 = 16 * cw;
+    if (cw >= kWinTok / 16 || t0 >= n_tok) return;
+    const unsigned char* kb = st;
+    const unsigned char* vb = st + kWinTok * C::WROW;
+    const bool bf = gm.dtype == KVQ_BF16;
+    const int mi = lane >> 3, ri = lane & 7;   // ldmatrix: matrix and row this lane addresses
+    // scores: A = key rows t0 .. t0 + 15 (matrix mi: rows + 8 (mi & 1), channels + 8 (mi >> 1));
+    // B = q, column gr = head gr >> 1 on even gr, zero on odd gr
+    const int krow = min(t0 + 8 * (mi & 1) + ri, kWinTok - 1);
+    const bool qcol = !(gr & 1) && (gr >> 1) < gm.g;
+    const uint16_t* qr = sq + (gr >> 1) * D;
+    float sw[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kt = 0; kt < NKT; ++kt) {
+      uint32_t ak[4];
+      ldsm_x4(ak, kb + krow * C::WROW + (16 * kt + 8 * (mi >> 1)) * 2);
+      const uint32_t b0 = qcol ? *reinterpret_cast<const uint32_t*>(qr + 16 * kt + 2 * tc) : 0u;
+      const uint32_t b1 = qcol ? *reinterpret_cast<const uint32_t*>(qr + 16 * kt + 8 + 2 * tc) : 0u;
+      if (bf) mma_bf16_16816(sw[kt & 1], ak, b0, b1);
+      else mma_f16_16816(sw[kt & 1], ak, b0, b1);
+    }
+    float xv[2];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int e2 = 0; e2 < 2; ++e2) {
+      const bool valid = t0 + gr + 8 * e2 < n_tok;
+      xv[e2] = valid ? (sw[0][2 * e2] + sw[1][2 * e2]) * a.scale_log2 : -INFINITY;
+      mx = fmaxf(mx, xv[e2]);
+    }
+    rescale_to(tr_head_max(mx));
+    float pw[2];
+#pragma unroll
+    for (int e2 = 0; e2 < 2; ++e2) {
+      pw[e2] = xv[e2] == -INFINITY ? 0.f : fast_exp2(xv[e2] - m);
+      l += pw[e2];
+    }
+    // P tile rows = tokens gr, gr + 8; word tc = (hi, lo) of head tc
+    const uint32_t ph = pack2_in16(pw[0], pw[1], gm.dtype);
+    const float2 pb = unpack2_in16(ph, gm.dtype);
+    const uint32_t pl = pack2_in16(pw[0] - pb.x, pw[1] - pb.y, gm.dtype);
+    sm_pw[gr * 4 + tc] = (ph & 0xFFFFu) | (pl << 16);
+    sm_pw[(gr + 8) * 4 + tc] = (ph >> 16) | (pl & 0xFFFF0000u);
+    __syncwarp();
+    uint32_t bp[2];
+    ldsm_x2_t(bp, sm_pw + 4 * (lane & 15));
+    // P.V: A = value rows transposed (matrix mi: tokens + 8 (mi >> 1), channels + 8 (mi & 1));
+    // rows past n_tok are zeroed so stale shared memory never meets the zero weights
+    const int vrow = min(t0 + 8 * (mi >> 1) + ri, kWinTok - 1);
+    const uint32_t m01 = (t0 + 2 * tc < n_tok ? 0x0000FFFFu : 0u) | (t0 + 2 * tc + 1 < n_tok ? 0xFFFF0000u : 0u);
+    const uint32_t m23 =
+        (t0 + 8 + 2 * tc < n_tok ? 0x0000FFFFu : 0u) | (t0 + 8 + 2 * tc + 1 < n_tok ? 0xFFFF0000u : 0u);
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      uint32_t av[4];
+      ldsm_x4_t(av, vb + vrow * C::WROW + (16 * mt + 8 * (mi & 1)) * 2);
+      av[0] &= m01;
+      av[1] &= m01;
+      av[2] &= m23;
+      av[3] &= m23;
+      if (bf) mma_bf16_16816(o[mt], av, bp[0], bp[1]);
+      else mma_f16_16816(o[mt], av, bp[0], bp[1]);
+    }
+    __syncwarp();
   };
 
   auto chunk = [&](int s, int row, bool win, int64_t first, int cnt) {
@@ -382,7 +740,10 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
       *abort_flag = 1;
     }
     const unsigned char* st = smem + slot * C::STAGE;
-    if (ok && !win && cw < cnt * C::NTB) {
+    if constexpr (TR) {
+      if (ok && !win && cw < cnt * C::NTB) tr_block(st, slot);
+      else if (ok && win) tr_window(st, first);
+    } else if (ok && !win && cw < cnt * C::NTB) {
       // ---------------------------------------------------------- one quantized TB
       const int grp = cw / C::NTB, tbg = cw - grp * C::NTB;
       const unsigned char* rec = st + grp * C::REC;
@@ -554,152 +915,89 @@ __global__ void __launch_bounds__(kThreads, 1) kivi_decode_kernel(AttnArgs a) {
     if (lane == 0) mbar_arrive(&bar_empty[slot]);
   };
 
+  int final_row = -1;
+  float* final_sb = nullptr;
   auto seg_end = [&](int row) {
-    // warp states -> shared memory (consumer warps only)
-    const float ls = quad_sum(l), wzs = quad_sum(wz);
-    if (tc == 0) {
-      sm_m[cw * 8 + gr] = m;
-      sm_l[cw * 8 + gr] = ls;
+    // warp state -> state buffer k & 1, once the merge warp is done with segment k - 2
+    const int k = qseg - 1;
+    const int sbi = k & 1;
+    float* sb = sm_state + sbi * C::SBUF_F;
+    if (k >= 2) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfree[sbi], ((k >> 1) - 1) & 1, abort_flag));
+      if (!ok) {
+        if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
+        *abort_flag = 1;
+      }
     }
+    float* s_m = sb;
+    float* s_l = sb + C::NC * C::HS;
+    float* s_o = sb + C::SO;
+    if constexpr (TR) {
+      // head tc: l and wz summed over the 8 lanes gr
+      float ls = l, wzs = wz;
 #pragma unroll
-    for (int nt = 0; nt < NNT; ++nt)
+      for (int x = 4; x < 32; x <<= 1) {
+        ls += __shfl_xor_sync(0xffffffffu, ls, x);
+        wzs += __shfl_xor_sync(0xffffffffu, wzs, x);
+      }
+      if (gr == 0) {
+        s_m[cw * C::HS + tc] = m;
+        s_l[cw * C::HS + tc] = ls;
+      }
 #pragma unroll
-      for (int e = 0; e < 2; ++e) sm_o[(cw * 8 + gr) * D + 8 * nt + 2 * tc + e] = o[nt][e] + o[nt][2 + e] + wzs;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bar_qempty[(qseg - 1) & 1]);   // this warp is done with the segment's q
-    consumer_bar();
-    const int ct = threadIdx.x - 64;
-    const int b = row / gm.Hkv, hkv = row - b * gm.Hkv;
-    const int64_t first_it = (int64_t)row * Pt.n_items;
-    const int c_first = Pt.cta_of(first_it), c_last = Pt.cta_of(first_it + Pt.n_items - 1);
-    const int expected = c_last - c_first + 1;
-    float* out_row = a.out + ((int64_t)b * gm.Hq + (int64_t)hkv * gm.g) * D;
-    if (expected == 1) {
-      for (int i = ct; i < gm.g * D; i += kConsumers * 32) {
-        const int h = i / D, c = i - h * D;
-        float M = -INFINITY;
-        for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, sm_m[w * 8 + h]);
-        float O = 0.f, L = 0.f;
-        for (int w = 0; w < kConsumers; ++w) {
-          const float f = M == -INFINITY ? 0.f : exp2f(sm_m[w * 8 + h] - M);
-          O += sm_o[(w * 8 + h) * D + c] * f;
-          L += sm_l[w * 8 + h] * f;
-        }
-        if (!*abort_flag) out_row[i] = O / L;
+      for (int mt = 0; mt < NO; ++mt) {
+        s_o[(cw * C::HS + tc) * D + 16 * mt + gr] = o[mt][0] + o[mt][1] + wzs;
+        s_o[(cw * C::HS + tc) * D + 16 * mt + 8 + gr] = o[mt][2] + o[mt][3] + wzs;
       }
     } else {
-      float* part = a.ws + ((int64_t)(cta + row) * gm.g) * (D + 2);
-      for (int i = ct; i < gm.g * (D + 2); i += kConsumers * 32) {
-        const int h = i / (D + 2), c = i - h * (D + 2);
-        float M = -INFINITY;
-        for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, sm_m[w * 8 + h]);
-        float val;
-        if (c == D) {
-          val = M;
-        } else {
-          val = 0.f;
-          for (int w = 0; w < kConsumers; ++w) {
-            const float f = M == -INFINITY ? 0.f : exp2f(sm_m[w * 8 + h] - M);
-            val += (c < D ? sm_o[(w * 8 + h) * D + c] : sm_l[w * 8 + h]) * f;
-          }
-        }
-        part[i] = val;
+      const float ls = quad_sum(l), wzs = quad_sum(wz);
+      if (tc == 0) {
+        s_m[cw * C::HS + gr] = m;
+        s_l[cw * C::HS + gr] = ls;
       }
-      // The CTA barrier orders every thread's partial stores before thread 0's
-      // gpu-scope acq_rel atomic (release is cumulative), so one fenced atomic
-      // publishes the whole partial; the last arriver's acquire plus the next
-      // barrier make every partial visible to all its threads.
-      consumer_bar();
-      if (ct == 0) {
-        int last = 0;
-        if (!*abort_flag) {
-          unsigned old;
-          asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;\n" : "=r"(old) : "l"(a.counters + row) : "memory");
-          last = old == (unsigned)(expected - 1);
-        }
-        *last_flag = last;
-      }
-      consumer_bar();
-      if (*last_flag) {
-        // last CTA of the row: merge its np partials.  All loads of a step are
-        // independent and issued together; the per-partial weights
-        // 2^(m_j - M) / L go through shared memory (the warp-state area).
-        const int np = c_last - c_first + 1;
-        const int g = gm.g;
-        float* pm = sm_o;                  // [np][g]
-        float* pw = sm_o + np * g;         // [np][g]
-        float* pl = sm_o + 2 * np * g;     // [np][g]
-        float* hm = sm_o + 3 * np * g;     // [g] max, then [g] 1/L
-        const float* ws_row = a.ws + (int64_t)(c_first + row) * g * (D + 2);
-        for (int i = ct; i < np * g; i += kConsumers * 32) {
-          pm[i] = __ldcg(ws_row + (int64_t)i * (D + 2) + D);
-          pl[i] = __ldcg(ws_row + (int64_t)i * (D + 2) + D + 1);
-        }
-        consumer_bar();
-        for (int h = ct; h < g; h += kConsumers * 32) {
-          float M = -INFINITY;
-          for (int j = 0; j < np; ++j) M = fmaxf(M, pm[j * g + h]);
-          float L = 0.f;
-          for (int j = 0; j < np; ++j) L += pm[j * g + h] == -INFINITY ? 0.f : pl[j * g + h] * exp2f(pm[j * g + h] - M);
-          hm[h] = M;
-          hm[g + h] = 1.f / L;
-        }
-        consumer_bar();
-        for (int i = ct; i < np * g; i += kConsumers * 32) {
-          const int h = i % g;
-          pw[i] = pm[i] == -INFINITY ? 0.f : exp2f(pm[i] - hm[h]) * hm[g + h];
-        }
-        consumer_bar();
-        for (int e = ct; e < g * D; e += kConsumers * 32) {
-          const int h = e / D, c = e - h * D;
-          const float* col = ws_row + (int64_t)h * (D + 2) + c;
-          float acc = 0.f;
-          int j = 0;
-          for (; j + 8 <= np; j += 8) {
-            float v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = __ldcg(col + (int64_t)(j + u) * g * (D + 2));
+      for (int nt = 0; nt < NNT; ++nt)
 #pragma unroll
-            for (int u = 0; u < 8; ++u) acc = fmaf(v[u], pw[(j + u) * g + h], acc);
-          }
-          for (; j < np; ++j) acc = fmaf(__ldcg(col + (int64_t)j * g * (D + 2)), pw[j * g + h], acc);
-          out_row[e] = acc;
-        }
-        if (ct == 0) a.counters[row] = 0u;
-      }
+        for (int e = 0; e < 2; ++e) s_o[(cw * C::HS + gr) * D + 8 * nt + 2 * tc + e] = o[nt][e] + o[nt][2 + e] + wzs;
     }
-    consumer_bar();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&bar_qempty[k & 1]);   // this warp is done with the segment's q
+      mbar_arrive(&bar_sfull[sbi]);
+    }
+    if (row == last_row) {   // the CTA's last segment: merged by all consumer warps after the loop
+      final_row = row;
+      final_sb = sb;
+    }
   };
 
   for_each_chunk<C::SG>(Pt, i0, i1, chunk, seg_begin, seg_end);
+  if (final_row >= 0) {
+    consumer_bar<C::NC>();   // every consumer warp's state of the segment is written
+    merge_segment(final_row, final_sb, threadIdx.x - 96, C::NC * 32, [] { consumer_bar<C::NC>(); });
+  }
 }
 
-template <int BITS, int D, int G>
+template <int BITS, int D, int G, bool TR>
 void launch_decode(const AttnArgs& a, cudaStream_t st) {
-  using C = K<BITS, D, G>;
-  auto kern = kivi_decode_kernel<BITS, D, G>;
+  using C = K<BITS, D, G, TR>;
+  auto kern = kivi_decode_kernel<BITS, D, G, TR>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     attr_set = true;
   }
-  kern<<<a.n_cta, kThreads, C::SMEM, st>>>(a);
+  kern<<<a.n_cta, C::THREADS, C::SMEM, st>>>(a);
   count_launch(1);
 }
 
-}  // namespace
-
-int decode_stage_bytes(int bits, int d, int G) {
-  if (bits == 2 && d == 128 && G == 32) return K<2, 128, 32>::STAGE;
-  if (bits == 2 && d == 64 && G == 32) return K<2, 64, 32>::STAGE;
-  if (bits == 4 && d == 128 && G == 64) return K<4, 128, 64>::STAGE;
-  if (bits == 4 && d == 128 && G == 32) return K<4, 128, 32>::STAGE;
-  if (bits == 2 && d == 128 && G == 64) return K<2, 128, 64>::STAGE;
-  if (bits == 4 && d == 64 && G == 32) return K<4, 64, 32>::STAGE;
-  if (bits == 2 && d == 64 && G == 64) return K<2, 64, 64>::STAGE;
-  if (bits == 4 && d == 64 && G == 64) return K<4, 64, 64>::STAGE;
-  return 0;
+template <int BITS, int D, int G>
+void launch_decode(const AttnArgs& a, cudaStream_t st) {
+  if (a.geom.g <= 4) launch_decode<BITS, D, G, true>(a, st);
+  else launch_decode<BITS, D, G, false>(a, st);
 }
+
+}  // namespace
 
 void launch_kivi_attention(const AttnArgs& a, cudaStream_t st) {
   const Geom& g = a.geom;

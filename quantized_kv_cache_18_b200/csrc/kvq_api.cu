@@ -125,7 +125,7 @@ static int plan_ctas(const kvq_config& c, int64_t n_groups, int r) {
   const int64_t w_tot = rows * (n_groups * rec + (int64_t)r * tokb);
   const int64_t w_max = r > 0 ? (rec > 32 * tokb ? rec : 32 * tokb) : rec;
   int64_t n = w_tot / w_max;
-  const int64_t sms = num_sms();
+  const int64_t sms = num_sms() < kMaxDecodeCtas ? num_sms() : kMaxDecodeCtas;
   if (n > sms) n = sms;
   if (n < 1) n = 1;
   return (int)n;
@@ -158,7 +158,8 @@ size_t kvq_workspace_bytes(const kvq_config* cfg) {
   const int g = cfg->num_q_heads / cfg->num_kv_heads;
   if (cfg->scheme == KVQ_TURBO)
     return tq_qprep_bytes(cfg) + (size_t)((2 * rows + num_sms()) * g * (cfg->head_dim + 2) * sizeof(float));
-  return (size_t)((rows + num_sms()) * g * (cfg->head_dim + 2) * sizeof(float));
+  // KIVI partial rows are (o[d], m, l) padded to d + 4 floats for 16-byte loads
+  return (size_t)((rows + num_sms()) * g * (cfg->head_dim + 4) * sizeof(float));
 }
 
 kvq_status kvq_get_layout(const kvq_config* cfg, kvq_layout* out) {

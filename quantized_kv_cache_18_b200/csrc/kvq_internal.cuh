@@ -36,6 +36,7 @@
 namespace kvq {
 
 constexpr int kTB = 32;         // tokens per token block
+constexpr int kMaxDecodeCtas = 160;   // decode launches use at most this many CTAs (one per SM)
 
 struct Geom {
   int scheme, d, bits, G, R, cap, B, Hkv, Hq, g, dtype;
@@ -229,7 +230,6 @@ void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_
 void launch_tq_quantize(const QuantArgs& a, cudaStream_t st);
 void launch_tq_query_prep(const Geom& g, const uint16_t* q, unsigned char* qprep, cudaStream_t st);
 void launch_tq_attention(const AttnArgs& a, cudaStream_t st);
-int decode_stage_bytes(int bits, int d, int G);
 size_t cache_workspace_bytes(const kvq_cache* cache);   // kvq_workspace_bytes of the cache's config
 
 int num_sms();

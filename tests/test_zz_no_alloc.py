@@ -63,7 +63,7 @@ def test_static_entry_point_matches_workspace_entry_point(name, kw, S):
 
 
 def test_static_entry_point_rejects_configs_over_the_limit():
-    # (rows + SMs) * g * (d + 2) * 4 bytes of scratch > 4 MiB for 2048 rows of GQA 4, d 128
+    # (rows + SMs) * g * (d + 4) * 4 bytes of scratch > 4 MiB for 2048 rows of GQA 4, d 128
     cfg = make_config("kivi", 2, 32, 32, 128, 8, 32, 256, 64, "bf16")
     assert workspace_bytes(cfg) > 4 * 1024 * 1024
     cache = QuantizedKVCache(cfg)
