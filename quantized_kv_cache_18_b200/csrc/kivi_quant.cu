@@ -5,8 +5,13 @@
 // (2^b - 1) and zero-point z = min ("Quantification du KV-Cache : TurboQuant et
 // l'etat de l'art en 2026", section "KIVI (2024)"; zubnet.ai survey, "Famille
 // deux, c'est la quantification").  Codes are packed 16 INT2 or 8 INT4 per
-// 32-bit word ("TurboQuant : les cinq innovations", item 3) in the v1 order
-// described in kvq_internal.cuh.
+// 32-bit word ("TurboQuant : les cinq innovations", item 3) in the fragment
+// order described in kvq_internal.cuh.
+//
+// A CTA handles one group record in four passes over shared memory: stage the
+// key and value tiles, reduce the parameters (key and value warps side by
+// side), decide the codes (a thread keeps one channel pair's or one token
+// pair's parameters in registers), pack 16-byte pieces of the record.
 #include <cuda_runtime.h>
 
 #include "kvq_internal.cuh"
@@ -21,21 +26,61 @@ __device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bits) {
   if (bits) atomicOr(status, bits);
 }
 
-// One CTA quantizes one group record (G tokens of one row).
-template <int BITS, int D, int G>
+// Codes are round half to even of (x - z) / s, clamped to [0, levels], with
+// s, z the fp16 scale and zero-point.  The fp32 estimate r = fma(x, 1/s, -z/s)
+// differs from the exact quotient by less than 2^-24 (2 levels + |z| / s) up to
+// second-order terms (one rounding each in 1/s, z/s and the fma; r is only used
+// where it lies in [0, levels]); eb below is four times that.  An estimate more
+// than eb away from every rounding boundary k + 1/2 decides.  Within eb, which
+// takes in the exact ties that 16-bit inputs and fp16 scales often produce, the
+// exact double-precision comparison of 2 (x - z) with (2k + 1) s decides.
+struct CodeParams {
+  float s, z, inv, zinv, eb;
+};
+__device__ __forceinline__ CodeParams code_params(float s, float z, int levels) {
+  CodeParams p;
+  p.s = s;
+  p.z = z;
+  p.inv = s > 0.f ? 1.f / s : 0.f;
+  p.zinv = z * p.inv;
+  p.eb = 2.384185791015625e-7f * (2.f * (float)levels + 2.f + fabsf(p.zinv));   // 2^-22 (...)
+  return p;
+}
+__device__ __forceinline__ uint32_t code_of(float x, const CodeParams& p, int levels) {
+  float r = fmaf(x, p.inv, -p.zinv);
+  r = fminf(fmaxf(r, 0.f), (float)levels);   // also maps NaN to 0
+  const float k = rintf(r);
+  if (fabsf(fabsf(r - k) - 0.5f) > p.eb) return (uint32_t)k;
+  return (uint32_t)exact_code((double)x, (double)p.z, (double)p.s, p.s > 0.f ? 1.0 / (double)p.s : 0.0, levels);
+}
+
+template <bool BF>
+__device__ __forceinline__ float in16f(uint16_t bits) {
+  return BF ? __uint_as_float((uint32_t)bits << 16) : __half2float(__ushort_as_half(bits));
+}
+
+// One CTA quantizes one group record (G tokens of one row); BF: bf16 inputs
+// (else fp16).
+template <int BITS, int D, int G, bool BF>
 __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs a) {
   constexpr int LEVELS = (1 << BITS) - 1;
   constexpr int NTB = G / kTB;
   constexpr int P = D * BITS / 32;              // words per lane per TB
   constexpr int PAIRS = 16 / BITS;              // pairs per word
   constexpr int J = BITS == 2 ? 4 : 2;          // pairs per half word
+  constexpr int PITCH = D + 8;                  // staged row pitch (halves): rows 8 apart land 4 banks apart
+  // key codes: thread = (channel pair, token range); value codes: thread = (token pair, channel range)
+  constexpr int KCP = D / 2, KTR = kQuantThreads / KCP, KTOK = G / KTR;
+  constexpr int VTP = G / 2, VCR = kQuantThreads / VTP, VCH = D / VCR;
+  static_assert(kQuantThreads % KCP == 0 && G % KTR == 0, "key code split");
+  static_assert(kQuantThreads % VTP == 0 && D % VCR == 0 && VCH % 8 == 0, "value code split");
   extern __shared__ __align__(16) unsigned char smem[];
-  uint16_t* sk = reinterpret_cast<uint16_t*>(smem);            // [G][D]
-  uint16_t* sv = sk + G * D;                                   // [G][D]
-  uint8_t* ck = reinterpret_cast<uint8_t*>(sv + G * D);        // [G][D]
-  uint8_t* cv = ck + G * D;                                    // [G][D]
-  __shared__ double k_s[D], k_z[D], k_inv[D];
-  __shared__ double v_s[G], v_z[G], v_inv[G];
+  uint16_t* sk = reinterpret_cast<uint16_t*>(smem);            // [G][PITCH] staged keys
+  uint16_t* sv = sk + G * PITCH;                               // [G][PITCH] staged values
+  uint8_t* ck = reinterpret_cast<uint8_t*>(sv + G * PITCH);    // [G][D] key codes
+  uint8_t* cvt = ck + G * D;                                   // [D][G] value codes (channel-major)
+  __shared__ float k_s[D], k_z[D];
+  __shared__ float v_s[G], v_z[G];
   __shared__ uint16_t k_sb[D], k_zb[D], v_sb[G], v_zb[G];
   __shared__ uint32_t s_flags;
 
@@ -49,61 +94,70 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
   const uint16_t* gk = a.src_k + (int64_t)row * a.src_row_stride + (int64_t)grp * G * D;
   const uint16_t* gv = a.src_v + (int64_t)row * a.src_row_stride + (int64_t)grp * G * D;
   for (int i = tid; i < G * D / 8; i += kQuantThreads) {
-    reinterpret_cast<uint4*>(sk)[i] = ldg_nc_v4(reinterpret_cast<const uint4*>(gk) + i);
-    reinterpret_cast<uint4*>(sv)[i] = ldg_nc_v4(reinterpret_cast<const uint4*>(gv) + i);
+    const int t = i / (D / 8), c8 = i - t * (D / 8);
+    *reinterpret_cast<uint4*>(sk + t * PITCH + 8 * c8) = ldg_nc_v4(reinterpret_cast<const uint4*>(gk) + i);
+    *reinterpret_cast<uint4*>(sv + t * PITCH + 8 * c8) = ldg_nc_v4(reinterpret_cast<const uint4*>(gv) + i);
   }
   __syncthreads();
 
   uint32_t flags = 0;
-  // 2. key parameters, one channel per thread
-  for (int c = tid; c < D; c += kQuantThreads) {
-    float mn = in16_to_float(sk[c], gm.dtype), mx = mn;
-    bool fin = isfinite(mn);
-    for (int t = 1; t < G; ++t) {
-      const float x = in16_to_float(sk[t * D + c], gm.dtype);
-      fin &= isfinite(x);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+  // 2. parameters.  Warps 0-1: keys, one channel pair per thread over the G
+  // tokens; warps 2-3: values, one token per warp at a time.  An input that is
+  // inf or NaN turns the running fma(x, 0, .) into NaN.
+  static_assert(D / 2 <= 64, "key parameter split");
+  if (tid < 64) {
+    for (int cp = tid; cp < D / 2; cp += 64) {
+      const int c = 2 * cp;
+      float mn0 = INFINITY, mx0 = -INFINITY, mn1 = INFINITY, mx1 = -INFINITY, nf = 0.f;
+#pragma unroll 8
+      for (int t = 0; t < G; ++t) {
+        const uint32_t x2 = *reinterpret_cast<const uint32_t*>(sk + t * PITCH + c);
+        const float x0 = in16f<BF>((uint16_t)(x2 & 0xFFFFu)), x1 = in16f<BF>((uint16_t)(x2 >> 16));
+        nf = fmaf(x0, 0.f, fmaf(x1, 0.f, nf));
+        mn0 = fminf(mn0, x0);
+        mx0 = fmaxf(mx0, x0);
+        mn1 = fminf(mn1, x1);
+        mx1 = fmaxf(mx1, x1);
+      }
+      if (nf != 0.f) flags |= KVQ_DEV_NONFINITE_INPUT;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float mn = e ? mn1 : mn0, mx = e ? mx1 : mx0;
+        const __half hs = __double2half(((double)mx - (double)mn) / (double)LEVELS);
+        const __half hz = __double2half((double)mn);
+        const float sc = __half2float(hs), z = __half2float(hz);
+        if (!isfinite(sc) || !isfinite(z)) flags |= KVQ_DEV_PARAM_OVERFLOW;
+        k_s[c + e] = sc;
+        k_z[c + e] = z;
+        k_sb[c + e] = __half_as_ushort(hs);
+        k_zb[c + e] = __half_as_ushort(hz);
+      }
     }
-    const double range = (double)mx - (double)mn;
-    const __half hs = __double2half(range / (double)LEVELS);
-    const __half hz = __double2half((double)mn);
-    const double s = (double)__half2float(hs), z = (double)__half2float(hz);
-    if (!fin) flags |= KVQ_DEV_NONFINITE_INPUT;
-    if (!isfinite(s) || !isfinite(z)) flags |= KVQ_DEV_PARAM_OVERFLOW;
-    k_s[c] = s;
-    k_z[c] = z;
-    k_inv[c] = s > 0.0 ? 1.0 / s : 0.0;
-    k_sb[c] = __half_as_ushort(hs);
-    k_zb[c] = __half_as_ushort(hz);
-  }
-  // 3. value parameters, one token per warp
-  {
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int t = warp; t < G; t += kQuantThreads / 32) {
-      float mn = INFINITY, mx = -INFINITY;
-      bool fin = true;
-      for (int c = lane; c < D; c += 32) {
-        const float x = in16_to_float(sv[t * D + c], gm.dtype);
-        fin &= isfinite(x);
-        mn = fminf(mn, x);
-        mx = fmaxf(mx, x);
+  } else {
+    const int warp = (tid >> 5) - 2, lane = tid & 31;
+    for (int t = warp; t < G; t += 2) {
+      float mn = INFINITY, mx = -INFINITY, nf = 0.f;
+#pragma unroll
+      for (int c2 = lane; c2 < D / 2; c2 += 32) {
+        const uint32_t x2 = *reinterpret_cast<const uint32_t*>(sv + t * PITCH + 2 * c2);
+        const float x0 = in16f<BF>((uint16_t)(x2 & 0xFFFFu)), x1 = in16f<BF>((uint16_t)(x2 >> 16));
+        nf = fmaf(x0, 0.f, fmaf(x1, 0.f, nf));
+        mn = fminf(mn, fminf(x0, x1));
+        mx = fmaxf(mx, fmaxf(x0, x1));
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       }
-      fin = __all_sync(0xffffffffu, fin);
+      if (__any_sync(0xffffffffu, nf != 0.f)) flags |= KVQ_DEV_NONFINITE_INPUT;
       if (lane == 0) {
         const __half hs = __double2half(((double)mx - (double)mn) / (double)LEVELS);
         const __half hz = __double2half((double)mn);
-        const double s = (double)__half2float(hs), z = (double)__half2float(hz);
-        if (!fin) flags |= KVQ_DEV_NONFINITE_INPUT;
-        if (!isfinite(s) || !isfinite(z)) flags |= KVQ_DEV_PARAM_OVERFLOW;
-        v_s[t] = s;
+        const float sc = __half2float(hs), z = __half2float(hz);
+        if (!isfinite(sc) || !isfinite(z)) flags |= KVQ_DEV_PARAM_OVERFLOW;
+        v_s[t] = sc;
         v_z[t] = z;
-        v_inv[t] = s > 0.0 ? 1.0 / s : 0.0;
         v_sb[t] = __half_as_ushort(hs);
         v_zb[t] = __half_as_ushort(hz);
       }
@@ -111,17 +165,45 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
   }
   __syncthreads();
 
-  // 4. codes
-  for (int i = tid; i < G * D; i += kQuantThreads) {
-    const int t = i / D, c = i - t * D;
-    const double xk = (double)in16_to_float(sk[i], gm.dtype);
-    const double xv = (double)in16_to_float(sv[i], gm.dtype);
-    ck[i] = (uint8_t)exact_code(xk, k_z[c], k_s[c], k_inv[c], LEVELS);
-    cv[i] = (uint8_t)exact_code(xv, v_z[t], v_s[t], v_inv[t], LEVELS);
+  // 4. codes.  Keys: channels (2 cp, 2 cp + 1) of tokens [tr * KTOK, +KTOK);
+  // the two codes of a token land side by side in ck.
+  {
+    const int cp = tid % KCP, tr = tid / KCP;
+    const int c = 2 * cp;
+    const CodeParams p0 = code_params(k_s[c], k_z[c], LEVELS), p1 = code_params(k_s[c + 1], k_z[c + 1], LEVELS);
+#pragma unroll 4
+    for (int t = tr * KTOK; t < (tr + 1) * KTOK; ++t) {
+      const uint32_t x2 = *reinterpret_cast<const uint32_t*>(sk + t * PITCH + c);
+      const uint32_t q0 = code_of(in16f<BF>((uint16_t)(x2 & 0xFFFFu)), p0, LEVELS);
+      const uint32_t q1 = code_of(in16f<BF>((uint16_t)(x2 >> 16)), p1, LEVELS);
+      *reinterpret_cast<uint16_t*>(ck + t * D + c) = (uint16_t)(q0 | (q1 << 8));
+    }
+  }
+  // Values: tokens (2 tp, 2 tp + 1), channels [cr * VCH, +VCH); the two codes of
+  // a channel land side by side in the channel-major cvt.
+  {
+    const int tp = tid % VTP, cr = tid / VTP;
+    const int t = 2 * tp;
+    const CodeParams p0 = code_params(v_s[t], v_z[t], LEVELS), p1 = code_params(v_s[t + 1], v_z[t + 1], LEVELS);
+#pragma unroll 2
+    for (int c8 = cr * VCH; c8 < (cr + 1) * VCH; c8 += 8) {
+      const uint4 x0 = *reinterpret_cast<const uint4*>(sv + t * PITCH + c8);
+      const uint4 x1 = *reinterpret_cast<const uint4*>(sv + (t + 1) * PITCH + c8);
+      const uint32_t w0[4] = {x0.x, x0.y, x0.z, x0.w}, w1[4] = {x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint16_t h0 = (uint16_t)(w0[e >> 1] >> (16 * (e & 1))), h1 = (uint16_t)(w1[e >> 1] >> (16 * (e & 1)));
+        const uint32_t q0 = code_of(in16f<BF>(h0), p0, LEVELS);
+        const uint32_t q1 = code_of(in16f<BF>(h1), p1, LEVELS);
+        *reinterpret_cast<uint16_t*>(cvt + (c8 + e) * G + t) = (uint16_t)(q0 | (q1 << 8));
+      }
+    }
   }
   __syncthreads();
 
-  // 5. pack: one 16-byte piece (4 words of one lane) per iteration
+  // 5. packing: one 16-byte piece (4 words of one lane) per iteration; a pair
+  // is the codes of two adjacent channels of a token (keys) or of two adjacent
+  // tokens of a channel (values), one 16-bit load either way
   char* rec = record_ptr(gm, row, a.dst_group0 + grp);
   constexpr int PIECES = NTB * 32 * (P / 4);   // per key (or value) part
   for (int i = tid; i < 2 * PIECES; i += kQuantThreads) {
@@ -131,7 +213,6 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
     const int rem = pi - tb * 32 * (P / 4);
     const int p = rem / 32, lane = rem & 31;
     const int gr = lane >> 2, tc = lane & 3;
-    const uint8_t* cc = (is_v ? cv : ck) + tb * kTB * D;
     uint32_t wv[4];
 #pragma unroll
     for (int e4 = 0; e4 < 4; ++e4) {
@@ -141,16 +222,13 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
       for (int j = 0; j < PAIRS; ++j) {
         const int half = j / J, jp = j % J;
         const int slot = 2 * w + half;
-        int t0, c0, dt, dc;   // first code's (token, channel) and the step to the second
+        uint32_t pr;
         if (!is_v) {
           constexpr int SPN = BITS == 2 ? D / 32 : D / 16;   // slots per key n-tile
           const int nt = slot / SPN;
           const int u = BITS == 2 ? 4 * (slot % SPN) + jp : 2 * (slot % SPN) + jp;
           const int kt = u >> 1, rho = u & 1;
-          t0 = 8 * nt + gr;
-          c0 = 16 * kt + 8 * rho + 2 * tc;
-          dt = 0;
-          dc = 1;
+          pr = *reinterpret_cast<const uint16_t*>(ck + (tb * kTB + 8 * nt + gr) * D + 16 * kt + 8 * rho + 2 * tc);
         } else {
           int nt, u;
           if (BITS == 2) {
@@ -161,14 +239,10 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
             u = 2 * (slot & 1) + jp;
           }
           const int kt = u >> 1, rho = u & 1;
-          c0 = 8 * nt + gr;
-          t0 = 16 * kt + 8 * rho + 2 * tc;
-          dt = 1;
-          dc = 0;
+          pr = *reinterpret_cast<const uint16_t*>(cvt + (8 * nt + gr) * G + tb * kTB + 16 * kt + 8 * rho + 2 * tc);
         }
-        const uint32_t lo = cc[t0 * D + c0];
-        const uint32_t hi = cc[(t0 + dt) * D + c0 + dc];
-        word |= (lo << (BITS * j)) | (hi << (16 + BITS * j));
+        // pr = lo | hi << 8  ->  lo at bit b j, hi at bit 16 + b j
+        word |= ((pr | (pr << 8)) & 0x00FF00FFu) << (BITS * j);
       }
       wv[e4] = word;
     }
@@ -229,10 +303,10 @@ __global__ void clear_words_kernel(uint32_t* words, int n) {
   for (int i = threadIdx.x; i < n; i += blockDim.x) words[i] = 0u;
 }
 
-template <int BITS, int D, int G>
-void launch_q(const QuantArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)G * D * (2 + 2 + 1 + 1);
-  auto kern = kivi_quantize_kernel<BITS, D, G>;
+template <int BITS, int D, int G, bool BF>
+void launch_q_dtype(const QuantArgs& a, cudaStream_t st) {
+  const size_t smem = (size_t)G * (D + 8) * 2 * 2 + (size_t)G * D * 2;
+  auto kern = kivi_quantize_kernel<BITS, D, G, BF>;
   static bool attr_set = false;   // per template instance; the attribute is per device function
   if (!attr_set) {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -240,6 +314,11 @@ void launch_q(const QuantArgs& a, cudaStream_t st) {
   }
   dim3 grid(a.n_groups, a.geom.B * a.geom.Hkv);
   kern<<<grid, kQuantThreads, smem, st>>>(a);
+}
+template <int BITS, int D, int G>
+void launch_q(const QuantArgs& a, cudaStream_t st) {
+  if (a.geom.dtype == KVQ_BF16) launch_q_dtype<BITS, D, G, true>(a, st);
+  else launch_q_dtype<BITS, D, G, false>(a, st);
 }
 
 }  // namespace

@@ -101,6 +101,36 @@ def test_fp16_and_bf16_give_same_path_on_same_values():
     assert torch.equal(c1.records_view()[:, :ng], c2.records_view()[:, :ng])
 
 
+@pytest.mark.parametrize("dtype,bits", [("fp16", 2), ("fp16", 4), ("bf16", 2)])
+def test_code_decisions_on_large_offsets_and_ties(dtype, bits):
+    """Groups whose zero-point is large against their scale (the fp32 estimate
+    of a code is then least accurate) and inputs sitting exactly on rounding
+    boundaries (ties, decided half to even) quantize bit-exactly like the
+    oracle."""
+    w = W.with_sizes(W.WORKLOADS["tiny"], dtype=dtype, bits=bits)
+    rng = np.random.default_rng(7)
+    S = 300
+    x = np.empty((1, 2, S, 64), np.float32)
+    # head 0: offsets of 512 / -300 / 1000 with noise a few ulps wide
+    for t0, off in ((0, 512.0), (96, -300.0), (192, 1000.0)):
+        x[0, 0, t0:t0 + 108] = off + rng.normal(0.0, 1.5, (min(108, S - t0), 64))
+    # head 1: values on the grid z + k s / 2 (every other one a tie), z = 512, s = 1
+    levels = (1 << bits) - 1
+    x[0, 1] = 512.0 + rng.integers(0, 2 * levels + 1, (S, 64)) / 2.0
+    x[0, 1, :, 0] = 512.0          # pins min = 512 and max = 512 + levels in every group
+    x[0, 1, :, 1] = 512.0 + levels
+    k, v = W.to_bits(x, dtype), W.to_bits(x[..., ::-1].copy(), dtype)
+    _run_prefill_bits(w, k, v)
+
+
+def _run_prefill_bits(w, K, V):
+    cache = gpu_prefill(w, K, V)
+    for b in range(w.batch):
+        for h in range(w.num_kv_heads):
+            check_row_bits(cache, b * w.num_kv_heads + h, oracle_row(w, K[b, h], V[b, h]))
+    assert cache.status() == 0
+
+
 def test_nonfinite_input_sets_status_bit():
     w = W.WORKLOADS["tiny"]
     K, V = W.prefill(w, seq_len=256)
