@@ -299,10 +299,20 @@ def run_gpu(args, w, rank, world):
     d_q, d_kn, d_vn = torch.empty_like(q[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
     e_caches = [QuantizedKVCache(cfg, device=device) for _ in range(n_rep)]
     K, V, _, _, _ = device_inputs(w, device, 1, rank)
-    for c in e_caches:
-        if turbo is not None:
+    if turbo is not None:
+        for c in e_caches:
             c.turbo_setup(*turbo)
+    # prefill (quantize + window copy) of the replicas, timed on the device:
+    # bytes = the K/V inputs read plus the packed records and window written
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for c in e_caches:
         c.prefill(K, V)
+    p1.record(stream)
+    torch.cuda.synchronize()
+    prefill_ms = p0.elapsed_time(p1) / n_rep
+    prefill_bytes = int(K.numel() * 2 + V.numel() * 2) + step_bytes(e_caches[0])
     del K, V
     torch.cuda.synchronize()
     e_bytes = 0
@@ -325,7 +335,7 @@ def run_gpu(args, w, rank, world):
     res = dict(ms=ms, bytes=total_bytes, attn_ms=attn_ms, launches=launches, clocks=clk.summary(),
                e2e_ms=e_ms, e2e_bytes=e_bytes, n_rep=n_rep, splits=caches[0].decode_splits,
                h2d=int(q[0].numel() * 2 + kn[0].numel() * 2 + vn[0].numel() * 2), d2h=int(out.numel() * 4),
-               step_bytes_last=attn_bytes // args.steps)
+               step_bytes_last=attn_bytes // args.steps, prefill_ms=prefill_ms, prefill_bytes=prefill_bytes)
     return res
 
 
@@ -447,6 +457,12 @@ def main():
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
         "gpu_launches": res["launches"], "clocks": res["clocks"], "replicas": res["n_rep"],
         "decode_splits": res["splits"],
+        # secondary: the prefill (quantize kernel + window copy) of one replica,
+        # algorithmic bytes = K/V inputs read + packed records and window written
+        "prefill": {"us": round(res["prefill_ms"] * 1e3, 1), "bytes": res["prefill_bytes"],
+                    "achieved": round(res["prefill_bytes"] / (res["prefill_ms"] * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "frac": round(res["prefill_bytes"] / (res["prefill_ms"] * 1e-3) / 1e9 / hbm, 4),
+                    "kernel": "tq_quantize_kernel" if w.scheme == "turbo" else "kivi_quantize_kernel"},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         samp = oracle_sample(w, args.cpu_budget)
