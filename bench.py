@@ -1,10 +1,11 @@
 #!/usr/bin/env python
 """Decode-step benchmark of the quantized KV cache (libkvq.so, one process per GPU).
 
-A step is one decode step of the whole batch: kvq_append_token (the new
-token enters the residual window; a flush quantizes G tokens when due) and
-kvq_decode_attention over the packed cache.  Metric: packed-KV bytes read by
-the decode attention per second (GB/s), with tokens/s alongside.
+A step is one decode step of the whole batch through kvq_append_decode: the
+new token enters the residual window (a flush quantizes G tokens when due) and
+the attention runs over the packed cache, in one kernel launch on steps that
+do not flush.  Metric: packed-KV bytes read by the decode attention per
+second (GB/s), with tokens/s alongside.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 8b2] [--impl kivi|reference]
 
@@ -216,10 +217,12 @@ def run_gpu(args, w, rank, world):
     vnp = [ptr(vn[i]) for i in range(steps_total)]
     outp = ptr(out)
 
+    # one decode step = append the new token + attend (kvq_append_decode: one
+    # launch, or quantize + attend on a step that flushes the window)
     def one_step(i):
         c = caches[i % n_rep]
-        L.check(lib.kvq_append_token(c.handle, knp[i], vnp[i], sp), "append")
-        L.check(lib.kvq_decode_attention(c.handle, qp[i], outp, scale, ptr(c.ws), c.ws.numel(), sp), "attention")
+        L.check(lib.kvq_append_decode(c.handle, knp[i], vnp[i], qp[i], outp, scale, ptr(c.ws), c.ws.numel(), sp),
+                "append_decode")
         return step_bytes(c)
 
     for i in range(args.warmup):
@@ -240,9 +243,8 @@ def run_gpu(args, w, rank, world):
             for j in range(args.steps):
                 i = args.warmup + j
                 c = caches[i % n_rep]
-                L.check(lib.kvq_append_token(c.handle, knp[i], vnp[i], csp), "append")
-                L.check(lib.kvq_decode_attention(c.handle, qp[i], outp, scale, ptr(c.ws), c.ws.numel(), csp),
-                        "attention")
+                L.check(lib.kvq_append_decode(c.handle, knp[i], vnp[i], qp[i], outp, scale, ptr(c.ws),
+                                              c.ws.numel(), csp), "append_decode")
                 total_bytes += step_bytes(c)
     launches = launch_count() - launches0
     # attention-only graph over the same replicas, for the per-launch kernel time
@@ -323,8 +325,7 @@ def run_gpu(args, w, rank, world):
         d_q.copy_(h_q[j], non_blocking=True)
         d_kn.copy_(h_kn[j], non_blocking=True)
         d_vn.copy_(h_vn[j], non_blocking=True)
-        c.append(d_kn, d_vn)
-        c.attention(d_q, out=out)
+        c.append_attention(d_kn, d_vn, d_q, out=out)
         h_out[j].copy_(out, non_blocking=True)
         e_bytes += step_bytes(c)
     e1.record(stream)

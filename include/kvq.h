@@ -101,7 +101,9 @@ typedef struct {
  * start).  For KIVI every (batch, kv head) row holds `groups_per_row` group
  * records of `record_bytes` each; a record packs G tokens: the key codes and
  * value codes of its 32-token blocks (16 INT2 or 8 INT4 codes per 32-bit word,
- * in the fragment order of the decode kernel), the fp16 (scale, zero) of each
+ * ordered so that a lane's word yields its mma fragments directly; the exact
+ * bit order is the packed format v1 the oracle also implements), the fp16
+ * (scale, zero) of each
  * key channel, and the fp16 (scale, zero) of each value token.  Each row also
  * owns a ring of `ring_tokens` 16-bit key rows and one of value rows (the
  * residual window).
@@ -189,6 +191,23 @@ kvq_status kvq_append_token(kvq_cache* cache, const void* k_new, const void* v_n
  */
 kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, float* out, float softmax_scale,
                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One whole decode step: kvq_append_token(cache, k_new, v_new) followed by
+ * kvq_decode_attention(cache, q, out, ...), with the same results, cache
+ * state and errors ([DEC]: the step on either side of the path).  When the
+ * appended token does not complete a flush, both run as one kernel launch:
+ * the attention reads the new token from k_new / v_new and stores it into the
+ * residual window itself.  A step that flushes the window's oldest G tokens
+ * quantizes them first, as kvq_append_token does, then attends.
+ *   k_new, v_new   device [B][Hkv][d], 16-bit (as for kvq_append_token).
+ *   q, out, softmax_scale, workspace, workspace_bytes, stream
+ *                  as for kvq_decode_attention.
+ * Errors: those of kvq_append_token and kvq_decode_attention, all detected
+ * before anything is launched; on an error the cache state is unchanged.
+ */
+kvq_status kvq_append_decode(kvq_cache* cache, const void* k_new, const void* v_new, const void* q, float* out,
+                             float softmax_scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Decode attention that allocates nothing and needs no workspace argument.

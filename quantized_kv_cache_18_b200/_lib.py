@@ -37,6 +37,7 @@ _SIGS = {
     "kvq_append_token": (ctypes.c_int, [_P, _P, _P, _P]),
     "kvq_decode_attention": (ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
     "kvq_decode_attention_static": (ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P]),
+    "kvq_append_decode": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),
     "kvq_get_status": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32, _P]),
     "kvq_seq_len": (ctypes.c_int32, [_P]),
     "kvq_quantized_len": (ctypes.c_int32, [_P]),

@@ -152,6 +152,25 @@ class QuantizedKVCache:
                                               self.ws.numel(), _stream_ptr(stream)), "kvq_decode_attention")
         return out
 
+    def append_attention(self, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+                         out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                         stream=None) -> torch.Tensor:
+        """append(k_new, v_new) then attention(q) as one decode step
+        (kvq_append_decode: one kernel launch unless the step flushes)."""
+        c = self.cfg
+        shape = (c.batch, c.num_kv_heads, c.head_dim)
+        self._check_16(k_new, shape, "k_new")
+        self._check_16(v_new, shape, "v_new")
+        self._check_16(q, (c.batch, c.num_q_heads, c.head_dim), "q")
+        if out is None:
+            out = torch.empty((c.batch, c.num_q_heads, c.head_dim), dtype=torch.float32, device=self.buf.device)
+        if scale is None:
+            scale = 1.0 / math.sqrt(c.head_dim)
+        L.check(self.lib.kvq_append_decode(self.handle, _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(out), float(scale),
+                                           _ptr(self.ws), self.ws.numel(), _stream_ptr(stream)),
+                "kvq_append_decode")
+        return out
+
     def status(self, clear: bool = False, stream=None) -> int:
         bits = ctypes.c_uint32(0)
         self.lib.kvq_get_status(self.handle, ctypes.byref(bits), 1 if clear else 0, _stream_ptr(stream))

@@ -373,11 +373,20 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
               const int n = min(kWinTok, a.r - t0);
               const int slot0 = (a.head + t0) % gm.cap;
               // two copies (key rows, value rows): a CTA's bulk copies complete
-              // roughly one after another, so few large copies beat many small ones
-              const uint32_t bytes = (uint32_t)n * D * 2;
-              mbar_expect_tx(&bar_full[slot], 2 * bytes);
-              bulk_g2s(dst, ring_ptr(gm, row, 0) + (int64_t)slot0 * D, bytes, &bar_full[slot]);
-              bulk_g2s(dst + kWinTok * C::WROW, ring_ptr(gm, row, 1) + (int64_t)slot0 * D, bytes, &bar_full[slot]);
+              // roughly one after another, so few large copies beat many small ones;
+              // with a fused append the chunk's last token comes from k_new / v_new
+              const bool fused = a.k_new != nullptr && t0 + n == a.r;
+              const int n_ring = fused ? n - 1 : n;
+              mbar_expect_tx(&bar_full[slot], 2u * (uint32_t)n * D * 2);
+              if (n_ring > 0) {
+                const uint32_t bytes = (uint32_t)n_ring * D * 2;
+                bulk_g2s(dst, ring_ptr(gm, row, 0) + (int64_t)slot0 * D, bytes, &bar_full[slot]);
+                bulk_g2s(dst + kWinTok * C::WROW, ring_ptr(gm, row, 1) + (int64_t)slot0 * D, bytes, &bar_full[slot]);
+              }
+              if (fused) {
+                bulk_g2s(dst + n_ring * C::WROW, a.k_new + (int64_t)row * D, D * 2, &bar_full[slot]);
+                bulk_g2s(dst + (kWinTok + n_ring) * C::WROW, a.v_new + (int64_t)row * D, D * 2, &bar_full[slot]);
+              }
             }
             issued = s + 1;
           },
@@ -740,6 +749,20 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
       *abort_flag = 1;
     }
     const unsigned char* st = smem + slot * C::STAGE;
+    if (ok && win && a.k_new != nullptr && cw == C::NC - 1) {
+      // fused append: the new token of this row (the chunk's last) into its ring slot
+      const int t0 = (int)first * kWinTok;
+      const int n = min(kWinTok, a.r - t0);
+      if (t0 + n == a.r) {
+        const int slot_new = (a.head + a.r - 1) % gm.cap;
+        constexpr int CH = D * 2 / 16;   // 16-byte chunks per row
+        if (lane < 2 * CH) {
+          const int part = lane / CH, ci = lane - part * CH;
+          const uint4 v = lds128(st + (part * kWinTok + n - 1) * C::WROW + 16 * ci);
+          reinterpret_cast<uint4*>(ring_ptr(gm, row, part) + (int64_t)slot_new * D)[ci] = v;
+        }
+      }
+    }
     if constexpr (TR) {
       if (ok && !win && cw < cnt * C::NTB) tr_block(st, slot);
       else if (ok && win) tr_window(st, first);

@@ -267,15 +267,22 @@ kvq_status kvq_append_token(kvq_cache* h, const void* k_new, const void* v_new, 
   return KVQ_OK;
 }
 
-kvq_status kvq_decode_attention(const kvq_cache* h, const void* q, float* out, float softmax_scale, void* workspace,
-                                size_t workspace_bytes, void* stream) {
+// Argument checks of a decode attention call (also those of the fused call).
+static kvq_status check_attention_args(const kvq_cache* h, const void* q, const float* out, float softmax_scale,
+                                       const void* workspace, size_t workspace_bytes) {
   if (!h || !q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
-  if (h->seq_len <= 0) return KVQ_ERR_INVALID_ARG;
   if (!(std::isfinite(softmax_scale))) return KVQ_ERR_INVALID_ARG;
+  if (workspace_bytes < kvq_workspace_bytes(&h->cfg)) return KVQ_ERR_INVALID_ARG;
+  if (h->cfg.scheme == KVQ_TURBO && !h->tq_ready) return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
+// Launches the attention over the cache state (T_q = h->tq, window of r tokens
+// from h->head); with k_new / v_new the window's last token is the new one.
+static kvq_status launch_attention(const kvq_cache* h, int r, const void* q, float* out, float softmax_scale,
+                                   void* workspace, cudaStream_t st, const void* k_new, const void* v_new) {
   const kvq_config& c = h->cfg;
-  if (workspace_bytes < kvq_workspace_bytes(&c)) return KVQ_ERR_INVALID_ARG;
-  if (c.scheme == KVQ_TURBO && !h->tq_ready) return KVQ_ERR_INVALID_ARG;
   AttnArgs a;
   a.geom = make_geom(h);
   a.q = static_cast<const uint16_t*>(q);
@@ -292,16 +299,46 @@ kvq_status kvq_decode_attention(const kvq_cache* h, const void* q, float* out, f
   a.counters = reinterpret_cast<unsigned*>(h->base + h->lay.status_offset) + 1;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.n_groups = h->tq / c.group;
-  a.n_cta = plan_ctas(c, a.n_groups, h->r);
-  a.r = h->r;
+  a.n_cta = plan_ctas(c, a.n_groups, r);
+  a.r = r;
   a.head = h->head;
+  a.k_new = static_cast<const uint16_t*>(k_new);
+  a.v_new = static_cast<const uint16_t*>(v_new);
   if (c.scheme == KVQ_TURBO) {
-    launch_tq_query_prep(a.geom, a.q, const_cast<unsigned char*>(a.qprep), (cudaStream_t)stream);
-    launch_tq_attention(a, (cudaStream_t)stream);
+    launch_tq_query_prep(a.geom, a.q, const_cast<unsigned char*>(a.qprep), st);
+    launch_tq_attention(a, st);
   } else {
-    launch_kivi_attention(a, (cudaStream_t)stream);
+    launch_kivi_attention(a, st);
   }
   if (check_launch() != KVQ_OK) return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention(const kvq_cache* h, const void* q, float* out, float softmax_scale, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  const kvq_status e = check_attention_args(h, q, out, softmax_scale, workspace, workspace_bytes);
+  if (e != KVQ_OK) return e;
+  if (h->seq_len <= 0) return KVQ_ERR_INVALID_ARG;
+  return launch_attention(h, h->r, q, out, softmax_scale, workspace, (cudaStream_t)stream, nullptr, nullptr);
+}
+
+kvq_status kvq_append_decode(kvq_cache* h, const void* k_new, const void* v_new, const void* q, float* out,
+                             float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  const kvq_status e = check_attention_args(h, q, out, softmax_scale, workspace, workspace_bytes);
+  if (e != KVQ_OK) return e;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
+  if (h->seq_len + 1 > h->cfg.max_seq) return KVQ_ERR_CAPACITY;
+  const int32_t r_new = h->r + 1;
+  if (r_new == h->cfg.residual + h->cfg.group) {
+    // a flush is due: the oldest G window tokens are quantized before the attention reads them
+    const kvq_status ea = kvq_append_token(h, k_new, v_new, stream);
+    if (ea != KVQ_OK) return ea;
+    return launch_attention(h, h->r, q, out, softmax_scale, workspace, (cudaStream_t)stream, nullptr, nullptr);
+  }
+  const kvq_status el = launch_attention(h, r_new, q, out, softmax_scale, workspace, (cudaStream_t)stream, k_new, v_new);
+  if (el != KVQ_OK) return el;
+  h->r = r_new;
+  h->seq_len += 1;
   return KVQ_OK;
 }
 

@@ -218,6 +218,11 @@ struct AttnArgs {
   int n_cta;               // CTAs of the launch (one per SM at most)
   int r;                   // window tokens
   int head;                // ring slot of the oldest window token
+  // Fused append (or null): window token r - 1 is the new token of each row,
+  // read from k_new / v_new ([B][Hkv][d]) instead of the ring, and the CTA
+  // that attends it also stores it into ring slot (head + r - 1) % cap.
+  const uint16_t* k_new;
+  const uint16_t* v_new;
 };
 
 void launch_kivi_quantize(const QuantArgs& a, cudaStream_t st);

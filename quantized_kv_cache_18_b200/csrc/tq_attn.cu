@@ -224,10 +224,19 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
               const int t0 = (int)first * kTqWin;
               const int n = min(kTqWin, a.r - t0);
               const int slot0 = (a.head + t0) % gm.cap;
-              const uint32_t bytes = (uint32_t)n * D * 2;
-              mbar_expect_tx(&bar_full[slot], 2 * bytes);
-              bulk_g2s(dst, ring_ptr(gm, row, 0) + (int64_t)slot0 * D, bytes, &bar_full[slot]);
-              bulk_g2s(dst + kTqWin * C::WROW, ring_ptr(gm, row, 1) + (int64_t)slot0 * D, bytes, &bar_full[slot]);
+              // with a fused append the chunk's last token comes from k_new / v_new
+              const bool fused = a.k_new != nullptr && t0 + n == a.r;
+              const int n_ring = fused ? n - 1 : n;
+              mbar_expect_tx(&bar_full[slot], 2u * (uint32_t)n * D * 2);
+              if (n_ring > 0) {
+                const uint32_t bytes = (uint32_t)n_ring * D * 2;
+                bulk_g2s(dst, ring_ptr(gm, row, 0) + (int64_t)slot0 * D, bytes, &bar_full[slot]);
+                bulk_g2s(dst + kTqWin * C::WROW, ring_ptr(gm, row, 1) + (int64_t)slot0 * D, bytes, &bar_full[slot]);
+              }
+              if (fused) {
+                bulk_g2s(dst + n_ring * C::WROW, a.k_new + (int64_t)row * D, D * 2, &bar_full[slot]);
+                bulk_g2s(dst + (kTqWin + n_ring) * C::WROW, a.v_new + (int64_t)row * D, D * 2, &bar_full[slot]);
+              }
             }
             issued = s + 1;
           },
@@ -331,7 +340,6 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
   };
 
   auto chunk = [&](int s, int row, bool win, int64_t first, int cnt) {
-    (void)row;
     const int slot = s % C::NST;
     const uint32_t par = (s / C::NST) & 1;
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_full[slot], par, abort_flag));
@@ -340,6 +348,20 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
       *abort_flag = 1;
     }
     const unsigned char* st = smem + slot * C::STAGE;
+    if (ok && win && a.k_new != nullptr && cw == kTqConsumers - 1) {
+      // fused append: the new token of this row (the chunk's last) into its ring slot
+      const int t0 = (int)first * kTqWin;
+      const int n = min(kTqWin, a.r - t0);
+      if (t0 + n == a.r) {
+        const int slot_new = (a.head + a.r - 1) % gm.cap;
+        constexpr int CH = D * 2 / 16;   // 16-byte chunks per row
+        if (lane < 2 * CH) {
+          const int part = lane / CH, ci = lane - part * CH;
+          const uint4 v = lds128(st + (part * kTqWin + n - 1) * C::WROW + 16 * ci);
+          reinterpret_cast<uint4*>(ring_ptr(gm, row, part) + (int64_t)slot_new * D)[ci] = v;
+        }
+      }
+    }
     if (ok && !win && cw < cnt) {
       // ---------------------------------------------------------- one token block
       const unsigned char* tb = st + cw * kTqTbBytes;
