@@ -29,6 +29,10 @@ sketch of m = 128 Gaussian rows on keys only, per-vector fp16 norms):
 * values: v_hat = n Pi^T c_hat, so sum_t p_t v_hat_t = Pi^T sum_t p_t n_t c_hat_t;
 * Pi is the Q factor of the QR decomposition of a seeded N(0, 1) d x d draw with
   the signs fixed so that diag(R) > 0 (unique); S is a seeded N(0, 1) m x d draw.
+* Walsh-Hadamard variant ("TurboQuant : les cinq innovations", item 1 names a
+  Walsh-Hadamard transform as the rotation): Pi = H_d / sqrt(d) with H_d the
+  Sylvester-order Hadamard matrix, no random sign flips (the page describes the
+  plain transform); every other step is unchanged.
 """
 from __future__ import annotations
 
@@ -87,6 +91,17 @@ def rotation(gauss: np.ndarray) -> np.ndarray:
     sgn = np.sign(np.diag(r))
     sgn[sgn == 0] = 1.0
     return q * sgn[None, :]
+
+
+def rotation_wht(d: int) -> np.ndarray:
+    """Walsh-Hadamard rotation H_d / sqrt(d), float64, with H_1 = [1] and
+    H_2n = [[H_n, H_n], [H_n, -H_n]] (Sylvester order); d a power of two."""
+    if d < 1 or d & (d - 1):
+        raise ValueError("d must be a power of two")
+    h = np.ones((1, 1))
+    while h.shape[0] < d:
+        h = np.block([[h, h], [h, -h]])
+    return h / math.sqrt(d)
 
 
 # ------------------------------------------------------------------ quantizer

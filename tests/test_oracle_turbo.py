@@ -99,6 +99,53 @@ def test_rotation_preserves_norms_and_spreads_outliers():
     assert np.median(ratio(x)) > 7.0 and np.median(ratio(y)) < 4.0
 
 
+def _fwht(x):
+    """Textbook in-place fast Walsh-Hadamard transform (butterflies of span
+    1, 2, 4, ...) along the last axis, unnormalised."""
+    x = np.array(x, np.float64)
+    n = x.shape[-1]
+    h = 1
+    while h < n:
+        for i in range(0, n, 2 * h):
+            a = x[..., i:i + h].copy()
+            b = x[..., i + h:i + 2 * h].copy()
+            x[..., i:i + h] = a + b
+            x[..., i + h:i + 2 * h] = a - b
+        h *= 2
+    return x
+
+
+@pytest.mark.parametrize("d", [1, 2, 4, 64, 128])
+def test_wht_rotation_is_scipys_hadamard_normalised(d):
+    from scipy.linalg import hadamard
+    assert np.array_equal(turbo.rotation_wht(d) * math.sqrt(d), hadamard(d).astype(np.float64))
+
+
+def test_wht_rotation_is_an_orthogonal_involution_and_the_fast_transform():
+    pi = turbo.rotation_wht(128)
+    assert np.abs(pi.T @ pi - np.eye(128)).max() < 1e-14
+    assert np.abs(pi @ pi - np.eye(128)).max() < 1e-14          # symmetric: its own inverse
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((7, 128))
+    assert np.abs(x @ pi.T - _fwht(x) / math.sqrt(128)).max() < 1e-12
+
+
+def test_wht_rotation_spreads_an_outlier():
+    pi = turbo.rotation_wht(128)
+    # a single spike becomes a flat vector of the same norm
+    y = pi @ np.eye(128)[:, 37]
+    assert np.allclose(np.abs(y), 1 / math.sqrt(128))
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((200, 128))
+    x[:, [5, 77]] *= 20.0
+    y = x @ pi.T
+    ratio = lambda v: np.abs(v).max(axis=1) / np.sqrt((v * v).mean(axis=1))
+    assert np.allclose(np.linalg.norm(x, axis=1), np.linalg.norm(y, axis=1))
+    assert np.median(ratio(x)) > 7.0 and np.median(ratio(y)) < 4.0
+    with pytest.raises(ValueError):
+        turbo.rotation_wht(96)
+
+
 # ------------------------------------------------------------------ quantizer
 def _params(d=128, m=128, seed=3):
     rng = np.random.default_rng(seed)
