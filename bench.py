@@ -183,7 +183,8 @@ def run_gpu(args, w, rank, world):
     import torch
     from quantized_kv_cache_18_b200 import build as kbuild
     from quantized_kv_cache_18_b200 import _lib as L
-    from quantized_kv_cache_18_b200.cache import QuantizedKVCache, config_from_workload, launch_count
+    from quantized_kv_cache_18_b200.cache import (QuantizedKVCache, config_from_workload, launch_count,
+                                                   turbo_setup_from_workload)
 
     kbuild.build()
     device = torch.device("cuda", torch.cuda.current_device())
@@ -195,14 +196,10 @@ def run_gpu(args, w, rank, world):
     probe = QuantizedKVCache(cfg, device=device)
     n_rep = max(2, math.ceil(3 * l2 / probe.nbytes) + 1)
     caches = [probe] + [QuantizedKVCache(cfg, device=device) for _ in range(n_rep - 1)]
-    turbo = None
-    if w.scheme == "turbo":
-        from quantized_kv_cache_18_b200 import workloads as W
-        turbo = (torch.from_numpy(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)).to(device),
-                 torch.from_numpy(W.gaussian_matrix(w, "qjl", w.qjl_dim, w.head_dim)).to(device))
+    turbo = w.scheme == "turbo"
     for c in caches:
-        if turbo is not None:
-            c.turbo_setup(*turbo)
+        if turbo:
+            turbo_setup_from_workload(c, w)
         c.prefill(K, V)
     del K, V
     torch.cuda.synchronize()
@@ -301,9 +298,9 @@ def run_gpu(args, w, rank, world):
     d_q, d_kn, d_vn = torch.empty_like(q[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
     e_caches = [QuantizedKVCache(cfg, device=device) for _ in range(n_rep)]
     K, V, _, _, _ = device_inputs(w, device, 1, rank)
-    if turbo is not None:
+    if turbo:
         for c in e_caches:
-            c.turbo_setup(*turbo)
+            turbo_setup_from_workload(c, w)
     # prefill (quantize + window copy) of the replicas, timed on the device:
     # bytes = the K/V inputs read plus the packed records and window written
     torch.cuda.synchronize()
@@ -353,7 +350,8 @@ def oracle_sample(w, budget_s: float, steps: int = 1):
     from quantized_kv_cache_18_b200 import workloads as W
 
     if w.scheme == "turbo":
-        tq_params = (turbo.rotation(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)),
+        tq_params = (turbo.rotation_wht(w.head_dim) if w.rotation == "wht"
+                     else turbo.rotation(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)),
                      W.gaussian_matrix(w, "qjl", w.qjl_dim, w.head_dim).astype(np.float64),
                      *turbo.deployed_codebook(w.head_dim))
 

@@ -148,14 +148,27 @@ kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes,
  * deployment constants of [TQ] on the device and stores them in the cache
  * buffer:
  *   rot_gauss  device float32 [d][d]: a seeded N(0,1) draw; the rotation is
- *              the Q factor of its QR decomposition with diag(R) > 0
- *              ("rotation orthogonale aleatoire").
+ *              the Q factor of its QR decomposition with diag(R) > 0, a random
+ *              orthogonal matrix as [TQ] asks for.
  *   qjl_gauss  device float32 [m][d]: the N(0,1) QJL projection S, used as is.
  * The 8-level Lloyd-Max codebook for N(0, 1/d) ("TurboQuant : les cinq
  * innovations", item 2) is computed on the device as well.
+ * Errors: KVQ_ERR_UNSUPPORTED for a KIVI cache; KVQ_ERR_INVALID_ARG for null
+ * or misaligned pointers or a cache that already holds tokens.
  */
 kvq_status kvq_turbo_setup(kvq_cache* cache, const float* rot_gauss, const float* qjl_gauss,
                            void* stream);
+
+/*
+ * As kvq_turbo_setup, with the Walsh-Hadamard rotation instead of a random
+ * one ("TurboQuant : les cinq innovations", item 1): Pi = H_d / sqrt(d), H_d
+ * the Sylvester-order Hadamard matrix (entry (i, j) = (-1)^popcount(i & j)),
+ * stored as exactly +-fp32(1 / sqrt(d)).  The quantizer then applies Pi with
+ * the fast transform (add/sub butterflies) instead of a d x d product.
+ *   qjl_gauss  device float32 [m][d], as for kvq_turbo_setup.
+ * Errors: as kvq_turbo_setup.
+ */
+kvq_status kvq_turbo_setup_wht(kvq_cache* cache, const float* qjl_gauss, void* stream);
 
 /*
  * Prefill ([KIVI] / [TQ]).  k, v: device [B][Hkv][seq_len][d], 16-bit.

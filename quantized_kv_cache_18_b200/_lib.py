@@ -33,6 +33,7 @@ _SIGS = {
     "kvq_get_layout": (ctypes.c_int, [ctypes.POINTER(KvqConfig), ctypes.POINTER(KvqLayout)]),
     "kvq_cache_init": (ctypes.c_int, [ctypes.POINTER(KvqConfig), _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
     "kvq_turbo_setup": (ctypes.c_int, [_P, _P, _P, _P]),
+    "kvq_turbo_setup_wht": (ctypes.c_int, [_P, _P, _P]),
     "kvq_quantize_prefill": (ctypes.c_int, [_P, _P, _P, ctypes.c_int32, _P]),
     "kvq_append_token": (ctypes.c_int, [_P, _P, _P, _P]),
     "kvq_decode_attention": (ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),

@@ -116,6 +116,17 @@ class QuantizedKVCache:
         L.check(self.lib.kvq_turbo_setup(self.handle, _ptr(rot_gauss), _ptr(qjl_gauss), _stream_ptr(stream)),
                 "kvq_turbo_setup")
 
+    def turbo_setup_wht(self, qjl_gauss: torch.Tensor, stream=None):
+        """TurboQuant scheme with the Walsh-Hadamard rotation H / sqrt(d): the
+        codebook and sketch tables from the [m][d] float32 N(0, 1) draw."""
+        c = self.cfg
+        if qjl_gauss.device != self.buf.device or qjl_gauss.dtype != torch.float32 or not qjl_gauss.is_contiguous():
+            raise ValueError(f"qjl_gauss: needs a contiguous float32 tensor on {self.buf.device}")
+        if tuple(qjl_gauss.shape) != (c.qjl_dim, c.head_dim):
+            raise ValueError(f"qjl_gauss: shape {tuple(qjl_gauss.shape)} != {(c.qjl_dim, c.head_dim)}")
+        L.check(self.lib.kvq_turbo_setup_wht(self.handle, _ptr(qjl_gauss), _stream_ptr(stream)),
+                "kvq_turbo_setup_wht")
+
     # ------------------------------------------------------------------ the three calls
     def _check_16(self, t: torch.Tensor, shape, what: str):
         if t.device != self.buf.device or not t.is_contiguous() or t.element_size() != 2:
@@ -199,3 +210,16 @@ class QuantizedKVCache:
 
 def launch_count() -> int:
     return int(L.load().kvq_launch_count())
+
+
+def turbo_setup_from_workload(cache: "QuantizedKVCache", w, stream=None):
+    """TurboQuant set-up of a cache with the workload's seeded draws: the QR
+    rotation from the [d][d] draw, or the Walsh-Hadamard one (w.rotation)."""
+    from . import workloads as W
+    dev = cache.buf.device
+    qjl = torch.from_numpy(W.gaussian_matrix(w, "qjl", w.qjl_dim, w.head_dim)).to(dev)
+    if w.rotation == "wht":
+        cache.turbo_setup_wht(qjl, stream)
+    else:
+        rot = torch.from_numpy(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)).to(dev)
+        cache.turbo_setup(rot, qjl, stream)

@@ -20,6 +20,7 @@ struct kvq_cache {
   int32_t r;
   int32_t head;
   bool tq_ready;   // TURBO: the parameter block holds the deployment constants
+  bool tq_wht;     // TURBO: the rotation is the Walsh-Hadamard one
 };
 
 namespace kvq {
@@ -93,6 +94,7 @@ static Geom make_geom(const kvq_cache* h) {
   Geom g;
   const kvq_config& c = h->cfg;
   g.scheme = c.scheme;
+  g.rot_wht = h->tq_wht ? 1 : 0;
   g.d = c.head_dim;
   g.bits = c.bits;
   g.G = c.group;
@@ -182,6 +184,7 @@ kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes, vo
   h->base = static_cast<char*>(dev_buf);
   h->seq_len = h->tq = h->r = h->head = 0;
   h->tq_ready = false;
+  h->tq_wht = false;
   launch_clear_words(reinterpret_cast<uint32_t*>(h->base + L.status_offset),
                      1 + cfg->batch * cfg->num_kv_heads, (cudaStream_t)stream);
   if (check_launch() != KVQ_OK) {
@@ -197,7 +200,20 @@ kvq_status kvq_turbo_setup(kvq_cache* h, const float* rot_gauss, const float* qj
   if (h->cfg.scheme != KVQ_TURBO) return KVQ_ERR_UNSUPPORTED;
   if (!aligned16(rot_gauss) || !aligned16(qjl_gauss)) return KVQ_ERR_INVALID_ARG;
   if (h->seq_len != 0) return KVQ_ERR_INVALID_ARG;
-  launch_turbo_setup(make_geom(h), rot_gauss, qjl_gauss, (cudaStream_t)stream);
+  h->tq_wht = false;
+  launch_turbo_setup(make_geom(h), rot_gauss, qjl_gauss, false, (cudaStream_t)stream);
+  if (check_launch() != KVQ_OK) return KVQ_ERR_CUDA;
+  h->tq_ready = true;
+  return KVQ_OK;
+}
+
+kvq_status kvq_turbo_setup_wht(kvq_cache* h, const float* qjl_gauss, void* stream) {
+  if (!h || !qjl_gauss) return KVQ_ERR_INVALID_ARG;
+  if (h->cfg.scheme != KVQ_TURBO) return KVQ_ERR_UNSUPPORTED;
+  if (!aligned16(qjl_gauss)) return KVQ_ERR_INVALID_ARG;
+  if (h->seq_len != 0) return KVQ_ERR_INVALID_ARG;
+  h->tq_wht = true;
+  launch_turbo_setup(make_geom(h), nullptr, qjl_gauss, true, (cudaStream_t)stream);
   if (check_launch() != KVQ_OK) return KVQ_ERR_CUDA;
   h->tq_ready = true;
   return KVQ_OK;

@@ -40,6 +40,7 @@ constexpr int kMaxDecodeCtas = 160;   // decode launches use at most this many C
 
 struct Geom {
   int scheme, d, bits, G, R, cap, B, Hkv, Hq, g, dtype;
+  int rot_wht;              // TURBO: Pi is the Walsh-Hadamard rotation H / sqrt(d)
   int64_t groups_per_row;   // record capacity of a row
   int64_t rec_bytes;        // bytes of one group record
   int64_t tb_code_bytes;    // bytes of one TB's key (or value) codes
@@ -231,7 +232,7 @@ void launch_window_copy(const Geom& g, const uint16_t* k, const uint16_t* v, int
 void launch_append(const Geom& g, const uint16_t* k, const uint16_t* v, int slot, cudaStream_t st);
 void launch_kivi_attention(const AttnArgs& a, cudaStream_t st);
 void launch_clear_words(uint32_t* words, int n, cudaStream_t st);
-void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_gauss, cudaStream_t st);
+void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_gauss, bool wht, cudaStream_t st);
 void launch_tq_quantize(const QuantArgs& a, cudaStream_t st);
 void launch_tq_query_prep(const Geom& g, const uint16_t* q, unsigned char* qprep, cudaStream_t st);
 void launch_tq_attention(const AttnArgs& a, cudaStream_t st);

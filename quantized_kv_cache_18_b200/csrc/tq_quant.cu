@@ -16,7 +16,9 @@
 //
 // One persistent CTA per SM keeps Pi^T and S^T (fp32, 64 KB each) in shared
 // memory and loops over (row, block) tasks.  Each task runs three 32 x 128 x 128
-// products on the CUDA cores (keys: Pi U and S E, values: Pi U).
+// products on the CUDA cores (keys: Pi U and S E, values: Pi U); with the
+// Walsh-Hadamard rotation, Pi U is the in-register fast transform instead
+// (7 add/sub stages per vector), leaving S E as the one product.
 #include <cuda_runtime.h>
 
 #include "kvq_internal.cuh"
@@ -67,9 +69,30 @@ __device__ __forceinline__ void matvec_tile(const float* WT, const float* X, int
   }
 }
 
+// In-register Walsh-Hadamard transform (Sylvester order, unnormalised) of a
+// 128-vector held as element lane + 32 r in v[r]: butterflies of span 1..16
+// across lanes, of span 32 and 64 across the four registers.
+__device__ __forceinline__ void fwht128(float v[4], int lane) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float p = __shfl_xor_sync(0xffffffffu, v[r], h);
+      v[r] = (lane & h) ? p - v[r] : v[r] + p;
+    }
+  }
+  const float a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
+  v[0] = a0 + a2;
+  v[2] = a0 - a2;
+  v[1] = a1 + a3;
+  v[3] = a1 - a3;
+}
+
 // Norms and unit vectors of the 32 tokens in X: warp w handles tokens 4w..4w+3.
+// With wht, U receives y = H u / sqrt(d) instead of u (the rotation applied by
+// the fast transform; Pi = H / sqrt(d) holds exactly +-fp32(1 / sqrt(d))).
 __device__ __forceinline__ uint32_t unit_vectors(const uint16_t* X, float* U, double* nrm, int dtype, int warp,
-                                                 int lane) {
+                                                 int lane, bool wht) {
   uint32_t flags = 0;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -84,8 +107,17 @@ __device__ __forceinline__ uint32_t unit_vectors(const uint16_t* X, float* U, do
     }
     const double n = sqrt(warp_sum_d(s));
     const double inv = n > 0.0 ? 1.0 / n : 0.0;
+    float u[4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) U[(lane + 32 * r) * kTok + t] = (float)((double)x[r] * inv);
+    for (int r = 0; r < 4; ++r) u[r] = (float)((double)x[r] * inv);
+    if (wht) {
+      fwht128(u, lane);
+      const float c = (float)(1.0 / sqrt((double)kTqD));
+#pragma unroll
+      for (int r = 0; r < 4; ++r) u[r] *= c;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) U[(lane + 32 * r) * kTok + t] = u[r];
     if (lane == 0) nrm[t] = n;
   }
   return flags;
@@ -137,11 +169,22 @@ __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) 
       for (int i = tid; i < kTok * kTqD / 8; i += kQThreads)
         reinterpret_cast<uint4*>(sX)[i] = ldg_nc_v4(reinterpret_cast<const uint4*>(src) + i);
       __syncthreads();
-      flags |= unit_vectors(sX, sU, kv == 0 ? sNK : sNV, gm.dtype, warp, lane);
+      flags |= unit_vectors(sX, sU, kv == 0 ? sNK : sNV, gm.dtype, warp, lane, gm.rot_wht != 0);
       __syncthreads();
       // ---------------------------------------------------------- y = Pi u, codes
       float acc[4][4];
-      matvec_tile(sPiT, sU, ti, tt, acc);
+      if (gm.rot_wht) {
+#pragma unroll
+        for (int a4 = 0; a4 < 4; ++a4) {
+          const float4 y4 = *reinterpret_cast<const float4*>(sU + (4 * ti + a4) * kTok + 4 * tt);
+          acc[a4][0] = y4.x;
+          acc[a4][1] = y4.y;
+          acc[a4][2] = y4.z;
+          acc[a4][3] = y4.w;
+        }
+      } else {
+        matvec_tile(sPiT, sU, ti, tt, acc);
+      }
       uint8_t* codes = kv == 0 ? sCK : sCV;
       double esq[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll

@@ -4,7 +4,8 @@
 // decomposition of a seeded N(0, 1) draw, with the sign of each column fixed so
 // that diag(R) > 0 ("Quantification du KV-Cache : TurboQuant et l'etat de l'art
 // en 2026", "TurboQuant : les cinq innovations", item 1; zubnet.ai survey,
-// "Famille deux ...").  Each rotated coordinate then has the law N(0, 1/d), and
+// "Famille deux ..."), or, in the Walsh-Hadamard variant that item 1 names,
+// H_d / sqrt(d) in Sylvester order.  Each rotated coordinate then has the law N(0, 1/d), and
 // the scalar quantizer is the 8-level Lloyd-Max quantizer of that law, fixed at
 // deployment (same page, item 2): levels are the Lloyd-Max levels of N(0, 1)
 // scaled by 1/sqrt(d) and stored in fp16, thresholds are the midpoints of
@@ -36,7 +37,7 @@ __device__ __forceinline__ double warp_sum_d(double x) {
 // 2 / (v_k . v_k) (0 for an identity step) and rdiag[k] = R[k][k].
 __global__ void __launch_bounds__(kSetupThreads, 1)
     turbo_setup_kernel(const float* __restrict__ rot_gauss, const float* __restrict__ qjl_gauss,
-                       unsigned char* __restrict__ params, uint32_t* status) {
+                       unsigned char* __restrict__ params, uint32_t* status, int wht) {
   constexpr int D = kTqD, M = kTqM;
   extern __shared__ __align__(16) double A[];   // [D][D]
   __shared__ double tau[D], rdiag[D];
@@ -47,6 +48,19 @@ __global__ void __launch_bounds__(kSetupThreads, 1)
   __syncthreads();
 
   uint32_t flags = 0;
+  float* Pi = reinterpret_cast<float*>(params + kTqPi);
+  float* PiT = reinterpret_cast<float*>(params + kTqPiT);
+  if (wht) {
+    // Walsh-Hadamard rotation: Pi[i][j] = (-1)^popcount(i & j) / sqrt(d)
+    // (Sylvester order), exactly +-fp32(1 / sqrt(d)); symmetric, so Pi^T = Pi
+    const float c = (float)(1.0 / sqrt((double)D));
+    for (int e = tid; e < D * D; e += kSetupThreads) {
+      const int i = e / D, j = e - i * D;
+      const float v = (__popc(i & j) & 1) ? -c : c;
+      Pi[e] = v;
+      PiT[e] = v;
+    }
+  } else {
   for (int e = tid; e < D * D; e += kSetupThreads) {
     const int i = e / D, j = e - i * D;
     const float g = rot_gauss[e];   // row-major [i][j]
@@ -89,8 +103,6 @@ __global__ void __launch_bounds__(kSetupThreads, 1)
   }
 
   // ---------------------------------------------------------------- Q = H_0 H_1 ... H_{D-1}, column by column
-  float* Pi = reinterpret_cast<float*>(params + kTqPi);
-  float* PiT = reinterpret_cast<float*>(params + kTqPiT);
   for (int j = warp; j < D; j += NW) {
     double x[D / 32];
 #pragma unroll
@@ -121,6 +133,7 @@ __global__ void __launch_bounds__(kSetupThreads, 1)
       PiT[j * D + i] = v;
     }
   }
+  }   // QR rotation
 
   // ---------------------------------------------------------------- S^T
   float* ST = reinterpret_cast<float*>(params + kTqST);
@@ -266,14 +279,14 @@ __global__ void __launch_bounds__(kPrepThreads)
 
 }  // namespace
 
-void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_gauss, cudaStream_t st) {
+void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_gauss, bool wht, cudaStream_t st) {
   const int smem = kTqD * kTqD * (int)sizeof(double);
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(turbo_setup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     attr_set = true;
   }
-  turbo_setup_kernel<<<1, kSetupThreads, smem, st>>>(rot_gauss, qjl_gauss, g.params, g.status);
+  turbo_setup_kernel<<<1, kSetupThreads, smem, st>>>(rot_gauss, qjl_gauss, g.params, g.status, wht ? 1 : 0);
   count_launch(1);
 }
 

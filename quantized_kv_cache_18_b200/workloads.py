@@ -49,6 +49,7 @@ class Workload:
     v_outlier_scale: float = 10.0
     v_channel_outliers: bool = False          # TurboQuant: V gets the K channel recipe
     qjl_dim: int = 128
+    rotation: str = "qr"                      # TurboQuant: "qr" (random orthogonal) or "wht"
     seed: int = 0
 
     @property
@@ -78,6 +79,9 @@ WORKLOADS: Dict[str, Workload] = {
     # TurboQuant-style 3-bit: 32 q heads, 8 kv heads, batch 8, 32768 tokens.
     "tq": Workload("tq", "turbo", 8, 8, 32, 128, 32768, "bf16", 3, 32, 128,
                    v_outlier_frac=0.0, v_channel_outliers=True, seed=4),
+    # The same with the Walsh-Hadamard rotation H / sqrt(d) instead of the QR one.
+    "tqw": Workload("tqw", "turbo", 8, 8, 32, 128, 32768, "bf16", 3, 32, 128,
+                    v_outlier_frac=0.0, v_channel_outliers=True, rotation="wht", seed=4),
 }
 
 

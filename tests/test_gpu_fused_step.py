@@ -12,7 +12,7 @@ import torch
 
 from gpu_util import check_row_attention, check_row_bits, gpu_prefill, oracle_row, to_dev
 from quantized_kv_cache_18_b200 import workloads as W
-from quantized_kv_cache_18_b200.cache import QuantizedKVCache, config_from_workload
+from quantized_kv_cache_18_b200.cache import QuantizedKVCache, config_from_workload, turbo_setup_from_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -68,15 +68,13 @@ def test_fused_step_matches_two_calls_and_oracle(name, kw, S, steps):
 
 def _turbo_cache(w, max_seq):
     cache = QuantizedKVCache(config_from_workload(w, max_seq))
-    rot = torch.from_numpy(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)).cuda()
-    qjl = torch.from_numpy(W.gaussian_matrix(w, "qjl", w.qjl_dim, w.head_dim)).cuda()
-    cache.turbo_setup(rot, qjl)
+    turbo_setup_from_workload(cache, w)
     return cache
 
 
-@pytest.mark.parametrize("S,steps", [(480, 72), (5, 40)])
-def test_fused_step_turbo_matches_two_calls(S, steps):
-    w = W.with_sizes(W.WORKLOADS["tq"], batch=1, num_kv_heads=2, num_q_heads=8, seq_len=S, decode_steps=steps)
+@pytest.mark.parametrize("name,S,steps", [("tq", 480, 72), ("tq", 5, 40), ("tqw", 480, 40)])
+def test_fused_step_turbo_matches_two_calls(name, S, steps):
+    w = W.with_sizes(W.WORKLOADS[name], batch=1, num_kv_heads=2, num_q_heads=8, seq_len=S, decode_steps=steps)
     K, V = W.prefill(w, seq_len=S)
     fused, split = _turbo_cache(w, S + steps + 1), _turbo_cache(w, S + steps + 1)
     for c in (fused, split):

@@ -28,7 +28,7 @@ from oracle import turbo, turbo_cache
 from oracle.numerics import decode16, fp16_bits
 from quantized_kv_cache_18_b200 import workloads as W
 from quantized_kv_cache_18_b200._lib import KVQ_DEV_NONFINITE_INPUT
-from quantized_kv_cache_18_b200.cache import QuantizedKVCache, config_from_workload
+from quantized_kv_cache_18_b200.cache import QuantizedKVCache, config_from_workload, turbo_setup_from_workload
 
 from gpu_util import ATOL, REL_L2, to_dev
 
@@ -44,7 +44,8 @@ SMALL = W.with_sizes(TQ, batch=1, num_kv_heads=2, num_q_heads=8, seq_len=480, de
 
 # ------------------------------------------------------------------ helpers
 def oracle_params(w):
-    Pi = turbo.rotation(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim))
+    Pi = (turbo.rotation_wht(w.head_dim) if w.rotation == "wht"
+          else turbo.rotation(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)))
     S = W.gaussian_matrix(w, "qjl", w.qjl_dim, w.head_dim).astype(np.float64)
     lv, th = turbo.deployed_codebook(w.head_dim)
     return Pi, S, lv, th
@@ -52,9 +53,7 @@ def oracle_params(w):
 
 def gpu_cache(w, max_seq=None):
     cache = QuantizedKVCache(config_from_workload(w, max_seq))
-    rot = torch.from_numpy(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)).cuda()
-    qjl = torch.from_numpy(W.gaussian_matrix(w, "qjl", w.qjl_dim, w.head_dim)).cuda()
-    cache.turbo_setup(rot, qjl)
+    turbo_setup_from_workload(cache, w)
     return cache
 
 
@@ -210,6 +209,34 @@ def test_setup_tables_match_the_oracle():
     idx = np.arange(64)
     want = fp16_bits(lv)[idx & 7].astype(np.uint32) | (fp16_bits(lv)[idx >> 3].astype(np.uint32) << 16)
     assert np.array_equal(lut, want)
+
+
+# ------------------------------------------------------------------ Walsh-Hadamard rotation
+SMALL_WHT = W.with_sizes(SMALL, rotation="wht")
+
+
+def test_wht_setup_tables_are_exact():
+    w = SMALL_WHT
+    cache = gpu_cache(w)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    p = cache.params_view().cpu().numpy()
+    d = w.head_dim
+    f32 = p[:3 * d * d * 4].view(np.float32)
+    gpi, gpit = f32[:d * d].reshape(d, d), f32[d * d:2 * d * d].reshape(d, d)
+    # exactly the oracle's H / sqrt(d) rounded to fp32 (entries +-fp32(1/sqrt(d)))
+    assert np.array_equal(gpi, turbo.rotation_wht(d).astype(np.float32))
+    assert np.array_equal(gpit, gpi)
+    assert np.array_equal(f32[2 * d * d:].reshape(d, d), W.gaussian_matrix(w, "qjl", w.qjl_dim, d).T)
+
+
+def test_wht_small_prefill_and_appends():
+    run_case(SMALL_WHT, 480, appends=72)
+
+
+@pytest.mark.parametrize("seq_len", [1, 33, 161])
+def test_wht_window_edges(seq_len):
+    run_case(SMALL_WHT, seq_len, appends=40)
 
 
 def test_turbo_calls_need_setup():
