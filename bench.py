@@ -183,7 +183,7 @@ def run_gpu(args, w, rank, world):
     import torch
     from quantized_kv_cache_18_b200 import build as kbuild
     from quantized_kv_cache_18_b200 import _lib as L
-    from quantized_kv_cache_18_b200.cache import (QuantizedKVCache, config_from_workload, launch_count,
+    from quantized_kv_cache_18_b200.cache import (QuantizedKVCache, config_from_workload, launch_count, layout,
                                                    turbo_setup_from_workload)
 
     kbuild.build()
@@ -191,11 +191,32 @@ def run_gpu(args, w, rank, world):
     steps_total = args.warmup + args.steps
     max_seq = w.seq_len + steps_total + 1
     cfg = config_from_workload(w, max_seq)
+    P = args.page_records
+    if P > 0:
+        # paged caches: a pool with exactly the pages the rows need, each row's
+        # block table a random slice of a permutation of the pool
+        gpr = layout(cfg).groups_per_row
+        ppr = (gpr + P - 1) // P
+        rows = w.batch * w.num_kv_heads
+        cfg = config_from_workload(w, max_seq, P, rows * ppr)
+        tables = []
+
+    def new_cache():
+        c = QuantizedKVCache(cfg, device=device)
+        if P > 0:
+            g = torch.Generator().manual_seed(rank_seed(w, rank) + len(tables))
+            perm = (torch.randperm(rows * ppr, generator=g) if args.page_order == "shuffled"
+                    else torch.arange(rows * ppr))
+            t = perm.to(torch.int32).view(rows, ppr).to(device)
+            tables.append(t)
+            c.set_page_table(t)
+        return c
+
     K, V, q, kn, vn = device_inputs(w, device, steps_total, rank)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    probe = QuantizedKVCache(cfg, device=device)
+    probe = new_cache()
     n_rep = max(2, math.ceil(3 * l2 / probe.nbytes) + 1)
-    caches = [probe] + [QuantizedKVCache(cfg, device=device) for _ in range(n_rep - 1)]
+    caches = [probe] + [new_cache() for _ in range(n_rep - 1)]
     turbo = w.scheme == "turbo"
     for c in caches:
         if turbo:
@@ -296,7 +317,7 @@ def run_gpu(args, w, rank, world):
     h_vn = vn[args.warmup:].cpu().pin_memory()
     h_out = torch.empty((args.steps,) + tuple(out.shape), dtype=torch.float32).pin_memory()
     d_q, d_kn, d_vn = torch.empty_like(q[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
-    e_caches = [QuantizedKVCache(cfg, device=device) for _ in range(n_rep)]
+    e_caches = [new_cache() for _ in range(n_rep)]
     K, V, _, _, _ = device_inputs(w, device, 1, rank)
     if turbo:
         for c in e_caches:
@@ -397,6 +418,10 @@ def main():
     ap.add_argument("--impl", default="kivi", choices=["kivi", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--page-records", type=int, default=0,
+                    help="paged caches: records per page (block tables are random permutations of the pool)")
+    ap.add_argument("--page-order", default="shuffled", choices=["shuffled", "in-order"],
+                    help="paged caches: pool pages handed out at random or in order")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -408,6 +433,8 @@ def main():
                             f"S{w.seq_len} {w.scheme} {w.bits}-bit G{w.group} R{w.residual}",
                 "global_batch": w.batch * world, "seq_len": w.seq_len, "parallelism": f"dp{world}",
                 "l2": "cache replicas > 3x L2, rotated per step"}
+    if args.page_records > 0:
+        cfg_desc["paged"] = f"{args.page_records} records per page, {args.page_order} block tables"
 
     if args.impl == "reference":
         if rank != 0:

@@ -62,7 +62,8 @@ enum { KVQ_BF16 = 0, KVQ_FP16 = 1 };
 enum {
   KVQ_DEV_NONFINITE_INPUT = 1u << 0, /* a quantized input was inf or nan       */
   KVQ_DEV_PARAM_OVERFLOW = 1u << 1,  /* a scale or zero-point overflowed fp16  */
-  KVQ_DEV_WAIT_TIMEOUT = 1u << 2     /* a bounded pipeline wait gave up        */
+  KVQ_DEV_WAIT_TIMEOUT = 1u << 2,    /* a bounded pipeline wait gave up        */
+  KVQ_DEV_BAD_PAGE = 1u << 3         /* a page table entry was outside the pool */
 };
 
 /*
@@ -80,6 +81,16 @@ enum {
  *   dtype         KVQ_BF16 or KVQ_FP16: the 16-bit format of k, v and q.
  *   qjl_dim       TURBO: m, rows of the 1-bit QJL sketch of the key residual
  *                 (128).  KIVI: 0.
+ *   page_records  0: each row's records are contiguous in the cache buffer.
+ *                 > 0: paged ("TurboQuant : les cinq innovations", item 3:
+ *                 block-wise paged decoding stays possible because the
+ *                 packing is aligned to token blocks).  The records live in
+ *                 a pool of num_pages pages of page_records (a power of
+ *                 two) records each
+ *                 (a record = G tokens for KIVI, 32 for TURBO), and a block
+ *                 table given to kvq_cache_set_page_table maps each row's
+ *                 logical pages to pool pages.
+ *   num_pages     paged caches: pages in the pool (>= 1); else 0.
  */
 typedef struct {
   int32_t scheme;
@@ -93,6 +104,8 @@ typedef struct {
   int32_t max_seq;
   int32_t dtype;
   int32_t qjl_dim;
+  int32_t page_records;
+  int32_t num_pages;
   int32_t reserved;
 } kvq_config;
 
@@ -119,6 +132,8 @@ typedef struct {
   uint64_t params_offset;    /* TURBO: rotation, sketch and codebook         */
   uint64_t params_bytes;
   uint64_t status_offset;    /* uint32 device status word                    */
+  uint64_t pages_per_row;    /* paged: block table entries per row (the pages */
+                             /* that groups_per_row records fill); else 0      */
 } kvq_layout;
 
 typedef struct kvq_cache kvq_cache; /* opaque host handle */
@@ -142,6 +157,21 @@ kvq_status kvq_get_layout(const kvq_config* cfg, kvq_layout* out);
  */
 kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes,
                           void* stream, kvq_cache** out);
+
+/*
+ * Paged caches only, after kvq_cache_init and before any call that touches
+ * records: the block table, device int32 [B * Hkv][pages_per_row] (row-major,
+ * caller-owned, 16-byte aligned).  Entry (row, p) is the pool page holding the
+ * row's records p * page_records .. (p + 1) * page_records - 1; only entries
+ * of pages a row's quantized tokens reach are read, so the caller may fill
+ * them as rows grow (stream-ordered with the calls that use them).  Rows must
+ * not share pages.  An entry outside [0, num_pages) is never dereferenced: the
+ * access is skipped and KVQ_DEV_BAD_PAGE is set.  May be called again to
+ * replace the table pointer.
+ * Errors: KVQ_ERR_UNSUPPORTED for a contiguous cache; KVQ_ERR_INVALID_ARG for
+ * a null or misaligned pointer.
+ */
+kvq_status kvq_cache_set_page_table(kvq_cache* cache, const int32_t* table);
 
 /*
  * TURBO only, once after kvq_cache_init and before any prefill.  Derives the

@@ -10,19 +10,19 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_CUDA, KVQ_ERR_DEVICE_STATUS = range(6)
 KVQ_KIVI, KVQ_TURBO = 0, 1
 KVQ_BF16, KVQ_FP16 = 0, 1
-KVQ_DEV_NONFINITE_INPUT, KVQ_DEV_PARAM_OVERFLOW, KVQ_DEV_WAIT_TIMEOUT = 1, 2, 4
+KVQ_DEV_NONFINITE_INPUT, KVQ_DEV_PARAM_OVERFLOW, KVQ_DEV_WAIT_TIMEOUT, KVQ_DEV_BAD_PAGE = 1, 2, 4, 8
 
 
 class KvqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "scheme", "bits", "group", "residual", "head_dim", "num_kv_heads", "num_q_heads",
-        "batch", "max_seq", "dtype", "qjl_dim", "reserved")]
+        "batch", "max_seq", "dtype", "qjl_dim", "page_records", "num_pages", "reserved")]
 
 
 class KvqLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in (
         "total_bytes", "records_offset", "record_bytes", "groups_per_row", "window_offset",
-        "ring_tokens", "params_offset", "params_bytes", "status_offset")]
+        "ring_tokens", "params_offset", "params_bytes", "status_offset", "pages_per_row")]
 
 
 # name -> (restype, argtypes)
@@ -34,6 +34,7 @@ _SIGS = {
     "kvq_cache_init": (ctypes.c_int, [ctypes.POINTER(KvqConfig), _P, ctypes.c_size_t, _P, ctypes.POINTER(_P)]),
     "kvq_turbo_setup": (ctypes.c_int, [_P, _P, _P, _P]),
     "kvq_turbo_setup_wht": (ctypes.c_int, [_P, _P, _P]),
+    "kvq_cache_set_page_table": (ctypes.c_int, [_P, _P]),
     "kvq_quantize_prefill": (ctypes.c_int, [_P, _P, _P, ctypes.c_int32, _P]),
     "kvq_append_token": (ctypes.c_int, [_P, _P, _P, _P]),
     "kvq_decode_attention": (ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, ctypes.c_size_t, _P]),

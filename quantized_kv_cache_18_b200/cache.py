@@ -22,16 +22,18 @@ def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
 
 
 def make_config(scheme: str, bits: int, group: int, residual: int, head_dim: int, num_kv_heads: int,
-                num_q_heads: int, batch: int, max_seq: int, dtype: str, qjl_dim: int = 0) -> L.KvqConfig:
+                num_q_heads: int, batch: int, max_seq: int, dtype: str, qjl_dim: int = 0,
+                page_records: int = 0, num_pages: int = 0) -> L.KvqConfig:
     return L.KvqConfig(L.KVQ_KIVI if scheme == "kivi" else L.KVQ_TURBO, bits, group, residual, head_dim,
                        num_kv_heads, num_q_heads, batch, max_seq,
-                       L.KVQ_BF16 if dtype == "bf16" else L.KVQ_FP16, qjl_dim, 0)
+                       L.KVQ_BF16 if dtype == "bf16" else L.KVQ_FP16, qjl_dim, page_records, num_pages, 0)
 
 
-def config_from_workload(w, max_seq: Optional[int] = None) -> L.KvqConfig:
+def config_from_workload(w, max_seq: Optional[int] = None, page_records: int = 0,
+                         num_pages: int = 0) -> L.KvqConfig:
     return make_config(w.scheme, w.bits, w.group, w.residual, w.head_dim, w.num_kv_heads, w.num_q_heads,
                        w.batch, max_seq if max_seq is not None else w.max_seq, w.dtype,
-                       w.qjl_dim if w.scheme == "turbo" else 0)
+                       w.qjl_dim if w.scheme == "turbo" else 0, page_records, num_pages)
 
 
 def cache_bytes(cfg: L.KvqConfig) -> int:
@@ -115,6 +117,30 @@ class QuantizedKVCache:
                 raise ValueError(f"{what}: shape {tuple(t.shape)} != {shape}")
         L.check(self.lib.kvq_turbo_setup(self.handle, _ptr(rot_gauss), _ptr(qjl_gauss), _stream_ptr(stream)),
                 "kvq_turbo_setup")
+
+    def set_page_table(self, table: torch.Tensor):
+        """Paged caches: the block table, int32 [B*Hkv][pages_per_row] on the
+        cache's device (kept referenced by this object)."""
+        c, lay = self.cfg, self.layout
+        shape = (c.batch * c.num_kv_heads, lay.pages_per_row)
+        if table.device != self.buf.device or table.dtype != torch.int32 or not table.is_contiguous():
+            raise ValueError(f"page table: needs a contiguous int32 tensor on {self.buf.device}")
+        if tuple(table.shape) != shape:
+            raise ValueError(f"page table: shape {tuple(table.shape)} != {shape}")
+        L.check(self.lib.kvq_cache_set_page_table(self.handle, _ptr(table)), "kvq_cache_set_page_table")
+        self.page_table = table
+
+    def row_records(self, row: int, n: int) -> torch.Tensor:
+        """[n][record_bytes] uint8 copy of a row's first n records, through the
+        block table for a paged cache."""
+        c, lay = self.cfg, self.layout
+        if c.page_records == 0:
+            return self.records_view()[row, :n]
+        pool = self.buf[lay.records_offset:lay.records_offset + c.num_pages * c.page_records * lay.record_bytes]
+        pool = pool.view(c.num_pages * c.page_records, lay.record_bytes)
+        k = torch.arange(n, device=self.buf.device)
+        pages = self.page_table[row].long()[k // c.page_records]
+        return pool[pages * c.page_records + k % c.page_records]
 
     def turbo_setup_wht(self, qjl_gauss: torch.Tensor, stream=None):
         """TurboQuant scheme with the Walsh-Hadamard rotation H / sqrt(d): the

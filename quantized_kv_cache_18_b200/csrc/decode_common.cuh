@@ -62,6 +62,65 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// Records first .. first + cnt - 1 of a row (cnt <= 16) into shared memory,
+// in steps so that a paged cache's page-id loads are in flight while the
+// producer waits for a free stage:
+//   record_pages  issues the loads of the ids of the pages the records touch
+//                 (nothing when contiguous);
+//   pages_valid   (after the wait) whether all of them are in the pool;
+//   copy_records  arms `bar` and issues one copy (contiguous) or one per page.
+struct RecordPages {
+  int32_t ids[16];
+  int nr, p0;
+};
+// Page sizes are powers of two (page_shift = log2 of records per page), so the
+// page arithmetic is shifts and masks on 32-bit record indices.
+__device__ __forceinline__ void record_pages(const Geom& gm, int row, int64_t first, int cnt, RecordPages& pg) {
+  pg.nr = 0;
+  if (gm.page_table == nullptr) return;
+  const int f = (int)first, sh = gm.page_shift;
+  pg.p0 = f >> sh;
+  pg.nr = ((f + cnt - 1) >> sh) - pg.p0 + 1;
+  const int32_t* tab = gm.page_table + (int64_t)row * gm.pages_per_row + pg.p0;
+  pg.ids[0] = __ldg(tab);
+  if (pg.nr > 1) {
+#pragma unroll
+    for (int i = 1; i < 16; ++i) pg.ids[i] = i < pg.nr ? __ldg(tab + i) : 0;
+  }
+}
+__device__ __forceinline__ bool pages_valid(const Geom& gm, const RecordPages& pg) {
+  if (pg.nr == 1) return pg.ids[0] >= 0 && pg.ids[0] < gm.num_pages;
+  bool ok = true;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    if (i < pg.nr && (pg.ids[i] < 0 || pg.ids[i] >= gm.num_pages)) ok = false;
+  return ok;
+}
+__device__ __forceinline__ void copy_records(const Geom& gm, int row, int64_t first, int cnt, int rec_bytes,
+                                             const RecordPages& pg, unsigned char* dst, uint64_t* bar) {
+  mbar_expect_tx(bar, (uint32_t)cnt * rec_bytes);
+  if (gm.page_table == nullptr) {
+    bulk_g2s(dst, record_ptr(gm, row, first), (uint32_t)cnt * rec_bytes, bar);
+    return;
+  }
+  const int f = (int)first, sh = gm.page_shift, mask = (1 << sh) - 1;
+  if (pg.nr == 1) {
+    bulk_g2s(dst, gm.records + (((int64_t)pg.ids[0] << sh) | (f & mask)) * rec_bytes, (uint32_t)cnt * rec_bytes,
+             bar);
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (i < pg.nr) {
+      const int pgi = pg.p0 + i;
+      const int g0 = max(f, pgi << sh), g1 = min(f + cnt, (pgi + 1) << sh);
+      bulk_g2s(dst + (int64_t)(g0 - f) * rec_bytes,
+               gm.records + (((int64_t)pg.ids[i] << sh) | (g0 & mask)) * rec_bytes, (uint32_t)(g1 - g0) * rec_bytes,
+               bar);
+    }
+  }
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "

@@ -86,6 +86,7 @@ struct K {
   static constexpr int OFF_FLAG = OFF_BAR + (3 * NST + 8) * 8;
   static constexpr int SMEM = OFF_FLAG + 16;
   static_assert(NST >= 2, "decode pipeline needs two stages");
+  static_assert(SG <= 16, "a stage copies at most 16 records");
   static_assert(SMEM <= 227 * 1024, "decode kernel shared memory exceeds the per-block limit");
 };
 
@@ -358,6 +359,9 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
           [&](int s, int row, bool win, int64_t first, int cnt) {
             if (*abort_flag) return;
             const int slot = s % C::NST;
+            // a paged stage's page ids load while the producer waits for the slot
+            RecordPages pages;
+            if (!win) record_pages(gm, row, first, cnt, pages);
             if (s >= C::NST && !mbar_wait(&bar_empty[slot], ((s / C::NST) - 1) & 1, abort_flag)) {
               atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
               *abort_flag = 1;
@@ -365,9 +369,12 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
             }
             unsigned char* dst = smem + slot * C::STAGE;
             if (!win) {
-              const uint32_t bytes = (uint32_t)cnt * C::REC;
-              mbar_expect_tx(&bar_full[slot], bytes);
-              bulk_g2s(dst, record_ptr(gm, row, first), bytes, &bar_full[slot]);
+              if (!pages_valid(gm, pages)) {
+                atomicOr(gm.status, KVQ_DEV_BAD_PAGE);
+                *abort_flag = 1;
+                return;
+              }
+              copy_records(gm, row, first, cnt, C::REC, pages, dst, &bar_full[slot]);
             } else {
               const int t0 = (int)first * kWinTok;
               const int n = min(kWinTok, a.r - t0);

@@ -205,8 +205,9 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
   // is the codes of two adjacent channels of a token (keys) or of two adjacent
   // tokens of a channel (values), one 16-bit load either way
   char* rec = record_ptr(gm, row, a.dst_group0 + grp);
+  if (rec == nullptr) flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
   constexpr int PIECES = NTB * 32 * (P / 4);   // per key (or value) part
-  for (int i = tid; i < 2 * PIECES; i += kQuantThreads) {
+  for (int i = rec != nullptr ? tid : 2 * PIECES; i < 2 * PIECES; i += kQuantThreads) {
     const bool is_v = i >= PIECES;
     const int pi = is_v ? i - PIECES : i;
     const int tb = pi / (32 * (P / 4));
@@ -253,14 +254,14 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
   // 6. metadata
   uint16_t* ksc = reinterpret_cast<uint16_t*>(rec + rec_kscale_off(gm));
   uint16_t* kzr = reinterpret_cast<uint16_t*>(rec + rec_kzero_off(gm));
-  for (int c = tid; c < D; c += kQuantThreads) {
+  for (int c = rec != nullptr ? tid : D; c < D; c += kQuantThreads) {
     const int kt = c >> 4, rho = (c >> 3) & 1, tc = (c >> 1) & 3, e = c & 1;
     const int pos = 8 * (4 * (kt >> 1) + tc) + 4 * (kt & 1) + 2 * rho + e;
     ksc[pos] = k_sb[c];
     kzr[pos] = k_zb[c];
   }
   uint32_t* vm = reinterpret_cast<uint32_t*>(rec + rec_vmeta_off(gm));
-  for (int t = tid; t < G; t += kQuantThreads) {
+  for (int t = rec != nullptr ? tid : G; t < G; t += kQuantThreads) {
     const int tb = t / kTB, tt = t % kTB;
     const int kt = tt >> 4, rho = (tt >> 3) & 1, tc = (tt >> 1) & 3, e = tt & 1;
     vm[tb * kTB + 8 * tc + 4 * kt + 2 * rho + e] = (uint32_t)v_sb[t] | ((uint32_t)v_zb[t] << 16);

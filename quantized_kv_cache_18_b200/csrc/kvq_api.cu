@@ -21,6 +21,7 @@ struct kvq_cache {
   int32_t head;
   bool tq_ready;   // TURBO: the parameter block holds the deployment constants
   bool tq_wht;     // TURBO: the rotation is the Walsh-Hadamard one
+  const int32_t* page_table;   // paged: [rows][pages_per_row] pool pages (device, caller-owned)
 };
 
 namespace kvq {
@@ -67,6 +68,9 @@ static bool config_ok(const kvq_config* c) {
   if (c->batch <= 0 || c->max_seq <= 0) return false;
   if ((int64_t)c->batch * c->num_kv_heads > 65535) return false;
   if (!(c->dtype == KVQ_BF16 || c->dtype == KVQ_FP16)) return false;
+  if (c->page_records < 0 || c->num_pages < 0) return false;
+  if ((c->page_records == 0) != (c->num_pages == 0)) return false;   // both set or both zero
+  if (c->page_records & (c->page_records - 1)) return false;          // a power of two
   return true;
 }
 
@@ -79,7 +83,9 @@ static kvq_layout make_layout(const kvq_config* c) {
   L.groups_per_row = c->max_seq > c->residual ? (uint64_t)(c->max_seq - c->residual) / G : 0;
   L.ring_tokens = (uint64_t)c->residual + G;
   L.records_offset = 0;
-  uint64_t off = align_up(rows * L.groups_per_row * L.record_bytes, 256);
+  const uint64_t n_records = c->page_records > 0 ? (uint64_t)c->num_pages * c->page_records : rows * L.groups_per_row;
+  L.pages_per_row = c->page_records > 0 ? (L.groups_per_row + c->page_records - 1) / c->page_records : 0;
+  uint64_t off = align_up(n_records * L.record_bytes, 256);
   L.window_offset = off;
   off = align_up(off + rows * 2 * L.ring_tokens * d * 2, 256);
   L.params_offset = off;
@@ -95,6 +101,12 @@ static Geom make_geom(const kvq_cache* h) {
   const kvq_config& c = h->cfg;
   g.scheme = c.scheme;
   g.rot_wht = h->tq_wht ? 1 : 0;
+  g.page_table = c.page_records > 0 ? h->page_table : nullptr;
+  g.page_recs = c.page_records;
+  g.page_shift = 0;
+  while (c.page_records > 0 && (1 << g.page_shift) < c.page_records) ++g.page_shift;
+  g.pages_per_row = (int64_t)h->lay.pages_per_row;
+  g.num_pages = c.num_pages;
   g.d = c.head_dim;
   g.bits = c.bits;
   g.G = c.group;
@@ -185,6 +197,7 @@ kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes, vo
   h->seq_len = h->tq = h->r = h->head = 0;
   h->tq_ready = false;
   h->tq_wht = false;
+  h->page_table = nullptr;
   launch_clear_words(reinterpret_cast<uint32_t*>(h->base + L.status_offset),
                      1 + cfg->batch * cfg->num_kv_heads, (cudaStream_t)stream);
   if (check_launch() != KVQ_OK) {
@@ -194,6 +207,17 @@ kvq_status kvq_cache_init(const kvq_config* cfg, void* dev_buf, size_t bytes, vo
   *out = h;
   return KVQ_OK;
 }
+
+kvq_status kvq_cache_set_page_table(kvq_cache* h, const int32_t* table) {
+  if (!h) return KVQ_ERR_INVALID_ARG;
+  if (h->cfg.page_records == 0) return KVQ_ERR_UNSUPPORTED;
+  if (!table || !aligned16(table)) return KVQ_ERR_INVALID_ARG;
+  h->page_table = table;
+  return KVQ_OK;
+}
+
+// A paged cache needs its block table before any call that touches records.
+static bool records_ready(const kvq_cache* h) { return h->cfg.page_records == 0 || h->page_table != nullptr; }
 
 kvq_status kvq_turbo_setup(kvq_cache* h, const float* rot_gauss, const float* qjl_gauss, void* stream) {
   if (!h || !rot_gauss || !qjl_gauss) return KVQ_ERR_INVALID_ARG;
@@ -224,6 +248,7 @@ kvq_status kvq_quantize_prefill(kvq_cache* h, const void* k, const void* v, int3
   if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_INVALID_ARG;
   if (h->seq_len != 0) return KVQ_ERR_INVALID_ARG;
   if (h->cfg.scheme == KVQ_TURBO && !h->tq_ready) return KVQ_ERR_INVALID_ARG;
+  if (!records_ready(h)) return KVQ_ERR_INVALID_ARG;
   if (seq_len > h->cfg.max_seq) return KVQ_ERR_CAPACITY;
   const kvq_config& c = h->cfg;
   const int32_t G = c.group, R = c.residual;
@@ -253,6 +278,7 @@ kvq_status kvq_append_token(kvq_cache* h, const void* k_new, const void* v_new, 
   if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
   if (h->seq_len + 1 > h->cfg.max_seq) return KVQ_ERR_CAPACITY;
   if (h->cfg.scheme == KVQ_TURBO && !h->tq_ready) return KVQ_ERR_INVALID_ARG;
+  if (!records_ready(h)) return KVQ_ERR_INVALID_ARG;
   const kvq_config& c = h->cfg;
   const int32_t G = c.group, R = c.residual, cap = R + G;
   const Geom g = make_geom(h);
@@ -291,6 +317,7 @@ static kvq_status check_attention_args(const kvq_cache* h, const void* q, const 
   if (!(std::isfinite(softmax_scale))) return KVQ_ERR_INVALID_ARG;
   if (workspace_bytes < kvq_workspace_bytes(&h->cfg)) return KVQ_ERR_INVALID_ARG;
   if (h->cfg.scheme == KVQ_TURBO && !h->tq_ready) return KVQ_ERR_INVALID_ARG;
+  if (!records_ready(h)) return KVQ_ERR_INVALID_ARG;
   return KVQ_OK;
 }
 

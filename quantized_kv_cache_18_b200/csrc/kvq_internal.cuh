@@ -41,6 +41,11 @@ constexpr int kMaxDecodeCtas = 160;   // decode launches use at most this many C
 struct Geom {
   int scheme, d, bits, G, R, cap, B, Hkv, Hq, g, dtype;
   int rot_wht;              // TURBO: Pi is the Walsh-Hadamard rotation H / sqrt(d)
+  const int32_t* page_table;   // paged: [rows][pages_per_row] pool pages, else null
+  int page_recs;               // paged: records per page (a power of two)
+  int page_shift;              // paged: log2(page_recs)
+  int num_pages;               // paged: pages in the pool
+  int64_t pages_per_row;
   int64_t groups_per_row;   // record capacity of a row
   int64_t rec_bytes;        // bytes of one group record
   int64_t tb_code_bytes;    // bytes of one TB's key (or value) codes
@@ -90,8 +95,15 @@ __host__ __device__ inline int64_t rec_kscale_off(const Geom& g) { return (int64
 __host__ __device__ inline int64_t rec_kzero_off(const Geom& g) { return rec_kscale_off(g) + 2 * g.d; }
 __host__ __device__ inline int64_t rec_vmeta_off(const Geom& g) { return rec_kscale_off(g) + 4 * g.d; }
 
-__host__ __device__ inline char* record_ptr(const Geom& g, int row, int64_t group) {
-  return g.records + ((int64_t)row * g.groups_per_row + group) * g.rec_bytes;
+// Address of record `group` of `row`.  Paged caches look the page up in the
+// block table; a page outside the pool gives null (the caller skips the access
+// and reports KVQ_DEV_BAD_PAGE).
+__device__ inline char* record_ptr(const Geom& g, int row, int64_t group) {
+  if (g.page_table == nullptr) return g.records + ((int64_t)row * g.groups_per_row + group) * g.rec_bytes;
+  const int64_t p = group >> g.page_shift;
+  const int32_t page = __ldg(g.page_table + (int64_t)row * g.pages_per_row + p);
+  if (page < 0 || page >= g.num_pages) return nullptr;
+  return g.records + (((int64_t)page << g.page_shift) + (group & (g.page_recs - 1))) * g.rec_bytes;
 }
 __host__ __device__ inline uint16_t* ring_ptr(const Geom& g, int row, int kv) {
   return g.window + ((int64_t)row * 2 + kv) * g.cap * g.d;

@@ -210,6 +210,9 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
           [&](int s, int row, bool win, int64_t first, int cnt) {
             if (*abort_flag) return;
             const int slot = s % C::NST;
+            // a paged stage's page ids load while the producer waits for the slot
+            RecordPages pages;
+            if (!win) record_pages(gm, row, first, cnt, pages);
             if (s >= C::NST && !mbar_wait(&bar_empty[slot], ((s / C::NST) - 1) & 1, abort_flag)) {
               atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
               *abort_flag = 1;
@@ -217,9 +220,12 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
             }
             unsigned char* dst = smem + slot * C::STAGE;
             if (!win) {
-              const uint32_t bytes = (uint32_t)cnt * kTqTbBytes;
-              mbar_expect_tx(&bar_full[slot], bytes);
-              bulk_g2s(dst, record_ptr(gm, row, first), bytes, &bar_full[slot]);
+              if (!pages_valid(gm, pages)) {
+                atomicOr(gm.status, KVQ_DEV_BAD_PAGE);
+                *abort_flag = 1;
+                return;
+              }
+              copy_records(gm, row, first, cnt, kTqTbBytes, pages, dst, &bar_full[slot]);
             } else {
               const int t0 = (int)first * kTqWin;
               const int n = min(kTqWin, a.r - t0);

@@ -222,7 +222,8 @@ __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) 
 
     // ---------------------------------------------------------- pack and store the token block
     uint32_t* dst = reinterpret_cast<uint32_t*>(record_ptr(gm, row, a.dst_group0 + blk));
-    for (int qw = tid; qw < 2 * 416 + 128 + 32; qw += kQThreads) {
+    if (dst == nullptr) flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
+    for (int qw = dst != nullptr ? tid : 2 * 416 + 128 + 32; qw < 2 * 416 + 128 + 32; qw += kQThreads) {
       if (qw < 2 * 416) {
         const int vblk = qw >= 416;
         const int q = qw - 416 * vblk;
