@@ -171,11 +171,13 @@ def device_inputs(w, device, steps_total, rank: int = 0):
 
 
 def step_bytes(cache) -> int:
-    """Packed bytes one decode attention reads: every group record and every
-    window token (16-bit key and value)."""
+    """Packed bytes one decode attention reads: every group record, every
+    window token (key and value rows: 16-bit, or FP8 rows in the mixed cache)
+    and the mixed cache's FP8 anchor rows."""
     c, lay = cache.cfg, cache.layout
     rows = c.batch * c.num_kv_heads
-    return rows * (cache.quantized_len // c.group * lay.record_bytes + cache.window_len * 2 * c.head_dim * 2)
+    return rows * (cache.quantized_len // c.group * lay.record_bytes +
+                   (cache.window_len + c.anchor_tokens) * 2 * lay.token_row_bytes)
 
 
 # ---------------------------------------------------------------- GPU arm

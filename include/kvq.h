@@ -20,6 +20,8 @@
  *           comme le premier levier d'inference", section "Minima-KV : la
  *           compression sans eviction" (partial attention states merged by a
  *           globally normalised online softmax).
+ *   [MIXED] the same section: recent and protected ("Anchor") pages in FP8,
+ *           older pages in TQ3, one attention over both.
  *
  * Conventions for every call:
  *   - Ownership: the caller allocates and frees all device memory (cache
@@ -91,6 +93,14 @@ enum {
  *                 table given to kvq_cache_set_page_table maps each row's
  *                 logical pages to pool pages.
  *   num_pages     paged caches: pages in the pool (>= 1); else 0.
+ *   fp8_recent    TURBO only, 0 or 1: the mixed-format cache of [MIXED]:
+ *                 the residual window and the anchor tokens are stored in
+ *                 FP8 E4M3 with one fp16 scale per token vector
+ *                 (s = RNE_fp16(max |x| / 448), codes RNE_e4m3(x / s)), and
+ *                 window tokens leave for TQ3 from their FP8 values.
+ *   anchor_tokens fp8_recent caches: A, a multiple of 32: the first A tokens
+ *                 of every sequence (from the prefill, which then needs
+ *                 seq_len >= A) stay in FP8 for good.  Else 0.
  */
 typedef struct {
   int32_t scheme;
@@ -106,7 +116,8 @@ typedef struct {
   int32_t qjl_dim;
   int32_t page_records;
   int32_t num_pages;
-  int32_t reserved;
+  int32_t fp8_recent;
+  int32_t anchor_tokens;
 } kvq_config;
 
 /*
@@ -134,6 +145,10 @@ typedef struct {
   uint64_t status_offset;    /* uint32 device status word                    */
   uint64_t pages_per_row;    /* paged: block table entries per row (the pages */
                              /* that groups_per_row records fill); else 0      */
+  uint64_t token_row_bytes;  /* bytes of one window token row of K or V: 2 d, */
+                             /* or 144 for FP8 rows (128 E4M3 codes, the fp16 */
+                             /* scale, 14 zero bytes)                         */
+  uint64_t anchor_offset;    /* fp8_recent: [B][Hkv][2][A][token_row_bytes]   */
 } kvq_layout;
 
 typedef struct kvq_cache kvq_cache; /* opaque host handle */

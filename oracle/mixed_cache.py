@@ -53,12 +53,16 @@ class MixedRow:
         self.ring = {kv: (np.zeros((self.cap, d), np.uint8), np.zeros(self.cap)) for kv in "kv"}
         self.head = 0
         self.r = 0
+        self.k_in = np.zeros((0, d))   # the float64 vectors that went into TQ3, in order
+        self.v_in = np.zeros((0, d))
 
     @property
     def tq(self) -> int:
         return self.kq["codes"].shape[0]
 
     def _quantize(self, k: np.ndarray, v: np.ndarray):
+        self.k_in = np.concatenate([self.k_in, k])
+        self.v_in = np.concatenate([self.v_in, v])
         a = turbo.quantize(k, self.Pi, self.levels, self.thresholds, self.S)
         b = turbo.quantize(v, self.Pi, self.levels, self.thresholds)
         for key in ("codes", "n", "gamma", "signs", "y", "se"):

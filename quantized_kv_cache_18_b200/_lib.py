@@ -16,13 +16,14 @@ KVQ_DEV_NONFINITE_INPUT, KVQ_DEV_PARAM_OVERFLOW, KVQ_DEV_WAIT_TIMEOUT, KVQ_DEV_B
 class KvqConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "scheme", "bits", "group", "residual", "head_dim", "num_kv_heads", "num_q_heads",
-        "batch", "max_seq", "dtype", "qjl_dim", "page_records", "num_pages", "reserved")]
+        "batch", "max_seq", "dtype", "qjl_dim", "page_records", "num_pages", "fp8_recent", "anchor_tokens")]
 
 
 class KvqLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in (
         "total_bytes", "records_offset", "record_bytes", "groups_per_row", "window_offset",
-        "ring_tokens", "params_offset", "params_bytes", "status_offset", "pages_per_row")]
+        "ring_tokens", "params_offset", "params_bytes", "status_offset", "pages_per_row", "token_row_bytes",
+        "anchor_offset")]
 
 
 # name -> (restype, argtypes)

@@ -23,17 +23,20 @@ def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
 
 def make_config(scheme: str, bits: int, group: int, residual: int, head_dim: int, num_kv_heads: int,
                 num_q_heads: int, batch: int, max_seq: int, dtype: str, qjl_dim: int = 0,
-                page_records: int = 0, num_pages: int = 0) -> L.KvqConfig:
+                page_records: int = 0, num_pages: int = 0, fp8_recent: int = 0,
+                anchor_tokens: int = 0) -> L.KvqConfig:
     return L.KvqConfig(L.KVQ_KIVI if scheme == "kivi" else L.KVQ_TURBO, bits, group, residual, head_dim,
                        num_kv_heads, num_q_heads, batch, max_seq,
-                       L.KVQ_BF16 if dtype == "bf16" else L.KVQ_FP16, qjl_dim, page_records, num_pages, 0)
+                       L.KVQ_BF16 if dtype == "bf16" else L.KVQ_FP16, qjl_dim, page_records, num_pages,
+                       fp8_recent, anchor_tokens)
 
 
 def config_from_workload(w, max_seq: Optional[int] = None, page_records: int = 0,
                          num_pages: int = 0) -> L.KvqConfig:
     return make_config(w.scheme, w.bits, w.group, w.residual, w.head_dim, w.num_kv_heads, w.num_q_heads,
                        w.batch, max_seq if max_seq is not None else w.max_seq, w.dtype,
-                       w.qjl_dim if w.scheme == "turbo" else 0, page_records, num_pages)
+                       w.qjl_dim if w.scheme == "turbo" else 0, page_records, num_pages,
+                       1 if w.fp8_recent else 0, w.anchor_tokens)
 
 
 def cache_bytes(cfg: L.KvqConfig) -> int:
@@ -225,6 +228,20 @@ class QuantizedKVCache:
         """uint8 view of the TurboQuant parameter block (empty for KIVI)."""
         lay = self.layout
         return self.buf[lay.params_offset:lay.params_offset + lay.params_bytes]
+
+    def fp8_ring_view(self) -> torch.Tensor:
+        """fp8_recent caches: [B*Hkv][2][ring_tokens][144] uint8 FP8 token rows of the window."""
+        c, lay = self.cfg, self.layout
+        n = c.batch * c.num_kv_heads * 2 * lay.ring_tokens * lay.token_row_bytes
+        return self.buf[lay.window_offset:lay.window_offset + n].view(
+            c.batch * c.num_kv_heads, 2, lay.ring_tokens, lay.token_row_bytes)
+
+    def anchor_view(self) -> torch.Tensor:
+        """fp8_recent caches: [B*Hkv][2][A][144] uint8 FP8 token rows of the anchors."""
+        c, lay = self.cfg, self.layout
+        n = c.batch * c.num_kv_heads * 2 * c.anchor_tokens * lay.token_row_bytes
+        return self.buf[lay.anchor_offset:lay.anchor_offset + n].view(
+            c.batch * c.num_kv_heads, 2, c.anchor_tokens, lay.token_row_bytes)
 
     def ring_view(self) -> torch.Tensor:
         """[B*Hkv][2][ring_tokens][d] 16-bit patterns (as int16) of the residual rings."""

@@ -71,6 +71,10 @@ static bool config_ok(const kvq_config* c) {
   if (c->page_records < 0 || c->num_pages < 0) return false;
   if ((c->page_records == 0) != (c->num_pages == 0)) return false;   // both set or both zero
   if (c->page_records & (c->page_records - 1)) return false;          // a power of two
+  if (!(c->fp8_recent == 0 || c->fp8_recent == 1)) return false;
+  if (c->fp8_recent && c->scheme != KVQ_TURBO) return false;          // the mixed cache is TQ3 + FP8
+  if (c->anchor_tokens < 0 || c->anchor_tokens % 32 != 0) return false;
+  if (c->anchor_tokens > 0 && !c->fp8_recent) return false;
   return true;
 }
 
@@ -80,14 +84,18 @@ static kvq_layout make_layout(const kvq_config* c) {
   const uint64_t rows = (uint64_t)c->batch * c->num_kv_heads;
   const uint64_t d = c->head_dim, G = c->group;
   L.record_bytes = c->scheme == KVQ_TURBO ? (uint64_t)kTqTbBytes : G * d * c->bits / 4 + 4 * d + 4 * G;
-  L.groups_per_row = c->max_seq > c->residual ? (uint64_t)(c->max_seq - c->residual) / G : 0;
+  const int64_t q_room = (int64_t)c->max_seq - c->residual - c->anchor_tokens;   // tokens that can be quantized
+  L.groups_per_row = q_room > 0 ? (uint64_t)q_room / G : 0;
   L.ring_tokens = (uint64_t)c->residual + G;
+  L.token_row_bytes = c->fp8_recent ? (uint64_t)kFp8RowBytes : 2 * d;
   L.records_offset = 0;
   const uint64_t n_records = c->page_records > 0 ? (uint64_t)c->num_pages * c->page_records : rows * L.groups_per_row;
   L.pages_per_row = c->page_records > 0 ? (L.groups_per_row + c->page_records - 1) / c->page_records : 0;
   uint64_t off = align_up(n_records * L.record_bytes, 256);
   L.window_offset = off;
-  off = align_up(off + rows * 2 * L.ring_tokens * d * 2, 256);
+  off = align_up(off + rows * 2 * L.ring_tokens * L.token_row_bytes, 256);
+  L.anchor_offset = off;
+  off = align_up(off + rows * 2 * (uint64_t)c->anchor_tokens * L.token_row_bytes, 256);
   L.params_offset = off;
   L.params_bytes = c->scheme == KVQ_TURBO ? (uint64_t)kTqParamBytes : 0;
   off = align_up(off + L.params_bytes, 256);
@@ -107,6 +115,9 @@ static Geom make_geom(const kvq_cache* h) {
   while (c.page_records > 0 && (1 << g.page_shift) < c.page_records) ++g.page_shift;
   g.pages_per_row = (int64_t)h->lay.pages_per_row;
   g.num_pages = c.num_pages;
+  g.fp8 = c.fp8_recent;
+  g.anchor = c.anchor_tokens;
+  g.anchors = reinterpret_cast<unsigned char*>(h->base + h->lay.anchor_offset);
   g.d = c.head_dim;
   g.bits = c.bits;
   g.G = c.group;
@@ -135,7 +146,8 @@ static int plan_ctas(const kvq_config& c, int64_t n_groups, int r) {
   const int64_t rows = (int64_t)c.batch * c.num_kv_heads;
   const int64_t rec = c.scheme == KVQ_TURBO ? (int64_t)kTqTbBytes
                                              : (int64_t)c.group * c.head_dim * c.bits / 4 + 4 * c.head_dim + 4 * c.group;
-  const int64_t tokb = 4 * (int64_t)c.head_dim;
+  const int64_t tokb = c.fp8_recent ? 2 * (int64_t)kFp8RowBytes : 4 * (int64_t)c.head_dim;
+  r += c.anchor_tokens;   // anchors weigh like window tokens
   const int64_t w_tot = rows * (n_groups * rec + (int64_t)r * tokb);
   const int64_t w_max = r > 0 ? (rec > 32 * tokb ? rec : 32 * tokb) : rec;
   int64_t n = w_tot / w_max;
@@ -251,24 +263,36 @@ kvq_status kvq_quantize_prefill(kvq_cache* h, const void* k, const void* v, int3
   if (!records_ready(h)) return KVQ_ERR_INVALID_ARG;
   if (seq_len > h->cfg.max_seq) return KVQ_ERR_CAPACITY;
   const kvq_config& c = h->cfg;
-  const int32_t G = c.group, R = c.residual;
-  const int32_t tq = seq_len > R ? G * ((seq_len - R) / G) : 0;
+  const int32_t G = c.group, R = c.residual, A = c.anchor_tokens;
+  if (seq_len < A) return KVQ_ERR_INVALID_ARG;   // the anchors come with the prefill
+  const int32_t rest = seq_len - A;               // tokens after the anchors
+  const int32_t tq = rest > R ? G * ((rest - R) / G) : 0;
   const Geom g = make_geom(h);
   cudaStream_t st = (cudaStream_t)stream;
   QuantArgs a;
   a.geom = g;
-  a.src_k = static_cast<const uint16_t*>(k);
-  a.src_v = static_cast<const uint16_t*>(v);
+  a.src_k = static_cast<const uint16_t*>(k) + (int64_t)A * c.head_dim;
+  a.src_v = static_cast<const uint16_t*>(v) + (int64_t)A * c.head_dim;
   a.src_row_stride = (int64_t)seq_len * c.head_dim;
+  a.src_fp8 = nullptr;
   a.dst_group0 = 0;
   a.n_groups = tq / G;
   if (c.scheme == KVQ_TURBO) launch_tq_quantize(a, st);
   else launch_kivi_quantize(a, st);
-  launch_window_copy(g, a.src_k, a.src_v, seq_len, tq, seq_len - tq, st);
+  if (c.fp8_recent) {
+    const uint16_t* k16 = static_cast<const uint16_t*>(k);
+    const uint16_t* v16 = static_cast<const uint16_t*>(v);
+    const int64_t ring_row = (int64_t)2 * g.cap * kFp8RowBytes, anc_row = (int64_t)2 * A * kFp8RowBytes;
+    launch_fp8_rows(g, k16, v16, seq_len, 0, A, g.anchors, anc_row, (int64_t)A * kFp8RowBytes, 0, st);
+    launch_fp8_rows(g, k16, v16, seq_len, A + tq, rest - tq, reinterpret_cast<unsigned char*>(g.window), ring_row,
+                    (int64_t)g.cap * kFp8RowBytes, 0, st);
+  } else {
+    launch_window_copy(g, a.src_k, a.src_v, seq_len, tq, seq_len - tq, st);
+  }
   if (check_launch() != KVQ_OK) return KVQ_ERR_CUDA;
   h->seq_len = seq_len;
   h->tq = tq;
-  h->r = seq_len - tq;
+  h->r = rest - tq;
   h->head = 0;
   return KVQ_OK;
 }
@@ -286,13 +310,21 @@ kvq_status kvq_append_token(kvq_cache* h, const void* k_new, const void* v_new, 
   const int slot = (h->head + h->r) % cap;
   int32_t r = h->r + 1, head = h->head, tq = h->tq;
   if (r == R + G && (uint64_t)(tq / G) >= h->lay.groups_per_row) return KVQ_ERR_CAPACITY;
-  launch_append(g, static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), slot, st);
+  if (c.fp8_recent)
+    launch_fp8_rows(g, static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), 1, 0, 1,
+                    reinterpret_cast<unsigned char*>(g.window), (int64_t)2 * cap * kFp8RowBytes,
+                    (int64_t)cap * kFp8RowBytes, slot, st);
+  else
+    launch_append(g, static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), slot, st);
   if (r == R + G) {
     QuantArgs a;
     a.geom = g;
     a.src_k = g.window + (int64_t)head * c.head_dim;
     a.src_v = g.window + ((int64_t)cap + head) * c.head_dim;
     a.src_row_stride = (int64_t)2 * cap * c.head_dim;
+    // mixed cache: the flushed tokens are the window's FP8 rows
+    a.src_fp8 = c.fp8_recent ? reinterpret_cast<const unsigned char*>(g.window) + (int64_t)head * kFp8RowBytes
+                             : nullptr;
     a.dst_group0 = tq / G;
     a.n_groups = 1;
     if (c.scheme == KVQ_TURBO) launch_tq_quantize(a, st);
@@ -372,8 +404,9 @@ kvq_status kvq_append_decode(kvq_cache* h, const void* k_new, const void* v_new,
   if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
   if (h->seq_len + 1 > h->cfg.max_seq) return KVQ_ERR_CAPACITY;
   const int32_t r_new = h->r + 1;
-  if (r_new == h->cfg.residual + h->cfg.group) {
-    // a flush is due: the oldest G window tokens are quantized before the attention reads them
+  if (r_new == h->cfg.residual + h->cfg.group || h->cfg.fp8_recent) {
+    // a flush is due, or the window holds FP8 rows (the new token is converted
+    // by kvq_append_token): append, then attend
     const kvq_status ea = kvq_append_token(h, k_new, v_new, stream);
     if (ea != KVQ_OK) return ea;
     return launch_attention(h, h->r, q, out, softmax_scale, workspace, (cudaStream_t)stream, nullptr, nullptr);
@@ -410,7 +443,7 @@ kvq_status kvq_cache_set_state(kvq_cache* h, int32_t seq_len, int32_t quantized_
   if (seq_len < 0 || quantized_len < 0 || quantized_len % G != 0 || window_head < 0 || window_head >= cap ||
       window_head % G != 0)
     return KVQ_ERR_INVALID_ARG;
-  const int32_t r = seq_len - quantized_len;
+  const int32_t r = seq_len - c.anchor_tokens - quantized_len;
   if (r < 0 || r >= cap) return KVQ_ERR_INVALID_ARG;
   if (seq_len > c.max_seq || (uint64_t)(quantized_len / G) > h->lay.groups_per_row) return KVQ_ERR_CAPACITY;
   h->seq_len = seq_len;

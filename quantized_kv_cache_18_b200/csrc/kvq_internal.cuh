@@ -36,6 +36,7 @@
 namespace kvq {
 
 constexpr int kTB = 32;         // tokens per token block
+constexpr int kFp8RowBytes = 144;   // FP8 token row: 128 E4M3 codes, fp16 scale, 14 zero bytes (d = 128)
 constexpr int kMaxDecodeCtas = 160;   // decode launches use at most this many CTAs (one per SM)
 
 struct Geom {
@@ -46,6 +47,9 @@ struct Geom {
   int page_shift;              // paged: log2(page_recs)
   int num_pages;               // paged: pages in the pool
   int64_t pages_per_row;
+  int fp8;                     // TURBO mixed cache: window (and anchors) in FP8 token rows
+  int anchor;                  // fp8: anchor tokens A per row
+  unsigned char* anchors;      // fp8: [rows][2][A][kFp8RowBytes]
   int64_t groups_per_row;   // record capacity of a row
   int64_t rec_bytes;        // bytes of one group record
   int64_t tb_code_bytes;    // bytes of one TB's key (or value) codes
@@ -214,6 +218,7 @@ struct QuantArgs {
   const uint16_t* src_k;   // token 0 of group `src_group0` of row 0
   const uint16_t* src_v;
   int64_t src_row_stride;  // elements between rows
+  const unsigned char* src_fp8;   // TURBO mixed flush: FP8 window rows of the first token (ring layout), or null
   int64_t dst_group0;      // first record index written
   int n_groups;            // groups per row handled by this launch
 };
@@ -241,6 +246,11 @@ struct AttnArgs {
 void launch_kivi_quantize(const QuantArgs& a, cudaStream_t st);
 void launch_window_copy(const Geom& g, const uint16_t* k, const uint16_t* v, int64_t seq_len, int64_t t0,
                         int n, cudaStream_t st);
+// FP8 token rows of tokens t0 .. t0 + n - 1 of every row of a [rows][seq][d]
+// 16-bit input: row r's token j goes to dst + r * row_stride + kv * kv_stride +
+// (slot0 + j) * kFp8RowBytes.
+void launch_fp8_rows(const Geom& g, const uint16_t* k, const uint16_t* v, int64_t seq, int64_t t0, int n,
+                     unsigned char* dst, int64_t row_stride, int64_t kv_stride, int slot0, cudaStream_t st);
 void launch_append(const Geom& g, const uint16_t* k, const uint16_t* v, int slot, cudaStream_t st);
 void launch_kivi_attention(const AttnArgs& a, cudaStream_t st);
 void launch_clear_words(uint32_t* words, int n, cudaStream_t st);

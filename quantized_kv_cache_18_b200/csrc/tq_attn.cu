@@ -26,6 +26,7 @@
 //
 // Every wait is bounded; on expiry the CTA sets KVQ_DEV_WAIT_TIMEOUT and stops
 // computing, and the producer waits (bounded) for its copies in flight.
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "decode_common.cuh"
@@ -59,7 +60,12 @@ struct TL {
   static constexpr int OFF_BAR = OFF_Q + 2 * QSLOT;
   static constexpr int N_BAR = 2 * NST + 5;
   static constexpr int OFF_FLAG = OFF_BAR + N_BAR * 8;
-  static constexpr int SMEM = OFF_FLAG + 16;
+  static constexpr int OFF_ZERO = (OFF_FLAG + 16 + 15) / 16 * 16;   // a zero 16-bit row (FP8 chunks)
+  static constexpr int SMEM = OFF_ZERO + WROW;
+  // FP8 window / anchor chunk in a stage: K rows [32][144], V rows [32][144],
+  // then each consumer warp's fp16 rows of its 4 tokens (K 1 KB, V 1 KB)
+  static constexpr int FP8_SCR = 2 * kTqWin * kFp8RowBytes;
+  static_assert(FP8_SCR + kTqConsumers * 2048 <= STAGE, "FP8 chunk scratch exceeds a stage");
 };
 static_assert(TL::SMEM <= 227 * 1024, "TurboQuant decode kernel exceeds shared memory");
 
@@ -179,6 +185,7 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
     }
     mbar_init(bar_pi, 1);
     *abort_flag = 0;
+    for (int i = 0; i < C::WROW / 16; ++i) reinterpret_cast<uint4*>(smem + C::OFF_ZERO)[i] = make_uint4(0u, 0u, 0u, 0u);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
   }
@@ -187,10 +194,12 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
   TPart Pt;
   Pt.n_tb = a.n_groups;
   Pt.r = a.r;
-  Pt.n_wc = (a.r + kTqWin - 1) / kTqWin;
+  // window-type items: the window's chunks, then (mixed cache) the anchors' chunks
+  const int n_wcw = (a.r + kTqWin - 1) / kTqWin;
+  Pt.n_wc = n_wcw + gm.anchor / kTqWin;
   Pt.n_items = (int)(Pt.n_tb + Pt.n_wc);
-  Pt.tokb = 4 * D;
-  Pt.W_row = Pt.n_tb * kTqTbBytes + (int64_t)a.r * 4 * D;
+  Pt.tokb = gm.fp8 ? 2 * kFp8RowBytes : 4 * D;
+  Pt.W_row = Pt.n_tb * kTqTbBytes + (int64_t)(a.r + gm.anchor) * Pt.tokb;
   Pt.rows = (int64_t)gm.B * gm.Hkv;
   Pt.W_tot = Pt.rows * Pt.W_row;
   Pt.n_cta = gridDim.x;
@@ -226,6 +235,28 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
                 return;
               }
               copy_records(gm, row, first, cnt, kTqTbBytes, pages, dst, &bar_full[slot]);
+            } else if (gm.fp8) {
+              // FP8 token rows of a window chunk (ring) or an anchor chunk
+              const int j = (int)first;
+              const unsigned char *srck, *srcv;
+              int n;
+              if (j < n_wcw) {
+                const int t0 = j * kTqWin;
+                n = min(kTqWin, a.r - t0);
+                const int slot0 = (a.head + t0) % gm.cap;
+                srck = reinterpret_cast<const unsigned char*>(gm.window) +
+                       ((int64_t)row * 2 * gm.cap + slot0) * kFp8RowBytes;
+                srcv = srck + (int64_t)gm.cap * kFp8RowBytes;
+              } else {
+                const int t0 = (j - n_wcw) * kTqWin;
+                n = kTqWin;
+                srck = gm.anchors + ((int64_t)row * 2 * gm.anchor + t0) * kFp8RowBytes;
+                srcv = srck + (int64_t)gm.anchor * kFp8RowBytes;
+              }
+              const uint32_t bytes = (uint32_t)n * kFp8RowBytes;
+              mbar_expect_tx(&bar_full[slot], 2 * bytes);
+              bulk_g2s(dst, srck, bytes, &bar_full[slot]);
+              bulk_g2s(dst + kTqWin * kFp8RowBytes, srcv, bytes, &bar_full[slot]);
             } else {
               const int t0 = (int)first * kTqWin;
               const int n = min(kTqWin, a.r - t0);
@@ -464,6 +495,97 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
 #undef TQ_PV_KT
 #undef TQ_PV
       }
+    } else if (ok && win && gm.fp8) {
+      // ---------------------------------------------------------- FP8 window / anchor tokens 4cw..4cw+3
+      // The warp turns its 4 tokens' E4M3 codes into exact fp16 rows of its own
+      // scratch (its other ldmatrix rows read the zero row); the per-token
+      // scales multiply the scores and p in fp32.  q goes to fp16 for the mma.
+      const uint16_t* qraw = reinterpret_cast<const uint16_t*>(sq + kTqQPrepBytes);
+      const int j = (int)first;
+      const int n_wcw = (a.r + kTqWin - 1) / kTqWin;
+      const int n_tok = j < n_wcw ? min(kTqWin, a.r - j * kTqWin) : kTqWin;
+      const int t0 = 4 * cw;
+      const unsigned char* kb8 = st;
+      const unsigned char* vb8 = st + kTqWin * kFp8RowBytes;
+      unsigned char* scr = smem + slot * C::STAGE + C::FP8_SCR + cw * 2048;   // K rows 0..3, then V rows 0..3
+      {
+        const int tt = lane >> 3, c0 = 16 * (lane & 7);
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint4 w = lds128((kv ? vb8 : kb8) + (t0 + tt) * kFp8RowBytes + c0);
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+          uint32_t hv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(
+                (__nv_fp8x2_storage_t)((wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu), __NV_E4M3);
+            hv[e] = (uint32_t)h2.x | ((uint32_t)h2.y << 16);
+          }
+          uint4* outp = reinterpret_cast<uint4*>(scr + kv * 1024 + tt * C::WROW + c0 * 2);
+          outp[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          outp[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+        }
+      }
+      __syncwarp();
+      const unsigned char* zero = smem + C::OFF_ZERO;
+      float sw[4] = {0.f, 0.f, 0.f, 0.f};
+      const int mi = lane >> 3, ri = lane & 7;
+      const unsigned char* krowp = ri < 4 ? scr + ri * C::WROW : zero;
+#pragma unroll
+      for (int kt2 = 0; kt2 < NKT / 2; ++kt2) {
+        uint32_t bk[4];
+        ldsm_x4(bk, krowp + (16 * (2 * kt2 + (mi >> 1)) + 8 * (mi & 1)) * 2);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int kt = 2 * kt2 + h2;
+          const uint32_t aq[4] = {
+              head_ok ? in16x2_to_h2(*reinterpret_cast<const uint32_t*>(qraw + gr * D + 16 * kt + 2 * tc), gm.dtype)
+                      : 0u,
+              0u,
+              head_ok ? in16x2_to_h2(*reinterpret_cast<const uint32_t*>(qraw + gr * D + 16 * kt + 8 + 2 * tc),
+                                     gm.dtype)
+                      : 0u,
+              0u};
+          mma_f16_16816(sw, aq, bk[2 * h2], bk[2 * h2 + 1]);
+        }
+      }
+      float xv[2], vsc[2];
+      float mt = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = t0 + 2 * tc + e;
+        const bool valid = head_ok && tc < 2 && t < n_tok;
+        const int tr = min(t, kTqWin - 1);
+        const float ks = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(kb8 + tr * kFp8RowBytes + D)));
+        vsc[e] = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(vb8 + tr * kFp8RowBytes + D)));
+        xv[e] = valid ? sw[e] * ks * a.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, xv[e]);
+      }
+      rescale_to(quad_max(mt));
+      float pw[2], pt[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        pw[e] = xv[e] == -INFINITY ? 0.f : fast_exp2(xv[e] - m);
+        l += pw[e];
+        pt[e] = xv[e] == -INFINITY ? 0.f : pw[e] * vsc[e];   // a masked token's scale may be stale bytes
+      }
+      const __half2 hi = __floats2half2_rn(pt[0], pt[1]);
+      const float2 hb = __half22float2(hi);
+      const __half2 lo = __floats2half2_rn(pt[0] - hb.x, pt[1] - hb.y);
+      const uint32_t apw[4] = {h2_as_u32(hi), h2_as_u32(lo), 0u, 0u};
+      const uint32_t vmask = (t0 + 2 * tc < n_tok ? 0x0000FFFFu : 0u) | (t0 + 2 * tc + 1 < n_tok ? 0xFFFF0000u : 0u);
+      const unsigned char* vrowp = ri < 4 ? scr + 1024 + ri * C::WROW : zero;
+#pragma unroll
+      for (int n4 = 0; n4 < NNT / 4; ++n4) {
+        uint32_t bv[4];
+        ldsm_x4_t(bv, vrowp + 8 * (4 * n4 + mi) * 2);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) mma_f16_16816(o[4 * n4 + jj], apw, bv[jj] & vmask, 0u);
+      }
+      // the scratch's generic writes come before the copy that will reuse this
+      // stage (async proxy), which the empty barrier alone does not order
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      __syncwarp();
     } else if (ok && win) {
       // ---------------------------------------------------------- window tokens 4cw..4cw+3 (exact 16-bit)
       const uint16_t* qraw = reinterpret_cast<const uint16_t*>(sq + kTqQPrepBytes);

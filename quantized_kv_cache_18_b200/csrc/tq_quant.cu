@@ -19,6 +19,7 @@
 // products on the CUDA cores (keys: Pi U and S E, values: Pi U); with the
 // Walsh-Hadamard rotation, Pi U is the in-register fast transform instead
 // (7 add/sub stages per vector), leaving S E as the one product.
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "kvq_internal.cuh"
@@ -42,7 +43,8 @@ struct QSmem {
   static constexpr int NK = SG + kTok * kTqM;                 // double [32] key norms
   static constexpr int NV = NK + kTok * 8;                    // double [32] value norms
   static constexpr int ESQ = NV + kTok * 8;                   // double [32] ||e||^2
-  static constexpr int BYTES = ESQ + kTok * 8;
+  static constexpr int XF = ESQ + kTok * 8;                   // float [32][128] FP8 input tile, exact values
+  static constexpr int BYTES = XF + kTok * kTqD * 4;
 };
 
 __device__ __forceinline__ double warp_sum_d(double x) {
@@ -88,11 +90,12 @@ __device__ __forceinline__ void fwht128(float v[4], int lane) {
   v[3] = a1 - a3;
 }
 
-// Norms and unit vectors of the 32 tokens in X: warp w handles tokens 4w..4w+3.
+// Norms and unit vectors of the 32 tokens in X (16-bit) or XF (exact fp32
+// values of FP8 rows): warp w handles tokens 4w..4w+3.
 // With wht, U receives y = H u / sqrt(d) instead of u (the rotation applied by
 // the fast transform; Pi = H / sqrt(d) holds exactly +-fp32(1 / sqrt(d))).
-__device__ __forceinline__ uint32_t unit_vectors(const uint16_t* X, float* U, double* nrm, int dtype, int warp,
-                                                 int lane, bool wht) {
+__device__ __forceinline__ uint32_t unit_vectors(const uint16_t* X, const float* XF, float* U, double* nrm,
+                                                 int dtype, int warp, int lane, bool wht) {
   uint32_t flags = 0;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -101,7 +104,7 @@ __device__ __forceinline__ uint32_t unit_vectors(const uint16_t* X, float* U, do
     double s = 0.0;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      x[r] = in16_to_float(X[t * kTqD + lane + 32 * r], dtype);
+      x[r] = XF != nullptr ? XF[t * kTqD + lane + 32 * r] : in16_to_float(X[t * kTqD + lane + 32 * r], dtype);
       if (!isfinite(x[r])) flags |= KVQ_DEV_NONFINITE_INPUT;
       s += (double)x[r] * (double)x[r];
     }
@@ -136,6 +139,7 @@ __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) 
   double* sNK = reinterpret_cast<double*>(smem + QSmem::NK);
   double* sNV = reinterpret_cast<double*>(smem + QSmem::NV);
   double* sESQ = reinterpret_cast<double*>(smem + QSmem::ESQ);
+  float* sXF = reinterpret_cast<float*>(smem + QSmem::XF);
   __shared__ float s_thr[8], s_lv[8];
   __shared__ uint32_t s_flags;
 
@@ -165,11 +169,26 @@ __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) 
     const int blk = (int)(task - (int64_t)row * a.n_groups);
     for (int kv = 0; kv < 2; ++kv) {
       // ---------------------------------------------------------- stage the 32 tokens
-      const uint16_t* src = (kv == 0 ? a.src_k : a.src_v) + (int64_t)row * a.src_row_stride + (int64_t)blk * kTok * kTqD;
-      for (int i = tid; i < kTok * kTqD / 8; i += kQThreads)
-        reinterpret_cast<uint4*>(sX)[i] = ldg_nc_v4(reinterpret_cast<const uint4*>(src) + i);
+      if (a.src_fp8 == nullptr) {
+        const uint16_t* src =
+            (kv == 0 ? a.src_k : a.src_v) + (int64_t)row * a.src_row_stride + (int64_t)blk * kTok * kTqD;
+        for (int i = tid; i < kTok * kTqD / 8; i += kQThreads)
+          reinterpret_cast<uint4*>(sX)[i] = ldg_nc_v4(reinterpret_cast<const uint4*>(src) + i);
+      } else {
+        // FP8 window rows (ring layout): x_hat = e4m3(code) * s, exact in fp32
+        const unsigned char* src8 = a.src_fp8 + (int64_t)row * 2 * gm.cap * kFp8RowBytes +
+                                    (int64_t)kv * gm.cap * kFp8RowBytes + (int64_t)blk * kTok * kFp8RowBytes;
+        for (int i = tid; i < kTok * kTqD; i += kQThreads) {
+          const int t = i / kTqD, c = i - t * kTqD;
+          const unsigned char* rowp = src8 + t * kFp8RowBytes;
+          const float sc = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(rowp + kTqD)));
+          const float code = __half2float(__half(__nv_cvt_fp8_to_halfraw(rowp[c], __NV_E4M3)));
+          sXF[i] = code * sc;
+        }
+      }
       __syncthreads();
-      flags |= unit_vectors(sX, sU, kv == 0 ? sNK : sNV, gm.dtype, warp, lane, gm.rot_wht != 0);
+      flags |= unit_vectors(sX, a.src_fp8 != nullptr ? sXF : nullptr, sU, kv == 0 ? sNK : sNV, gm.dtype, warp, lane,
+                            gm.rot_wht != 0);
       __syncthreads();
       // ---------------------------------------------------------- y = Pi u, codes
       float acc[4][4];

@@ -50,6 +50,8 @@ class Workload:
     v_channel_outliers: bool = False          # TurboQuant: V gets the K channel recipe
     qjl_dim: int = 128
     rotation: str = "qr"                      # TurboQuant: "qr" (random orthogonal) or "wht"
+    fp8_recent: bool = False                  # TurboQuant: FP8 window + anchors (mixed-format cache)
+    anchor_tokens: int = 0
     seed: int = 0
 
     @property
@@ -82,6 +84,9 @@ WORKLOADS: Dict[str, Workload] = {
     # The same with the Walsh-Hadamard rotation H / sqrt(d) instead of the QR one.
     "tqw": Workload("tqw", "turbo", 8, 8, 32, 128, 32768, "bf16", 3, 32, 128,
                     v_outlier_frac=0.0, v_channel_outliers=True, rotation="wht", seed=4),
+    # Mixed-format cache: the first 128 tokens and the window in FP8, the rest in TQ3.
+    "tqm": Workload("tqm", "turbo", 8, 8, 32, 128, 32768, "bf16", 3, 32, 128,
+                    v_outlier_frac=0.0, v_channel_outliers=True, fp8_recent=True, anchor_tokens=128, seed=4),
 }
 
 

@@ -78,9 +78,14 @@ def _near_fp16_midpoint(x):
 def check_blocks(got_rec, w, params, k_bits, v_bits):
     """got_rec: uint8 [n_tb][4032] from the GPU; k_bits, v_bits: the quantized
     tokens (uint16 [32 n_tb][d]).  Returns the ambiguous fraction."""
+    return check_blocks_values(got_rec, w, params, decode16(k_bits, w.dtype), decode16(v_bits, w.dtype))
+
+
+def check_blocks_values(got_rec, w, params, k, v):
+    """As check_blocks, with the quantized tokens as float64 vectors [32 n_tb][d]."""
     Pi, S, lv, th = params
-    kq = turbo.quantize(decode16(k_bits, w.dtype), Pi, lv, th, S)
-    vq = turbo.quantize(decode16(v_bits, w.dtype), Pi, lv, th)
+    kq = turbo.quantize(k, Pi, lv, th, S)
+    vq = turbo.quantize(v, Pi, lv, th)
     kc, kn, kg, ks, vc, vn = turbo_cache.unpack_tbs(got_rec, w.head_dim, w.qjl_dim)
     n_amb = 0
     n_dec = 0
