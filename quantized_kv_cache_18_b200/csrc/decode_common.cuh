@@ -65,10 +65,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 // Records first .. first + cnt - 1 of a row (cnt <= 16) into shared memory,
 // in steps so that a paged cache's page-id loads are in flight while the
 // producer waits for a free stage:
-//   record_pages  issues the loads of the ids of the pages the records touch
-//                 (nothing when contiguous);
+//   record_pages  issues the loads of the ids of the pages the records touch;
 //   pages_valid   (after the wait) whether all of them are in the pool;
-//   copy_records  arms `bar` and issues one copy (contiguous) or one per page.
+//   copy_records  arms `bar` and issues one copy per page.
+// (Paged caches only; a contiguous stage is one copy issued directly.)
 struct RecordPages {
   int32_t ids[16];
   int nr, p0;
@@ -76,8 +76,6 @@ struct RecordPages {
 // Page sizes are powers of two (page_shift = log2 of records per page), so the
 // page arithmetic is shifts and masks on 32-bit record indices.
 __device__ __forceinline__ void record_pages(const Geom& gm, int row, int64_t first, int cnt, RecordPages& pg) {
-  pg.nr = 0;
-  if (gm.page_table == nullptr) return;
   const int f = (int)first, sh = gm.page_shift;
   pg.p0 = f >> sh;
   pg.nr = ((f + cnt - 1) >> sh) - pg.p0 + 1;
@@ -99,10 +97,6 @@ __device__ __forceinline__ bool pages_valid(const Geom& gm, const RecordPages& p
 __device__ __forceinline__ void copy_records(const Geom& gm, int row, int64_t first, int cnt, int rec_bytes,
                                              const RecordPages& pg, unsigned char* dst, uint64_t* bar) {
   mbar_expect_tx(bar, (uint32_t)cnt * rec_bytes);
-  if (gm.page_table == nullptr) {
-    bulk_g2s(dst, record_ptr(gm, row, first), (uint32_t)cnt * rec_bytes, bar);
-    return;
-  }
   const int f = (int)first, sh = gm.page_shift, mask = (1 << sh) - 1;
   if (pg.nr == 1) {
     bulk_g2s(dst, gm.records + (((int64_t)pg.ids[0] << sh) | (f & mask)) * rec_bytes, (uint32_t)cnt * rec_bytes,

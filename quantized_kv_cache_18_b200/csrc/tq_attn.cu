@@ -220,15 +220,22 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
             if (*abort_flag) return;
             const int slot = s % C::NST;
             // a paged stage's page ids load while the producer waits for the slot
+            // (a contiguous cache skips all page bookkeeping: this thread's
+            // per-stage work is on the critical path)
+            const bool paged = !win && gm.page_table != nullptr;
             RecordPages pages;
-            if (!win) record_pages(gm, row, first, cnt, pages);
+            if (paged) record_pages(gm, row, first, cnt, pages);
             if (s >= C::NST && !mbar_wait(&bar_empty[slot], ((s / C::NST) - 1) & 1, abort_flag)) {
               atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
               *abort_flag = 1;
               return;
             }
             unsigned char* dst = smem + slot * C::STAGE;
-            if (!win) {
+            if (!win && !paged) {
+              const uint32_t bytes = (uint32_t)cnt * kTqTbBytes;
+              mbar_expect_tx(&bar_full[slot], bytes);
+              bulk_g2s(dst, record_ptr(gm, row, first), bytes, &bar_full[slot]);
+            } else if (!win) {
               if (!pages_valid(gm, pages)) {
                 atomicOr(gm.status, KVQ_DEV_BAD_PAGE);
                 *abort_flag = 1;
