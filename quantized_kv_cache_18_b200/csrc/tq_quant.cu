@@ -14,11 +14,15 @@
 // 1; the zero vector has u = 0.  Codes are decided on y computed in fp32 (Pi
 // in fp32, fp32 accumulation).
 //
-// One persistent CTA per SM keeps Pi^T and S^T (fp32, 64 KB each) in shared
-// memory and loops over (row, block) tasks.  Each task runs three 32 x 128 x 128
-// products on the CUDA cores (keys: Pi U and S E, values: Pi U); with the
-// Walsh-Hadamard rotation, Pi U is the in-register fast transform instead
-// (7 add/sub stages per vector), leaving S E as the one product.
+// One persistent CTA per SM keeps 16 Pi and S in shared memory as mma.sync
+// A fragments, each split into fp16 hi + lo, and loops over (row, block)
+// tasks.  Each task runs three 128 x 128 x 32 products on the tensor cores
+// (keys: Pi U and S E, values: Pi U) as hi*hi + hi*lo + lo*hi with fp32
+// accumulation (about 22 significant bits, the dropped lo*lo term below
+// 2^-22 of each product); U is scaled by 16 and E by 64 so that the lo parts
+// stay clear of fp16 subnormals.  With the Walsh-Hadamard rotation, Pi U is
+// the in-register fast transform instead (7 add/sub stages per vector),
+// leaving S E as the one product.
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -32,18 +36,21 @@ constexpr int kQThreads = 256;
 constexpr int kTok = 32;
 
 struct QSmem {
-  static constexpr int PIT = 0;                               // float [128][128]
-  static constexpr int ST = PIT + kTqD * kTqD * 4;            // float [128][128]
-  static constexpr int X = ST + kTqD * kTqM * 4;              // uint16 [32][128] input tile
-  static constexpr int U = X + kTok * kTqD * 2;               // float [128][32]
-  static constexpr int E = U + kTqD * kTok * 4;               // float [128][32]
+  // A operands of the two products, split fp16 hi + lo, in mma fragment order:
+  // [m-tile 8][k-tile 8][lane 32] x (hi a0..a3, lo a0..a3) = 32 bytes
+  static constexpr int AP = 0;                                // 16 Pi
+  static constexpr int AS = AP + 8 * 8 * 32 * 32;             // S
+  static constexpr int X = AS + 8 * 8 * 32 * 32;              // uint16 [32][128] input tile
+  static constexpr int U = X + kTok * kTqD * 2;               // float [128][32] unit vectors (or y)
+  static constexpr int E = U + kTqD * kTok * 4;               // float [128][32] key residuals
   static constexpr int CK = E + kTqD * kTok * 4;              // uint8 [32][128] key codes
   static constexpr int CV = CK + kTok * kTqD;                 // uint8 [32][128] value codes
   static constexpr int SG = CV + kTok * kTqD;                 // uint8 [32][128] sign bits
   static constexpr int NK = SG + kTok * kTqM;                 // double [32] key norms
   static constexpr int NV = NK + kTok * 8;                    // double [32] value norms
-  static constexpr int ESQ = NV + kTok * 8;                   // double [32] ||e||^2
-  static constexpr int XF = ESQ + kTok * 8;                   // float [32][128] FP8 input tile, exact values
+  static constexpr int ESQ = NV + kTok * 8;                   // double [8 warps][32] partial ||e||^2
+  static constexpr int XF = ESQ + 8 * kTok * 8;               // float [32][128] FP8 input tile, exact values;
+  static constexpr int BF = XF;                               // reused for the B operands [8][4][32] x 16 B
   static constexpr int BYTES = XF + kTok * kTqD * 4;
 };
 
@@ -53,21 +60,69 @@ __device__ __forceinline__ double warp_sum_d(double x) {
   return x;
 }
 
-// acc[a][b] = sum_j WT[j][4 ti + a] * X[j][4 tt + b]   (WT [128][128], X [128][32])
-__device__ __forceinline__ void matvec_tile(const float* WT, const float* X, int ti, int tt, float acc[4][4]) {
+// fp16 hi + lo split of two fp32 values, packed as fp16x2 pairs
+__device__ __forceinline__ void split2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(v0, v1);
+  const float2 hf = __half22float2(h);
+  hi = h2_as_u32(h);
+  lo = h2_as_u32(__floats2half2_rn(v0 - hf.x, v1 - hf.y));
+}
+
+// A operand of a 128 x 128 product (W[i][j] * scale, i = output row, j =
+// summed index; W read from global memory, stored row-major, or transposed
+// as W[j][i]) into mma fragment order, split hi + lo.
+__device__ __forceinline__ void build_a_frags(const float* W, float scale, bool transposed, unsigned char* dst,
+                                              int tid) {
+  auto w = [&](int i, int j) { return __ldg(transposed ? W + j * kTqD + i : W + i * kTqD + j) * scale; };
+  for (int q = tid; q < 8 * 8 * 32; q += kQThreads) {
+    const int mt = q >> 8, kt = (q >> 5) & 7, lane = q & 31;
+    const int gr = lane >> 2, tc = lane & 3;
+    const int r0 = 16 * mt + gr, c0 = 16 * kt + 2 * tc;
+    uint32_t h[4], l[4];
+    split2(w(r0, c0), w(r0, c0 + 1), h[0], l[0]);
+    split2(w(r0 + 8, c0), w(r0 + 8, c0 + 1), h[1], l[1]);
+    split2(w(r0, c0 + 8), w(r0, c0 + 9), h[2], l[2]);
+    split2(w(r0 + 8, c0 + 8), w(r0 + 8, c0 + 9), h[3], l[3]);
+    uint4* o = reinterpret_cast<uint4*>(dst + q * 32);
+    o[0] = make_uint4(h[0], h[1], h[2], h[3]);
+    o[1] = make_uint4(l[0], l[1], l[2], l[3]);
+  }
+}
+
+// B operand (K = 128 summed index j, N = 32 tokens) from X[j][32] * scale into
+// fragment order [k-tile 8][n-tile 4][lane 32] x (hi b0, hi b1, lo b0, lo b1).
+__device__ __forceinline__ void build_b_frags(const float* X, float scale, unsigned char* dst, int tid) {
+  for (int q = tid; q < 8 * 4 * 32; q += kQThreads) {
+    const int kt = q >> 7, nt = (q >> 5) & 3, lane = q & 31;
+    const int gr = lane >> 2, tc = lane & 3;
+    const int j0 = 16 * kt + 2 * tc, t = 8 * nt + gr;
+    uint32_t h0, l0, h1, l1;
+    split2(X[j0 * kTok + t] * scale, X[(j0 + 1) * kTok + t] * scale, h0, l0);
+    split2(X[(j0 + 8) * kTok + t] * scale, X[(j0 + 9) * kTok + t] * scale, h1, l1);
+    reinterpret_cast<uint4*>(dst)[q] = make_uint4(h0, h1, l0, l1);
+  }
+}
+
+// acc[nt] = rows 16 mt .. 16 mt + 15 (the warp's m-tile) x tokens 8 nt .. 8 nt + 7
+// of A B, as hi hi + hi lo + lo hi (about 22 bits; the lo lo term is dropped).
+// C layout: acc[nt][0..1] = row 16 mt + gr, tokens 8 nt + 2 tc + {0, 1};
+// acc[nt][2..3] = row 16 mt + 8 + gr, the same tokens.
+__device__ __forceinline__ void product_tile(const unsigned char* A, const unsigned char* B, int mt, int lane,
+                                             float acc[4][4]) {
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+  for (int kt = 0; kt < 8; ++kt) {
+    const uint4 ah = *reinterpret_cast<const uint4*>(A + ((mt * 8 + kt) * 32 + lane) * 32);
+    const uint4 al = *reinterpret_cast<const uint4*>(A + ((mt * 8 + kt) * 32 + lane) * 32 + 16);
+    const uint32_t ahv[4] = {ah.x, ah.y, ah.z, ah.w}, alv[4] = {al.x, al.y, al.z, al.w};
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-#pragma unroll 4
-  for (int j = 0; j < kTqD; ++j) {
-    const float4 w = *reinterpret_cast<const float4*>(WT + j * kTqD + 4 * ti);
-    const float4 x = *reinterpret_cast<const float4*>(X + j * kTok + 4 * tt);
-    const float wv[4] = {w.x, w.y, w.z, w.w}, xv[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(wv[a], xv[b], acc[a][b]);
+    for (int nt = 0; nt < 4; ++nt) {
+      const uint4 b = reinterpret_cast<const uint4*>(B)[(kt * 4 + nt) * 32 + lane];
+      mma_f16_16816(acc[nt], ahv, b.x, b.y);
+      mma_f16_16816(acc[nt], ahv, b.z, b.w);
+      mma_f16_16816(acc[nt], alv, b.x, b.y);
+    }
   }
 }
 
@@ -128,8 +183,6 @@ __device__ __forceinline__ uint32_t unit_vectors(const uint16_t* X, const float*
 
 __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  float* sPiT = reinterpret_cast<float*>(smem + QSmem::PIT);
-  float* sST = reinterpret_cast<float*>(smem + QSmem::ST);
   uint16_t* sX = reinterpret_cast<uint16_t*>(smem + QSmem::X);
   float* sU = reinterpret_cast<float*>(smem + QSmem::U);
   float* sE = reinterpret_cast<float*>(smem + QSmem::E);
@@ -140,20 +193,21 @@ __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) 
   double* sNV = reinterpret_cast<double*>(smem + QSmem::NV);
   double* sESQ = reinterpret_cast<double*>(smem + QSmem::ESQ);
   float* sXF = reinterpret_cast<float*>(smem + QSmem::XF);
+  unsigned char* sBF = smem + QSmem::BF;
   __shared__ float s_thr[8], s_lv[8];
   __shared__ uint32_t s_flags;
 
   const Geom& gm = a.geom;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ti = lane, tt = warp;   // matvec tile: rows 4ti..4ti+3, tokens 4tt..4tt+3
+  const int gr = lane >> 2, tc = lane & 3;   // C fragment: rows 16 warp + gr (+8), tokens 8 nt + 2 tc (+1)
 
   {
-    const uint4* p = reinterpret_cast<const uint4*>(gm.params + kTqPiT);
-    uint4* d = reinterpret_cast<uint4*>(sPiT);
-    for (int i = tid; i < 2 * kTqD * kTqD / 4; i += kQThreads) d[i] = __ldg(p + i);   // Pi^T then S^T
+    const float* P = reinterpret_cast<const float*>(gm.params);
+    if (!gm.rot_wht) build_a_frags(P + kTqPi / 4, 16.f, false, smem + QSmem::AP, tid);
+    build_a_frags(P + kTqST / 4, 1.f, true, smem + QSmem::AS, tid);
     if (tid < 8) {
-      s_thr[tid] = reinterpret_cast<const float*>(gm.params + kTqThr)[tid];
-      s_lv[tid] = reinterpret_cast<const float*>(gm.params + kTqLevels)[tid];
+      s_thr[tid] = P[kTqThr / 4 + tid];
+      s_lv[tid] = P[kTqLevels / 4 + tid];
     }
     if (tid == 0) s_flags = 0;
   }
@@ -194,47 +248,62 @@ __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) 
       float acc[4][4];
       if (gm.rot_wht) {
 #pragma unroll
-        for (int a4 = 0; a4 < 4; ++a4) {
-          const float4 y4 = *reinterpret_cast<const float4*>(sU + (4 * ti + a4) * kTok + 4 * tt);
-          acc[a4][0] = y4.x;
-          acc[a4][1] = y4.y;
-          acc[a4][2] = y4.z;
-          acc[a4][3] = y4.w;
-        }
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const float2 y2 = *reinterpret_cast<const float2*>(sU + (16 * warp + gr + 8 * h) * kTok + 8 * nt + 2 * tc);
+            acc[nt][2 * h] = y2.x;
+            acc[nt][2 * h + 1] = y2.y;
+          }
       } else {
-        matvec_tile(sPiT, sU, ti, tt, acc);
+        build_b_frags(sU, 16.f, sBF, tid);
+        __syncthreads();
+        product_tile(smem + QSmem::AP, sBF, warp, lane, acc);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[nt][e] *= 1.f / 256.f;
       }
       uint8_t* codes = kv == 0 ? sCK : sCV;
-      double esq[4] = {0.0, 0.0, 0.0, 0.0};
+      double esq[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
 #pragma unroll
-      for (int i4 = 0; i4 < 4; ++i4)
+      for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const float y = acc[i4][b];
+        for (int e = 0; e < 4; ++e) {
+          const float y = acc[nt][e];
           int c = 0;
 #pragma unroll
           for (int k = 0; k < 7; ++k) c += y > thr[k] ? 1 : 0;
-          const int i = 4 * ti + i4, t = 4 * tt + b;
+          const int i = 16 * warp + gr + 8 * (e >> 1), t = 8 * nt + 2 * tc + (e & 1);
           codes[t * kTqD + i] = (uint8_t)c;
           if (kv == 0) {
-            const float e = y - s_lv[c];
-            sE[i * kTok + t] = e;
-            esq[b] += (double)e * (double)e;
+            const float r = y - s_lv[c];
+            sE[i * kTok + t] = r;
+            esq[nt][e & 1] += (double)r * (double)r;
           }
         }
       if (kv == 0) {
+        // partial ||e||^2 of the warp's 16 rows, per token
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const double s = warp_sum_d(esq[b]);
-          if (lane == 0) sESQ[4 * tt + b] = s;
-        }
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            double s = esq[nt][b];
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            s += __shfl_xor_sync(0xffffffffu, s, 8);
+            s += __shfl_xor_sync(0xffffffffu, s, 16);
+            if (gr == 0) sESQ[warp * kTok + 8 * nt + 2 * tc + b] = s;
+          }
         __syncthreads();
         // ---------------------------------------------------------- sketch signs of S e
-        matvec_tile(sST, sE, ti, tt, acc);
+        build_b_frags(sE, 64.f, sBF, tid);
+        __syncthreads();
+        product_tile(smem + QSmem::AS, sBF, warp, lane, acc);
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4)
+        for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-          for (int b = 0; b < 4; ++b) sSG[(4 * tt + b) * kTqM + 4 * ti + i4] = acc[i4][b] >= 0.f ? 1 : 0;
+          for (int e = 0; e < 4; ++e)
+            sSG[(8 * nt + 2 * tc + (e & 1)) * kTqM + 16 * warp + gr + 8 * (e >> 1)] = acc[nt][e] >= 0.f ? 1 : 0;
       }
       __syncthreads();
     }
@@ -288,7 +357,10 @@ __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) 
         const int entry = 8 * tc + 4 * kt + 2 * rho + e;
         const double nk = sNK[t], nv = sNV[t];
         const __half hn = __double2half(nk);
-        const __half hg = __double2half(nk * sqrt(sESQ[t]));
+        double esq = 0.0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) esq += sESQ[w * kTok + t];
+        const __half hg = __double2half(nk * sqrt(esq));
         const __half hv = __double2half(nv);
         if (isinf(__half2float(hn)) || isinf(__half2float(hg)) || isinf(__half2float(hv)))
           flags |= KVQ_DEV_PARAM_OVERFLOW;
