@@ -11,6 +11,18 @@
 namespace kvq {
 namespace {
 
+// floor(a / b) for 0 <= a < 2^50 and b > 0, given rb = 1 / b rounded to double.
+// The 64-bit integer division is a long serial subroutine (the partition math
+// of a decode launch took microseconds with it); the double estimate is
+// within one of the quotient and is then corrected exactly in integers.
+__device__ __forceinline__ int64_t div_floor(int64_t a, int64_t b, double rb) {
+  int64_t q = (int64_t)((double)a * rb);
+  while (q > 0 && q * b > a) --q;
+  while ((q + 1) * b <= a) ++q;
+  return q;
+}
+__device__ __forceinline__ double recip(int64_t b) { return __drcp_rn((double)b); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(b)), "r"(count) : "memory");

@@ -97,28 +97,38 @@ struct K {
 struct Part {
   int64_t n_g, W_row, W_tot, rows;
   int n_items, n_wc, r, rec, tokb, n_cta;
+  double r_cta, r_row, r_tot, r_rec, r_wb, r_items;   // reciprocals (div_floor)
+  __device__ void set_reciprocals() {
+    r_cta = recip(n_cta);
+    r_row = recip(W_row);
+    r_tot = recip(W_tot);
+    r_rec = recip(rec);
+    r_wb = recip((int64_t)kWinTok * tokb);
+    r_items = recip(n_items);
+  }
+  __device__ int64_t row_of(int64_t item) const { return div_floor(item, n_items, r_items); }
   __device__ int64_t start_in_row(int k) const {
     return k < n_g ? (int64_t)k * rec : n_g * rec + (int64_t)(k - n_g) * kWinTok * tokb;
   }
-  __device__ int64_t lo(int c) const { return (int64_t)c * W_tot / n_cta; }
+  __device__ int64_t lo(int c) const { return div_floor((int64_t)c * W_tot, n_cta, r_cta); }
   // first global item whose start byte is >= x
   __device__ int64_t first_item(int64_t x) const {
-    const int64_t row = x / W_row;
+    const int64_t row = div_floor(x, W_row, r_row);
     if (row >= rows) return rows * n_items;
     const int64_t off = x - row * W_row;
     int64_t k;
     if (off <= n_g * rec) {
-      k = (off + rec - 1) / rec;
+      k = div_floor(off + rec - 1, rec, r_rec);
     } else {
       const int64_t wb = (int64_t)kWinTok * tokb;
-      k = n_g + (off - n_g * rec + wb - 1) / wb;
+      k = n_g + div_floor(off - n_g * rec + wb - 1, wb, r_wb);
     }
     return row * n_items + k;   // k == n_items rolls into the next row's item 0
   }
   __device__ int cta_of(int64_t item) const {
-    const int64_t row = item / n_items;
+    const int64_t row = row_of(item);
     const int64_t st = row * W_row + start_in_row((int)(item - row * n_items));
-    int c = (int)(st * n_cta / W_tot);
+    int c = (int)div_floor(st * n_cta, W_tot, r_tot);
     if (c > n_cta - 1) c = n_cta - 1;
     while (c + 1 < n_cta && lo(c + 1) <= st) ++c;
     while (c > 0 && lo(c) > st) --c;
@@ -134,7 +144,7 @@ template <int SG, class FC, class FS, class FE>
 __device__ __forceinline__ void for_each_chunk(const Part& P, int64_t i0, int64_t i1, FC f, FS seg, FE seg_end) {
   int s = 0;
   if (i0 >= i1) return;
-  for (int64_t row = i0 / P.n_items; row * P.n_items < i1; ++row) {
+  for (int64_t row = P.row_of(i0); row * P.n_items < i1; ++row) {
     const int64_t a = max(i0, row * P.n_items) - row * P.n_items;
     const int64_t b = min(i1, (row + 1) * P.n_items) - row * P.n_items;
     if (a >= b) continue;
@@ -207,11 +217,12 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
   Pt.rows = (int64_t)gm.B * gm.Hkv;
   Pt.W_tot = Pt.rows * Pt.W_row;
   Pt.n_cta = gridDim.x;
+  Pt.set_reciprocals();
   const int cta = blockIdx.x;
   const int64_t i0 = Pt.first_item(Pt.lo(cta));
   const int64_t i1 = Pt.first_item(Pt.lo(cta + 1));
   auto nop_seg = [](int) {};
-  const int64_t last_row = i1 > i0 ? (i1 - 1) / Pt.n_items : -1;
+  const int64_t last_row = i1 > i0 ? Pt.row_of(i1 - 1) : -1;
 
   // Merges the warp states of one segment (state buffer sb) and writes the
   // row's output when this CTA covers the whole row, else the CTA's partial
@@ -279,7 +290,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
     if (!*s_last) return;
     // Last CTA of the row: online log-sum-exp over the np partials, the loads
     // of up to kMB partials (o, m, l) in flight together.
-    constexpr int kMB = 4;
+    constexpr int kMB = 8;
     const float* ws_row = a.ws + (int64_t)(c_first + row) * g * DP;
     for (int e4 = tid; e4 < g * D / 4; e4 += nth) {
       const int h = e4 / (D / 4), c = 4 * (e4 - h * (D / 4));

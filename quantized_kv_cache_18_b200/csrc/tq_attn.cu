@@ -95,27 +95,37 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t w) {
 struct TPart {
   int64_t n_tb, W_row, W_tot, rows;
   int n_items, n_wc, r, tokb, n_cta;
+  double r_cta, r_row, r_tot, r_tb, r_wb, r_items;   // reciprocals (div_floor)
+  __device__ void set_reciprocals() {
+    r_cta = recip(n_cta);
+    r_row = recip(W_row);
+    r_tot = recip(W_tot);
+    r_tb = recip(kTqTbBytes);
+    r_wb = recip((int64_t)kTqWin * tokb);
+    r_items = recip(n_items);
+  }
+  __device__ int64_t row_of(int64_t item) const { return div_floor(item, n_items, r_items); }
   __device__ int64_t start_in_row(int k) const {
     return k < n_tb ? (int64_t)k * kTqTbBytes : n_tb * kTqTbBytes + (int64_t)(k - n_tb) * kTqWin * tokb;
   }
-  __device__ int64_t lo(int c) const { return (int64_t)c * W_tot / n_cta; }
+  __device__ int64_t lo(int c) const { return div_floor((int64_t)c * W_tot, n_cta, r_cta); }
   __device__ int64_t first_item(int64_t x) const {
-    const int64_t row = x / W_row;
+    const int64_t row = div_floor(x, W_row, r_row);
     if (row >= rows) return rows * n_items;
     const int64_t off = x - row * W_row;
     int64_t k;
     if (off <= n_tb * kTqTbBytes) {
-      k = (off + kTqTbBytes - 1) / kTqTbBytes;
+      k = div_floor(off + kTqTbBytes - 1, kTqTbBytes, r_tb);
     } else {
       const int64_t wb = (int64_t)kTqWin * tokb;
-      k = n_tb + (off - n_tb * kTqTbBytes + wb - 1) / wb;
+      k = n_tb + div_floor(off - n_tb * kTqTbBytes + wb - 1, wb, r_wb);
     }
     return row * n_items + k;
   }
   __device__ int cta_of(int64_t item) const {
-    const int64_t row = item / n_items;
+    const int64_t row = row_of(item);
     const int64_t st = row * W_row + start_in_row((int)(item - row * n_items));
-    int c = (int)(st * n_cta / W_tot);
+    int c = (int)div_floor(st * n_cta, W_tot, r_tot);
     if (c > n_cta - 1) c = n_cta - 1;
     while (c + 1 < n_cta && lo(c + 1) <= st) ++c;
     while (c > 0 && lo(c) > st) --c;
@@ -130,7 +140,7 @@ template <class FC, class FS, class FE>
 __device__ __forceinline__ void tq_for_each_chunk(const TPart& P, int64_t i0, int64_t i1, FC f, FS seg, FE seg_end) {
   int s = 0;
   if (i0 >= i1) return;
-  for (int64_t row = i0 / P.n_items; row * P.n_items < i1; ++row) {
+  for (int64_t row = P.row_of(i0); row * P.n_items < i1; ++row) {
     const int64_t a = max(i0, row * P.n_items) - row * P.n_items;
     const int64_t b = min(i1, (row + 1) * P.n_items) - row * P.n_items;
     if (a >= b) continue;
@@ -203,6 +213,7 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
   Pt.rows = (int64_t)gm.B * gm.Hkv;
   Pt.W_tot = Pt.rows * Pt.W_row;
   Pt.n_cta = gridDim.x;
+  Pt.set_reciprocals();
   const int cta = blockIdx.x;
   const int64_t i0 = Pt.first_item(Pt.lo(cta));
   const int64_t i1 = Pt.first_item(Pt.lo(cta + 1));
