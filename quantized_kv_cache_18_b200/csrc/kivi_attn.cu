@@ -47,7 +47,7 @@ namespace kvq {
 
 namespace {
 
-constexpr int kWinTok = 32;                     // tokens per window item
+constexpr int kWinTok = kDecodeWinTok;                     // tokens per window item
 
 template <int NC>
 __device__ __forceinline__ void consumer_bar() { named_bar_sync<NC * 32>(); }
@@ -56,7 +56,7 @@ __device__ __forceinline__ void consumer_bar() { named_bar_sync<NC * 32>(); }
 // to 4 heads, see the kernel comment), which runs 12 consumers.
 template <int BITS, int D, int G, bool TR>
 struct K {
-  static constexpr int NC = TR ? 12 : 8;                         // consumer warps
+  static constexpr int NC = TR ? kKiviConsumersTM : kKiviConsumersHM;   // consumer warps
   static constexpr int THREADS = (NC + 3) * 32;                  // + producer, prep, merge warps
   static constexpr int HS = TR ? 4 : 8;                          // heads per warp state
   static constexpr int DP = D + 4;                               // partial row (o[D], m, l, pad): 16-byte multiple
@@ -83,7 +83,7 @@ struct K {
   static constexpr int OFF_PW = OFF_S + 2 * SBUF_F * 4;          // per-warp P tile (TR): 32 tokens x 8 fp16
   static constexpr int OFF_Q = OFF_PW + (TR ? NC * 512 : 0);     // q ring: 2 slots x raw 16-bit q of 8 heads
   static constexpr int OFF_BAR = OFF_Q + 2 * 8 * D * 2;
-  static constexpr int OFF_FLAG = OFF_BAR + (3 * NST + 8) * 8;
+  static constexpr int OFF_FLAG = OFF_BAR + (3 * NST + 9) * 8;
   static constexpr int SMEM = OFF_FLAG + 16;
   static_assert(NST >= 2, "decode pipeline needs two stages");
   static_assert(SG <= 16, "a stage copies at most 16 records");
@@ -91,48 +91,22 @@ struct K {
 };
 
 // ------------------------------------------------------------------ work partition
-// Items of a row: groups 0..n_g-1, then window chunks of kWinTok tokens.  Item
-// weights are the bytes they read; CTA c owns the items whose start byte lies in
-// [c * W_tot / n, (c + 1) * W_tot / n).
+// Items of a row: groups 0..n_g-1, then window chunks of kWinTok tokens.  The
+// host cuts the (row, item) sequence into byte-balanced CTA ranges (item0 in
+// the launch arguments, read from the grid-constant parameter space).
 struct Part {
-  int64_t n_g, W_row, W_tot, rows;
-  int n_items, n_wc, r, rec, tokb, n_cta;
-  double r_cta, r_row, r_tot, r_rec, r_wb, r_items;   // reciprocals (div_floor)
-  __device__ void set_reciprocals() {
-    r_cta = recip(n_cta);
-    r_row = recip(W_row);
-    r_tot = recip(W_tot);
-    r_rec = recip(rec);
-    r_wb = recip((int64_t)kWinTok * tokb);
-    r_items = recip(n_items);
-  }
-  __device__ int64_t row_of(int64_t item) const { return div_floor(item, n_items, r_items); }
-  __device__ int64_t start_in_row(int k) const {
-    return k < n_g ? (int64_t)k * rec : n_g * rec + (int64_t)(k - n_g) * kWinTok * tokb;
-  }
-  __device__ int64_t lo(int c) const { return div_floor((int64_t)c * W_tot, n_cta, r_cta); }
-  // first global item whose start byte is >= x
-  __device__ int64_t first_item(int64_t x) const {
-    const int64_t row = div_floor(x, W_row, r_row);
-    if (row >= rows) return rows * n_items;
-    const int64_t off = x - row * W_row;
-    int64_t k;
-    if (off <= n_g * rec) {
-      k = div_floor(off + rec - 1, rec, r_rec);
-    } else {
-      const int64_t wb = (int64_t)kWinTok * tokb;
-      k = n_g + div_floor(off - n_g * rec + wb - 1, wb, r_wb);
+  int n_g, n_items, n_cta;
+  const int32_t* item0;   // [n_cta + 1]
+  __device__ int row_of(int item) const { return item / n_items; }
+  // CTA owning an item: the largest c with item0[c] <= item
+  __device__ int cta_of(int item) const {
+    int lo = 0, hi = n_cta - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (item0[mid] <= item) lo = mid;
+      else hi = mid - 1;
     }
-    return row * n_items + k;   // k == n_items rolls into the next row's item 0
-  }
-  __device__ int cta_of(int64_t item) const {
-    const int64_t row = row_of(item);
-    const int64_t st = row * W_row + start_in_row((int)(item - row * n_items));
-    int c = (int)div_floor(st * n_cta, W_tot, r_tot);
-    if (c > n_cta - 1) c = n_cta - 1;
-    while (c + 1 < n_cta && lo(c + 1) <= st) ++c;
-    while (c > 0 && lo(c) > st) --c;
-    return c;
+    return lo;
   }
 };
 
@@ -141,20 +115,20 @@ struct Part {
 // (count = 1, first = chunk index); calls seg(row, begin) at each segment start
 // and seg_end(row) at its end.
 template <int SG, class FC, class FS, class FE>
-__device__ __forceinline__ void for_each_chunk(const Part& P, int64_t i0, int64_t i1, FC f, FS seg, FE seg_end) {
+__device__ __forceinline__ void for_each_chunk(const Part& P, int i0, int i1, FC f, FS seg, FE seg_end) {
   int s = 0;
   if (i0 >= i1) return;
-  for (int64_t row = P.row_of(i0); row * P.n_items < i1; ++row) {
-    const int64_t a = max(i0, row * P.n_items) - row * P.n_items;
-    const int64_t b = min(i1, (row + 1) * P.n_items) - row * P.n_items;
+  for (int row = P.row_of(i0); row * P.n_items < i1; ++row) {
+    const int a = max(i0, row * P.n_items) - row * P.n_items;
+    const int b = min(i1, (row + 1) * P.n_items) - row * P.n_items;
     if (a >= b) continue;
-    seg((int)row);
-    for (int64_t k = a; k < min(b, P.n_g); k += SG) {
-      const int cnt = (int)min((int64_t)SG, min(b, P.n_g) - k);
-      f(s++, (int)row, false, k, cnt);
+    seg(row);
+    for (int k = a; k < min(b, P.n_g); k += SG) {
+      const int cnt = min(SG, min(b, P.n_g) - k);
+      f(s++, row, false, (int64_t)k, cnt);
     }
-    for (int64_t k = max(a, P.n_g); k < b; ++k) f(s++, (int)row, true, k - P.n_g, 1);
-    seg_end((int)row);
+    for (int k = max(a, P.n_g); k < b; ++k) f(s++, row, true, (int64_t)(k - P.n_g), 1);
+    seg_end(row);
   }
 }
 
@@ -163,7 +137,7 @@ __device__ __forceinline__ void for_each_chunk(const Part& P, int64_t i0, int64_
 // 512 (384) threads caps them at 128 (168) registers, so that the four (three)
 // warps one SM sub-partition holds fit its 16,384-entry register file.
 template <int BITS, int D, int G, bool TR>
-__global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __grid_constant__ AttnArgs a) {
   using C = K<BITS, D, G, TR>;
   constexpr int P = D * BITS / 32;
   constexpr int J = BITS == 2 ? 4 : 2;
@@ -182,6 +156,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
   uint64_t* bar_qempty = bar_qfull + 2;        // [2]
   uint64_t* bar_sfull = bar_qempty + 2;        // [2] warp states of a segment written
   uint64_t* bar_sfree = bar_sfull + 2;         // [2] merge warp done with a state buffer
+  uint64_t* bar_merge = bar_sfree + 2;         // [1] partials of the final row merge copied in
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
 
   const Geom& gm = a.geom;
@@ -200,6 +175,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
       mbar_init(&bar_sfull[i], C::NC);
       mbar_init(&bar_sfree[i], 1);
     }
+    mbar_init(bar_merge, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
@@ -207,22 +183,15 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
   __syncthreads();
 
   Part Pt;
-  Pt.n_g = a.n_groups;
-  Pt.r = a.r;
-  Pt.n_wc = (a.r + kWinTok - 1) / kWinTok;
-  Pt.n_items = (int)(Pt.n_g + Pt.n_wc);
-  Pt.rec = C::REC;
-  Pt.tokb = 4 * D;
-  Pt.W_row = Pt.n_g * C::REC + (int64_t)a.r * 4 * D;
-  Pt.rows = (int64_t)gm.B * gm.Hkv;
-  Pt.W_tot = Pt.rows * Pt.W_row;
-  Pt.n_cta = gridDim.x;
-  Pt.set_reciprocals();
+  Pt.n_g = (int)a.n_groups;
+  Pt.n_items = a.n_items;
+  Pt.n_cta = a.n_cta;
+  Pt.item0 = a.item0;
   const int cta = blockIdx.x;
-  const int64_t i0 = Pt.first_item(Pt.lo(cta));
-  const int64_t i1 = Pt.first_item(Pt.lo(cta + 1));
+  const int i0 = a.item0[cta];
+  const int i1 = a.item0[cta + 1];
   auto nop_seg = [](int) {};
-  const int64_t last_row = i1 > i0 ? Pt.row_of(i1 - 1) : -1;
+  const int last_row = i1 > i0 ? Pt.row_of(i1 - 1) : -1;
 
   // Merges the warp states of one segment (state buffer sb) and writes the
   // row's output when this CTA covers the whole row, else the CTA's partial
@@ -231,7 +200,11 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
   // threads running it together; sync(): their barrier.  A thread handles four
   // channels of one head at a time and derives that head's merge factors
   // itself, so only the publication of a partial needs barriers.
-  auto merge_segment = [&](int row, float* sb, int tid, int nth, auto sync) {
+  // c_first, np: the first CTA of the row and the number of CTAs with a partial
+  // of it.  The consumer warps (nth > 32) merge the CTA's last segment after
+  // the loop, when the stage ring is idle: their row merge copies the partials
+  // there with bulk copies instead of loading them (one round trip per chunk).
+  auto merge_segment = [&](int row, float* sb, int tid, int nth, auto sync, int c_first, int np) {
     constexpr int NC = C::NC, HS = C::HS, DP = C::DP;
     const float* s_m = sb;
     const float* s_l = sb + NC * HS;
@@ -239,9 +212,6 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
     const float* s_o = sb + C::SO;
     const int g = gm.g;
     const int b = row / gm.Hkv, hkv = row - b * gm.Hkv;
-    const int64_t first_it = (int64_t)row * Pt.n_items;
-    const int c_first = Pt.cta_of(first_it), c_last = Pt.cta_of(first_it + Pt.n_items - 1);
-    const int np = c_last - c_first + 1;
     float* out_row = a.out + ((int64_t)b * gm.Hq + (int64_t)hkv * g) * D;
     float* part = a.ws + ((int64_t)(cta + row) * g) * DP;
     // warp states -> this CTA's (o, M, L) of the row, four channels per step
@@ -288,10 +258,93 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
     }
     sync();
     if (!*s_last) return;
-    // Last CTA of the row: online log-sum-exp over the np partials, the loads
-    // of up to kMB partials (o, m, l) in flight together.
-    constexpr int kMB = 8;
     const float* ws_row = a.ws + (int64_t)(c_first + row) * g * DP;
+    if (nth > 32) {
+      // Last CTA of the row, consumer warps: the np partials (consecutive
+      // slots) are bulk-copied into the idle stage ring, KP at a time, and
+      // merged from there with an online log-sum-exp.
+      const int PB = g * DP * 4;
+      const int KP = (C::NST * C::STAGE) / PB;
+      const float* buf = reinterpret_cast<const float*>(smem);
+      float M[2], L[2];
+      float4 acc[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        M[i] = -INFINITY;
+        L[i] = 0.f;
+        acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      for (int j0 = 0, k = 0; j0 < np; j0 += KP, ++k) {
+        const int nj = min(KP, np - j0);
+        bool issued = false;
+        if (tid == 0 && !*abort_flag) {
+          // the partials are generic-proxy stores of this and other CTAs, seen
+          // through the acquire above; order them before the async-proxy copy
+          asm volatile("fence.proxy.async.global;\n" ::: "memory");
+          mbar_expect_tx(bar_merge, (uint32_t)(nj * PB));
+          bulk_g2s(smem, ws_row + (int64_t)j0 * g * DP, (uint32_t)(nj * PB), bar_merge);
+          issued = true;
+        }
+        const bool ok = !*abort_flag && mbar_wait(bar_merge, k & 1, abort_flag);
+        if (!ok && !*abort_flag) {
+          atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
+          *abort_flag = 1;
+        }
+        if (issued && !ok) {
+          // let the copy land before the CTA can exit (bounded)
+          const long long t0 = clock64();
+          while (!mbar_try_wait(bar_merge, k & 1) && clock64() - t0 < kWaitCycles) {
+          }
+        }
+        if (ok) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int e4 = tid + i * nth;
+            if (e4 < g * D / 4) {
+              const int h = e4 / (D / 4), c = 4 * (e4 - h * (D / 4));
+              float Mb = M[i];
+              for (int u = 0; u < nj; ++u) Mb = fmaxf(Mb, buf[(u * g + h) * DP + D]);
+              const float r = M[i] == -INFINITY ? 0.f : exp2f(M[i] - Mb);
+              L[i] *= r;
+              acc[i].x *= r;
+              acc[i].y *= r;
+              acc[i].z *= r;
+              acc[i].w *= r;
+              for (int u = 0; u < nj; ++u) {
+                const float* pu = buf + (u * g + h) * DP;
+                const float mu = pu[D];
+                const float f = mu == -INFINITY ? 0.f : exp2f(mu - Mb);
+                const float4 v = *reinterpret_cast<const float4*>(pu + c);
+                L[i] = fmaf(pu[D + 1], f, L[i]);
+                acc[i].x = fmaf(v.x, f, acc[i].x);
+                acc[i].y = fmaf(v.y, f, acc[i].y);
+                acc[i].z = fmaf(v.z, f, acc[i].z);
+                acc[i].w = fmaf(v.w, f, acc[i].w);
+              }
+              M[i] = Mb;
+            }
+          }
+        }
+        sync();   // every thread is done with the chunk before the next copy
+      }
+      if (!*abort_flag) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int e4 = tid + i * nth;
+          if (e4 < g * D / 4) {
+            const int h = e4 / (D / 4), c = 4 * (e4 - h * (D / 4));
+            const float r = 1.f / L[i];
+            *reinterpret_cast<float4*>(out_row + h * D + c) =
+                make_float4(acc[i].x * r, acc[i].y * r, acc[i].z * r, acc[i].w * r);
+          }
+        }
+      }
+      if (tid == 0) a.counters[row] = 0u;
+      return;
+    }
+    // Last CTA of the row, merge warp: online log-sum-exp over the np partials,
+    // the loads of up to kMB partials (o, m, l) in flight together.
+    constexpr int kMB = 8;
     for (int e4 = tid; e4 < g * D / 4; e4 += nth) {
       const int h = e4 / (D / 4), c = 4 * (e4 - h * (D / 4));
       const float* col = ws_row + (int64_t)h * DP;
@@ -353,7 +406,10 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
             if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
             *abort_flag = 1;
           } else {
-            merge_segment(row, sm_state + sbi * C::SBUF_F, lane, 32, [] { __syncwarp(); });
+            const int first_it = row * Pt.n_items;
+            const int c_first = Pt.cta_of(first_it);
+            merge_segment(row, sm_state + sbi * C::SBUF_F, lane, 32, [] { __syncwarp(); }, c_first,
+                          Pt.cta_of(first_it + Pt.n_items - 1) - c_first + 1);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar_sfree[sbi]);
@@ -1019,10 +1075,18 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(AttnArgs
     }
   };
 
+  // the CTA range of the last segment's row, computed while the first stage loads
+  int fin_c0 = 0, fin_np = 1;
+  if (last_row >= 0) {
+    const int it = last_row * Pt.n_items;
+    fin_c0 = Pt.cta_of(it);
+    fin_np = Pt.cta_of(it + Pt.n_items - 1) - fin_c0 + 1;
+    asm volatile("" ::"r"(fin_c0), "r"(fin_np));
+  }
   for_each_chunk<C::SG>(Pt, i0, i1, chunk, seg_begin, seg_end);
   if (final_row >= 0) {
     consumer_bar<C::NC>();   // every consumer warp's state of the segment is written
-    merge_segment(final_row, final_sb, threadIdx.x - 96, C::NC * 32, [] { consumer_bar<C::NC>(); });
+    merge_segment(final_row, final_sb, threadIdx.x - 96, C::NC * 32, [] { consumer_bar<C::NC>(); }, fin_c0, fin_np);
   }
 }
 

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -138,23 +139,66 @@ static Geom make_geom(const kvq_cache* h) {
   return g;
 }
 
-// Decode launch size: one CTA per SM at most, and few enough that every CTA's
-// byte range holds at least one whole item (a group record or a window chunk
-// of 32 tokens), so each CTA between a row's first and last contributor has
-// work in that row.
-static int plan_ctas(const kvq_config& c, int64_t n_groups, int r) {
+// The decode work partition.  A row's items are n_q quantized items (KIVI
+// groups, TurboQuant token blocks) and then n_w window-type chunks of 32
+// tokens.  The kernels take a CTA's quantized items `sg` at a time from the
+// start of its range, one stage per `sg` items, and one stage per window
+// chunk; a stage takes about the same time whatever its bytes, since the
+// consumer warps' instruction stream, not HBM, sets the pace.  So the
+// partition balances stages, not bytes: a row is a sequence of ceil(n_q / sg)
+// stage chunks of weight ws (each starting at a multiple of sg) and n_w window
+// chunks of weight ww, and CTA c takes the chunks whose start weight lies in
+// [c U / n, (c + 1) U / n), U the total weight.  Fills item0[0 .. n] (the
+// first item of each CTA, then the end); false when a CTA would own no chunk.
+static bool partition_items(int64_t rows, int64_t n_q, int sg, int64_t n_w, int64_t ws, int64_t ww, int n,
+                            int32_t* item0) {
+  const int64_t n_items = n_q + n_w, S = (n_q + sg - 1) / sg;
+  const int64_t U_row = S * ws + n_w * ww, U = rows * U_row;
+  for (int c = 0; c <= n; ++c) {
+    const int64_t x = (int64_t)c * U / n;
+    const int64_t row = x / U_row;
+    int64_t it;
+    if (row >= rows) {
+      it = rows * n_items;
+    } else {
+      const int64_t off = x - row * U_row;
+      const int64_t k = off <= S * ws ? (off + ws - 1) / ws : S + (off - S * ws + ww - 1) / ww;   // first chunk
+      it = row * n_items + (k < S ? k * sg : n_q + (k - S));   // k == S + n_w is the next row's item 0
+    }
+    item0[c] = (int32_t)it;
+    if (c > 0 && item0[c] <= item0[c - 1]) return false;
+  }
+  return true;
+}
+
+// Quantized items one decode stage carries (the kernels' consumer warps take
+// one 32-token block each).
+static int decode_stage_items(const kvq_config& c) {
+  if (c.scheme == KVQ_TURBO) return kTqDecodeConsumers;
+  const int g = c.num_q_heads / c.num_kv_heads;
+  return (g <= 4 ? kKiviConsumersTM : kKiviConsumersHM) / (c.group / kTB);
+}
+
+// Decode launch size and partition: one CTA per SM at most (kMaxDecodeCtas),
+// and few enough that every CTA owns at least one chunk, so each CTA between a
+// row's first and last contributor has work in that row.  Returns the CTA
+// count (0 when the item indices would not fit in 32 bits).
+static int plan_decode(const kvq_config& c, int64_t n_groups, int r, int32_t* n_items, int32_t* item0) {
+  // weights of a stage of quantized items and of a window chunk: a window
+  // chunk's stage takes about 1.5 times a full stage of groups (measured)
+  constexpr int64_t kWs = 2, kWw = 3;
   const int64_t rows = (int64_t)c.batch * c.num_kv_heads;
-  const int64_t rec = c.scheme == KVQ_TURBO ? (int64_t)kTqTbBytes
-                                             : (int64_t)c.group * c.head_dim * c.bits / 4 + 4 * c.head_dim + 4 * c.group;
-  const int64_t tokb = c.fp8_recent ? 2 * (int64_t)kFp8RowBytes : 4 * (int64_t)c.head_dim;
-  r += c.anchor_tokens;   // anchors weigh like window tokens
-  const int64_t w_tot = rows * (n_groups * rec + (int64_t)r * tokb);
-  const int64_t w_max = r > 0 ? (rec > 32 * tokb ? rec : 32 * tokb) : rec;
-  int64_t n = w_tot / w_max;
+  const int A = c.scheme == KVQ_TURBO ? c.anchor_tokens : 0;
+  const int64_t n_w = (r + kDecodeWinTok - 1) / kDecodeWinTok + A / kDecodeWinTok;
+  const int sg = decode_stage_items(c);
+  if (rows * (n_groups + n_w) >= ((int64_t)1 << 31)) return 0;
+  *n_items = (int32_t)(n_groups + n_w);
+  const int64_t U = rows * (((n_groups + sg - 1) / sg) * kWs + n_w * kWw);
   const int64_t sms = num_sms() < kMaxDecodeCtas ? num_sms() : kMaxDecodeCtas;
-  if (n > sms) n = sms;
-  if (n < 1) n = 1;
-  return (int)n;
+  int n = (int)std::max<int64_t>(1, std::min<int64_t>(sms, U / kWw));
+  while (n > 1 && !partition_items(rows, n_groups, sg, n_w, kWs, kWw, n, item0)) --n;
+  if (n == 1) partition_items(rows, n_groups, sg, n_w, kWs, kWw, 1, item0);
+  return n;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -374,7 +418,8 @@ static kvq_status launch_attention(const kvq_cache* h, int r, const void* q, flo
   a.counters = reinterpret_cast<unsigned*>(h->base + h->lay.status_offset) + 1;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.n_groups = h->tq / c.group;
-  a.n_cta = plan_ctas(c, a.n_groups, r);
+  a.n_cta = plan_decode(c, a.n_groups, r, &a.n_items, a.item0);
+  if (a.n_cta <= 0) return KVQ_ERR_UNSUPPORTED;
   a.r = r;
   a.head = h->head;
   a.k_new = static_cast<const uint16_t*>(k_new);
@@ -474,7 +519,8 @@ const char* kvq_cuda_error_string(void) { return g_cuda_error; }
 
 int32_t kvq_decode_splits(const kvq_cache* h) {
   if (!h) return -1;
-  return plan_ctas(h->cfg, h->tq / h->cfg.group, h->r);
+  int32_t n_items, item0[kMaxDecodeCtas + 1];
+  return plan_decode(h->cfg, h->tq / h->cfg.group, h->r, &n_items, item0);
 }
 
 }  // extern "C"

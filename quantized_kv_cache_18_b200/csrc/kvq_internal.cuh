@@ -38,6 +38,10 @@ namespace kvq {
 constexpr int kTB = 32;         // tokens per token block
 constexpr int kFp8RowBytes = 144;   // FP8 token row: 128 E4M3 codes, fp16 scale, 14 zero bytes (d = 128)
 constexpr int kMaxDecodeCtas = 160;   // decode launches use at most this many CTAs (one per SM)
+constexpr int kDecodeWinTok = 32;     // window tokens per decode work item
+constexpr int kKiviConsumersTM = 12;  // KIVI decode consumer warps, token-major formulation (GQA groups <= 4)
+constexpr int kKiviConsumersHM = 8;   // KIVI decode consumer warps, head-major formulation
+constexpr int kTqDecodeConsumers = 8; // TurboQuant decode consumer warps
 
 struct Geom {
   int scheme, d, bits, G, R, cap, B, Hkv, Hq, g, dtype;
@@ -241,6 +245,11 @@ struct AttnArgs {
   // that attends it also stores it into ring slot (head + r - 1) % cap.
   const uint16_t* k_new;
   const uint16_t* v_new;
+  // Work partition, computed on the host: CTA c owns the global items
+  // item0[c] .. item0[c + 1] - 1 (strictly increasing), where a row's items
+  // are its n_groups quantized items, then its window-type chunks.
+  int32_t n_items;                        // items per row
+  int32_t item0[kMaxDecodeCtas + 1];
 };
 
 void launch_kivi_quantize(const QuantArgs& a, cudaStream_t st);

@@ -35,9 +35,9 @@ namespace kvq {
 
 namespace {
 
-constexpr int kTqConsumers = 8;
+constexpr int kTqConsumers = kTqDecodeConsumers;
 constexpr int kTqThreads = (kTqConsumers + 1) * 32;
-constexpr int kTqWin = 32;
+constexpr int kTqWin = kDecodeWinTok;
 
 struct TL {
   static constexpr int D = kTqD;
@@ -89,47 +89,22 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t w) {
   return r;   // ((w << (15 - Q)) & 0x80008000) ^ 0xBC00BC00: bit 1 -> +1.0, bit 0 -> -1.0
 }
 
-// Work partition: items of a row are n_tb token blocks then n_wc window chunks,
-// weighted by the bytes they read; CTA c owns the items whose start byte lies
-// in [c W_tot / n, (c + 1) W_tot / n).
+// Work partition: items of a row are n_tb token blocks then n_wc window-type
+// chunks; the host cuts the (row, item) sequence into byte-balanced CTA ranges
+// (item0 in the launch arguments, read from the grid-constant parameter space).
 struct TPart {
-  int64_t n_tb, W_row, W_tot, rows;
-  int n_items, n_wc, r, tokb, n_cta;
-  double r_cta, r_row, r_tot, r_tb, r_wb, r_items;   // reciprocals (div_floor)
-  __device__ void set_reciprocals() {
-    r_cta = recip(n_cta);
-    r_row = recip(W_row);
-    r_tot = recip(W_tot);
-    r_tb = recip(kTqTbBytes);
-    r_wb = recip((int64_t)kTqWin * tokb);
-    r_items = recip(n_items);
-  }
-  __device__ int64_t row_of(int64_t item) const { return div_floor(item, n_items, r_items); }
-  __device__ int64_t start_in_row(int k) const {
-    return k < n_tb ? (int64_t)k * kTqTbBytes : n_tb * kTqTbBytes + (int64_t)(k - n_tb) * kTqWin * tokb;
-  }
-  __device__ int64_t lo(int c) const { return div_floor((int64_t)c * W_tot, n_cta, r_cta); }
-  __device__ int64_t first_item(int64_t x) const {
-    const int64_t row = div_floor(x, W_row, r_row);
-    if (row >= rows) return rows * n_items;
-    const int64_t off = x - row * W_row;
-    int64_t k;
-    if (off <= n_tb * kTqTbBytes) {
-      k = div_floor(off + kTqTbBytes - 1, kTqTbBytes, r_tb);
-    } else {
-      const int64_t wb = (int64_t)kTqWin * tokb;
-      k = n_tb + div_floor(off - n_tb * kTqTbBytes + wb - 1, wb, r_wb);
+  int n_tb, n_items, n_wc, n_cta;
+  const int32_t* item0;   // [n_cta + 1]
+  __device__ int row_of(int item) const { return item / n_items; }
+  // CTA owning an item: the largest c with item0[c] <= item
+  __device__ int cta_of(int item) const {
+    int lo = 0, hi = n_cta - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (item0[mid] <= item) lo = mid;
+      else hi = mid - 1;
     }
-    return row * n_items + k;
-  }
-  __device__ int cta_of(int64_t item) const {
-    const int64_t row = row_of(item);
-    const int64_t st = row * W_row + start_in_row((int)(item - row * n_items));
-    int c = (int)div_floor(st * n_cta, W_tot, r_tot);
-    if (c > n_cta - 1) c = n_cta - 1;
-    while (c + 1 < n_cta && lo(c + 1) <= st) ++c;
-    while (c > 0 && lo(c) > st) --c;
-    return c;
+    return lo;
   }
 };
 
@@ -137,30 +112,30 @@ struct TPart {
 // seg_end(row, part) after the token blocks (part 0) and the window chunks
 // (part 1) a CTA owns in a row.
 template <class FC, class FS, class FE>
-__device__ __forceinline__ void tq_for_each_chunk(const TPart& P, int64_t i0, int64_t i1, FC f, FS seg, FE seg_end) {
+__device__ __forceinline__ void tq_for_each_chunk(const TPart& P, int i0, int i1, FC f, FS seg, FE seg_end) {
   int s = 0;
   if (i0 >= i1) return;
-  for (int64_t row = P.row_of(i0); row * P.n_items < i1; ++row) {
-    const int64_t a = max(i0, row * P.n_items) - row * P.n_items;
-    const int64_t b = min(i1, (row + 1) * P.n_items) - row * P.n_items;
+  for (int row = P.row_of(i0); row * P.n_items < i1; ++row) {
+    const int a = max(i0, row * P.n_items) - row * P.n_items;
+    const int b = min(i1, (row + 1) * P.n_items) - row * P.n_items;
     if (a >= b) continue;
     if (a < P.n_tb) {
-      seg((int)row, 0);
-      for (int64_t k = a; k < min(b, P.n_tb); k += TL::SG) {
-        const int cnt = (int)min((int64_t)TL::SG, min(b, P.n_tb) - k);
-        f(s++, (int)row, false, k, cnt);
+      seg(row, 0);
+      for (int k = a; k < min(b, P.n_tb); k += TL::SG) {
+        const int cnt = min(TL::SG, min(b, P.n_tb) - k);
+        f(s++, row, false, (int64_t)k, cnt);
       }
-      seg_end((int)row, 0);
+      seg_end(row, 0);
     }
     if (b > P.n_tb) {
-      seg((int)row, 1);
-      for (int64_t k = max(a, P.n_tb); k < b; ++k) f(s++, (int)row, true, k - P.n_tb, 1);
-      seg_end((int)row, 1);
+      seg(row, 1);
+      for (int k = max(a, P.n_tb); k < b; ++k) f(s++, row, true, (int64_t)(k - P.n_tb), 1);
+      seg_end(row, 1);
     }
   }
 }
 
-__global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_constant__ AttnArgs a) {
   using C = TL;
   constexpr int D = C::D, NKT = C::NKT, NNT = C::NNT;
 
@@ -202,21 +177,16 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
   __syncthreads();
 
   TPart Pt;
-  Pt.n_tb = a.n_groups;
-  Pt.r = a.r;
+  Pt.n_tb = (int)a.n_groups;
   // window-type items: the window's chunks, then (mixed cache) the anchors' chunks
-  const int n_wcw = (a.r + kTqWin - 1) / kTqWin;
-  Pt.n_wc = n_wcw + gm.anchor / kTqWin;
-  Pt.n_items = (int)(Pt.n_tb + Pt.n_wc);
-  Pt.tokb = gm.fp8 ? 2 * kFp8RowBytes : 4 * D;
-  Pt.W_row = Pt.n_tb * kTqTbBytes + (int64_t)(a.r + gm.anchor) * Pt.tokb;
-  Pt.rows = (int64_t)gm.B * gm.Hkv;
-  Pt.W_tot = Pt.rows * Pt.W_row;
-  Pt.n_cta = gridDim.x;
-  Pt.set_reciprocals();
+  Pt.n_items = a.n_items;
+  Pt.n_wc = a.n_items - Pt.n_tb;
+  Pt.n_cta = a.n_cta;
+  Pt.item0 = a.item0;
+  const int n_wcw = (a.r + kTqWin - 1) / kTqWin;   // window chunks (the anchors' chunks follow)
   const int cta = blockIdx.x;
-  const int64_t i0 = Pt.first_item(Pt.lo(cta));
-  const int64_t i1 = Pt.first_item(Pt.lo(cta + 1));
+  const int i0 = a.item0[cta];
+  const int i1 = a.item0[cta + 1];
   auto nop_seg = [](int, int) {};
 
   if (warp == 0) {
@@ -520,7 +490,6 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
       // scales multiply the scores and p in fp32.  q goes to fp16 for the mma.
       const uint16_t* qraw = reinterpret_cast<const uint16_t*>(sq + kTqQPrepBytes);
       const int j = (int)first;
-      const int n_wcw = (a.r + kTqWin - 1) / kTqWin;
       const int n_tok = j < n_wcw ? min(kTqWin, a.r - j * kTqWin) : kTqWin;
       const int t0 = 4 * cw;
       const unsigned char* kb8 = st;
@@ -725,7 +694,7 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(AttnArgs a) {
       fin = y;
     }
     const int b = row / gm.Hkv, hkv = row - b * gm.Hkv;
-    const int64_t it0 = (int64_t)row * Pt.n_items;
+    const int it0 = row * Pt.n_items;
     const int np0 = Pt.n_tb > 0 ? Pt.cta_of(it0 + Pt.n_tb - 1) - Pt.cta_of(it0) + 1 : 0;
     const int c_f1 = Pt.n_wc > 0 ? Pt.cta_of(it0 + Pt.n_tb) : 0;
     const int np1 = Pt.n_wc > 0 ? Pt.cta_of(it0 + Pt.n_items - 1) - c_f1 + 1 : 0;
