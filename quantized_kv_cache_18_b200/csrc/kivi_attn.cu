@@ -652,11 +652,11 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
     uint4 kc[P / 4];
 #pragma unroll
     for (int p = 0; p < P / 4; ++p) kc[p] = lds128(rec + tbg * C::TBC + 16 * (32 * p + lane));
-    const float beta = sm_beta[(slot * C::SG + grp) * 8 + tc];
+    const float bs = sm_beta[(slot * C::SG + grp) * 8 + tc] * a.scale_log2;
     const unsigned char* psc = rec + C::KSOFF + 16 * tc;
     // fp16x2 (-1, -1) on lo lanes, (0, 0) on hi lanes: q~ column = fma(q, s, sel * round(q s))
     const uint32_t sel = (gr & 1) ? 0xBC00BC00u : 0u;
-    float sc[2][2][4];   // [k-tile parity][token m-tile]
+    float sc[2][2][4];   // [k-tile parity][token m-tile]: two independent chains per m-tile
 #pragma unroll
     for (int par = 0; par < 2; ++par)
 #pragma unroll
@@ -697,8 +697,8 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
 #pragma unroll
       for (int e2 = 0; e2 < 2; ++e2) {
         const int i = 2 * mt + e2;
-        x[i] = ((sc[0][mt][2 * e2] + sc[1][mt][2 * e2]) + (sc[0][mt][2 * e2 + 1] + sc[1][mt][2 * e2 + 1]) + beta) *
-               a.scale_log2;
+        x[i] = fmaf((sc[0][mt][2 * e2] + sc[1][mt][2 * e2]) + (sc[0][mt][2 * e2 + 1] + sc[1][mt][2 * e2 + 1]),
+                    a.scale_log2, bs);
         mx = fmaxf(mx, x[i]);
       }
     rescale_to(tr_head_max(mx));
@@ -829,6 +829,16 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
       if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
       *abort_flag = 1;
     }
+    if (s == 0 && cw >= 4) {
+      // The consumer warps of one SM sub-partition (cw, cw + 4, cw + 8) start
+      // a fraction of a block apart, so that one's softmax overlaps another's
+      // mma's instead of all of them alternating in step (the stage waits
+      // never resynchronise them: the ring runs ahead of the consumers).
+      const long long t0 = clock64();
+      const long long d = (cw >> 2) * (TR ? 800 : 1300);
+      while (clock64() - t0 < d) {
+      }
+    }
     const unsigned char* st = smem + slot * C::STAGE;
     if (ok && win && a.k_new != nullptr && cw == C::NC - 1) {
       // fused append: the new token of this row (the chunk's last) into its ring slot
@@ -854,14 +864,12 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
       uint4 kc[P / 4];
 #pragma unroll
       for (int p = 0; p < P / 4; ++p) kc[p] = lds128(rec + tbg * C::TBC + 16 * (32 * p + lane));
-      const float beta = sm_beta[(slot * C::SG + grp) * 8 + gr];
+      const float bs = sm_beta[(slot * C::SG + grp) * 8 + gr] * a.scale_log2;
       // this lane's key scales: 16 bytes per k-tile pair kt2 at 64 kt2 + 16 tc
       const unsigned char* psc = rec + C::KSOFF + 16 * tc;
-      float sc[2][4][4];   // [k-tile parity][n-tile]: two independent chains per n-tile
+      float sc[4][4];   // [n-tile]
 #pragma unroll
-      for (int par = 0; par < 2; ++par)
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) sc[par][nt][0] = sc[par][nt][1] = sc[par][nt][2] = sc[par][nt][3] = 0.f;
+      for (int nt = 0; nt < 4; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
       for (int wi = 0; wi < WPN; ++wi)
 #pragma unroll
@@ -883,7 +891,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
             const uint32_t aq[4] = {h2_as_u32(hi0), h2_as_u32(__hfma2(u32_as_h2(qh[kt][0]), u32_as_h2(s2.x), __hneg2(hi0))),
                                     h2_as_u32(hi1), h2_as_u32(__hfma2(u32_as_h2(qh[kt][1]), u32_as_h2(s2.y), __hneg2(hi1)))};
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) mma_f16_16816(sc[kt & 1][nt], aq, pr[nt][2 * m2], pr[nt][2 * m2 + 1]);
+            for (int nt = 0; nt < 4; ++nt) mma_f16_16816(sc[nt], aq, pr[nt][2 * m2], pr[nt][2 * m2 + 1]);
           }
         }
       float x[4][2];
@@ -892,7 +900,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          x[nt][e] = ((sc[0][nt][e] + sc[1][nt][e]) + (sc[0][nt][2 + e] + sc[1][nt][2 + e]) + beta) * a.scale_log2;
+          x[nt][e] = fmaf(sc[nt][e] + sc[nt][2 + e], a.scale_log2, bs);
           mt = fmaxf(mt, x[nt][e]);
         }
       rescale_to(quad_max(mt));
