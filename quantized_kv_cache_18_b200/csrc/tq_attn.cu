@@ -308,6 +308,11 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
   const int cw = warp - 1;
   const int ct = threadIdx.x - 32;
   const bool head_ok = gr < gm.g;
+  // GQA groups of up to 4 heads run the token blocks in the token-major
+  // formulation (codes as the A operand, the heads' hi | lo parts as the 8
+  // columns of B): half the mma's of the head-major form, whose 8 hi | lo rows
+  // such a group only half fills.  Window chunks stay head-major.
+  const bool tr = gm.g <= 4;
   {
     // per-lane copy of the pair table: entry idx of lane L at [idx][L]
     const uint32_t* lut_g = reinterpret_cast<const uint32_t*>(gm.params + kTqLut);
@@ -340,6 +345,25 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
         qa[kt][1] = v.y;
         qa[kt][2] = v.z;
         qa[kt][3] = v.w;
+      }
+      if (tr) {
+        // token-major: B operands, column n = head n >> 1, part n & 1 (hi | lo),
+        // taken from the A fragments (rows = heads hi | lo) of lane (n >> 1, tc):
+        // qa[kt][0..1] = Pi q, qa[kt][2..3] = S Pi q
+        const int src = (gr >> 1) * 4 + tc;
+        const bool lo = (gr & 1) != 0;
+#pragma unroll
+        for (int kt = 0; kt < NKT; ++kt) {
+          const uint4 w = ok ? lds128(sq + ((NKT + kt) * 32 + lane) * 16) : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t s0 = __shfl_sync(0xffffffffu, qa[kt][0], src), s1 = __shfl_sync(0xffffffffu, qa[kt][1], src);
+          const uint32_t s2 = __shfl_sync(0xffffffffu, qa[kt][2], src), s3 = __shfl_sync(0xffffffffu, qa[kt][3], src);
+          const uint32_t t0 = __shfl_sync(0xffffffffu, w.x, src), t1 = __shfl_sync(0xffffffffu, w.y, src);
+          const uint32_t t2 = __shfl_sync(0xffffffffu, w.z, src), t3 = __shfl_sync(0xffffffffu, w.w, src);
+          qa[kt][0] = lo ? s1 : s0;
+          qa[kt][1] = lo ? s3 : s2;
+          qa[kt][2] = lo ? t1 : t0;
+          qa[kt][3] = lo ? t3 : t2;
+        }
       }
     }
 #pragma unroll
@@ -387,8 +411,120 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
         }
       }
     }
-    if (ok && !win && cw < cnt) {
-      // ---------------------------------------------------------- one token block
+    if (ok && !win && cw < cnt && tr) {
+      // ---------------------------------------------------------- one token block, token-major
+      // A fragment of token m-tile MT = the B fragments of token n-tiles 2MT,
+      // 2MT + 1 of the packed format; lane (gr, tc) gets the scores of head tc,
+      // tokens gr + 8i, and the output of head tc, channels 16MT + gr (+8).
+      const unsigned char* tb = st + cw * kTqTbBytes;
+      float sc[2][4], ss[2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[mt][e] = ss[mt][e] = 0.f;
+      {
+        uint32_t kw[13];
+        const uint4 w0 = lds128(tb + kTqKCodes + 16 * lane), w1 = lds128(tb + kTqKCodes + 512 + 16 * lane),
+                    w2 = lds128(tb + kTqKCodes + 1024 + 16 * lane);
+        kw[0] = w0.x; kw[1] = w0.y; kw[2] = w0.z; kw[3] = w0.w;
+        kw[4] = w1.x; kw[5] = w1.y; kw[6] = w1.z; kw[7] = w1.w;
+        kw[8] = w2.x; kw[9] = w2.y; kw[10] = w2.z; kw[11] = w2.w;
+        kw[12] = *reinterpret_cast<const uint32_t*>(tb + kTqKCodes + 1536 + 4 * lane);
+        // <Pi q, c_hat>: key pair slot 16 nt + 2 kt + rho of token n-tile nt
+#define TQ_TR_KEY(KT)                                                                                \
+  {                                                                                                  \
+    const uint32_t a0[4] = {lut_pair<2 * KT>(kw, lut_lane), lut_pair<16 + 2 * KT>(kw, lut_lane),     \
+                            lut_pair<1 + 2 * KT>(kw, lut_lane), lut_pair<17 + 2 * KT>(kw, lut_lane)}; \
+    mma_f16_16816(sc[0], a0, qa[KT][0], qa[KT][1]);                                                  \
+    const uint32_t a1[4] = {lut_pair<32 + 2 * KT>(kw, lut_lane), lut_pair<48 + 2 * KT>(kw, lut_lane), \
+                            lut_pair<33 + 2 * KT>(kw, lut_lane), lut_pair<49 + 2 * KT>(kw, lut_lane)}; \
+    mma_f16_16816(sc[1], a1, qa[KT][0], qa[KT][1]);                                                  \
+  }
+        TQ_TR_KEY(0) TQ_TR_KEY(1) TQ_TR_KEY(2) TQ_TR_KEY(3) TQ_TR_KEY(4) TQ_TR_KEY(5) TQ_TR_KEY(6) TQ_TR_KEY(7)
+#undef TQ_TR_KEY
+      }
+      {
+        // <S Pi q, sign>: sign word nt of the lane, bits 2 kt + rho and 16 + 2 kt + rho
+        const uint4 swv = lds128(tb + kTqSigns + 16 * lane);
+        const uint32_t sw[4] = {swv.x, swv.y, swv.z, swv.w};
+#define TQ_TR_SGN(KT)                                                                                 \
+  {                                                                                                   \
+    const uint32_t a0[4] = {sign_pair<2 * KT>(sw[0]), sign_pair<2 * KT>(sw[1]), sign_pair<2 * KT + 1>(sw[0]), \
+                            sign_pair<2 * KT + 1>(sw[1])};                                            \
+    mma_f16_16816(ss[0], a0, qa[KT][2], qa[KT][3]);                                                   \
+    const uint32_t a1[4] = {sign_pair<2 * KT>(sw[2]), sign_pair<2 * KT>(sw[3]), sign_pair<2 * KT + 1>(sw[2]), \
+                            sign_pair<2 * KT + 1>(sw[3])};                                            \
+    mma_f16_16816(ss[1], a1, qa[KT][2], qa[KT][3]);                                                   \
+  }
+        TQ_TR_SGN(0) TQ_TR_SGN(1) TQ_TR_SGN(2) TQ_TR_SGN(3) TQ_TR_SGN(4) TQ_TR_SGN(5) TQ_TR_SGN(6) TQ_TR_SGN(7)
+#undef TQ_TR_SGN
+      }
+      // meta of token gr + 8i: entry 8 (gr >> 1) + 2i + (gr & 1) (key: n, gamma; value: n)
+      const int e0 = 8 * (gr >> 1) + (gr & 1);
+      const uint32_t* kmw = reinterpret_cast<const uint32_t*>(tb + kTqKMeta);
+      const uint16_t* vnw = reinterpret_cast<const uint16_t*>(tb + kTqVMeta);
+      float x[4];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int mt = i >> 1, e2 = i & 1;
+        const float2 ng = __half22float2(u32_as_h2(kmw[e0 + 2 * i]));
+        const float main = sc[mt][2 * e2] + sc[mt][2 * e2 + 1];
+        const float corr = ss[mt][2 * e2] + ss[mt][2 * e2 + 1];
+        x[i] = fmaf(ng.x, main, ng.y * a.qjl_c * corr) * a.scale_log2;
+        mx = fmaxf(mx, x[i]);
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      rescale_to(mx);
+      uint32_t pp[4];   // (hi, lo) of p~ = p n_v, head tc, token gr + 8i
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float p = fast_exp2(x[i] - m);
+        l += p;
+        const float pt = p * __half2float(__ushort_as_half(vnw[e0 + 2 * i]));
+        const __half hi = __float2half_rn(pt);
+        const __half lo = __float2half_rn(pt - __half2float(hi));
+        pp[i] = h2_as_u32(__halves2half2(hi, lo));
+      }
+      // B fragments of P.V (k = tokens 16 kt + 2 tc (+1, +8, +9), column gr =
+      // head gr >> 1, hi | lo) from the lanes holding those tokens
+      const int la = 8 * tc + (gr >> 1), lb = la + 4;
+      const uint32_t psel = (gr & 1) ? 0x7632u : 0x5410u;
+      uint32_t bp[2][2];
+#pragma unroll
+      for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t xa = __shfl_sync(0xffffffffu, pp[2 * kt + h], la);
+          const uint32_t xb = __shfl_sync(0xffffffffu, pp[2 * kt + h], lb);
+          bp[kt][h] = __byte_perm(xa, xb, psel);
+        }
+      {
+        uint32_t vw[13];
+        const uint4 w0 = lds128(tb + kTqVCodes + 16 * lane), w1 = lds128(tb + kTqVCodes + 512 + 16 * lane),
+                    w2 = lds128(tb + kTqVCodes + 1024 + 16 * lane);
+        vw[0] = w0.x; vw[1] = w0.y; vw[2] = w0.z; vw[3] = w0.w;
+        vw[4] = w1.x; vw[5] = w1.y; vw[6] = w1.z; vw[7] = w1.w;
+        vw[8] = w2.x; vw[9] = w2.y; vw[10] = w2.z; vw[11] = w2.w;
+        vw[12] = *reinterpret_cast<const uint32_t*>(tb + kTqVCodes + 1536 + 4 * lane);
+        // value pair slot 32 kt + 2 nt + rho of channel n-tile nt; A of channel
+        // m-tile MT = n-tiles 2MT, 2MT + 1
+#define TQ_TR_PV(KT, MT)                                                                                      \
+  {                                                                                                           \
+    const uint32_t av[4] = {lut_pair<32 * KT + 4 * MT>(vw, lut_lane), lut_pair<32 * KT + 4 * MT + 2>(vw, lut_lane), \
+                            lut_pair<32 * KT + 4 * MT + 1>(vw, lut_lane), lut_pair<32 * KT + 4 * MT + 3>(vw, lut_lane)}; \
+    mma_f16_16816(o[MT], av, bp[KT][0], bp[KT][1]);                                                          \
+  }
+#define TQ_TR_PV_KT(KT) \
+  TQ_TR_PV(KT, 0) TQ_TR_PV(KT, 1) TQ_TR_PV(KT, 2) TQ_TR_PV(KT, 3) TQ_TR_PV(KT, 4) TQ_TR_PV(KT, 5) TQ_TR_PV(KT, 6) TQ_TR_PV(KT, 7)
+        TQ_TR_PV_KT(0) TQ_TR_PV_KT(1)
+#undef TQ_TR_PV_KT
+#undef TQ_TR_PV
+      }
+    } else if (ok && !win && cw < cnt) {
+      // ---------------------------------------------------------- one token block, head-major
       const unsigned char* tb = st + cw * kTqTbBytes;
       float sc[4][4], ss[4][4];
 #pragma unroll
@@ -638,15 +774,32 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
   };
 
   auto seg_end = [&](int row, int part) {
-    const float ls = quad_sum(l);
-    if (tc == 0) {
-      sm_m[cw * 8 + gr] = m;
-      sm_l[cw * 8 + gr] = ls;
+    if (tr && part == 0) {
+      // token-major state: head tc, l summed over the 8 lanes gr
+      float ls = l;
+      ls += __shfl_xor_sync(0xffffffffu, ls, 4);
+      ls += __shfl_xor_sync(0xffffffffu, ls, 8);
+      ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+      if (gr == 0) {
+        sm_m[cw * 8 + tc] = m;
+        sm_l[cw * 8 + tc] = ls;
+      }
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        sm_o[(cw * 8 + tc) * D + 16 * mt + gr] = o[mt][0] + o[mt][1];
+        sm_o[(cw * 8 + tc) * D + 16 * mt + 8 + gr] = o[mt][2] + o[mt][3];
+      }
+    } else {
+      const float ls = quad_sum(l);
+      if (tc == 0) {
+        sm_m[cw * 8 + gr] = m;
+        sm_l[cw * 8 + gr] = ls;
+      }
+#pragma unroll
+      for (int nt = 0; nt < NNT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) sm_o[(cw * 8 + gr) * D + 8 * nt + 2 * tc + e] = o[nt][e] + o[nt][2 + e];
     }
-#pragma unroll
-    for (int nt = 0; nt < NNT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) sm_o[(cw * 8 + gr) * D + 8 * nt + 2 * tc + e] = o[nt][e] + o[nt][2 + e];
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar_qempty[(qseg - 1) & 1]);
     tq_consumer_bar();
