@@ -24,7 +24,8 @@
 //   warps 2..   consumers (8 head-major, 12 token-major): one 32-token block
 //               per warp per stage, online softmax
 // Work: the (row, item) sequence -- a row's groups then its 32-token window
-// chunks -- is cut into equal-byte ranges, one per CTA.  A CTA writes one
+// chunks -- is cut on the host into ranges of equal stage count, one per CTA
+// (a window chunk's stage weighs 1.5 group stages).  A CTA writes one
 // partial (m, l, o) per row it touches; the last CTA to finish a row (atomic
 // counter in the cache buffer, reset after use) merges that row's partials
 // with a log-sum-exp that normalises globally, as Minima-KV merges its partial
