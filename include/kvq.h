@@ -329,6 +329,24 @@ uint64_t kvq_launch_count(void);
 /* Decode-attention split count the library picks for the current state. */
 int32_t kvq_decode_splits(const kvq_cache* cache);
 
+/* The decode work partition for a cache of configuration `cfg` holding
+ * `n_groups` quantized groups (KIVI) or 32-token blocks (TURBO) and `r`
+ * window tokens per row, on a GPU with `sms` multiprocessors.  A row's work
+ * items are its quantized items, then its window chunks of 32 tokens (and, in
+ * the mixed TURBO cache, its anchor chunks); *n_items receives their count.
+ * CTA c of the decode launch owns the global items item0[c] .. item0[c+1]-1
+ * (global item = row x n_items + item); item0[0] = 0, item0[n] = rows x
+ * n_items, strictly increasing.  The ranges balance stages (a stage carries
+ * up to 12, 8, 6 or 4 KIVI groups, by formulation and G, or 8 TURBO blocks;
+ * a window chunk's stage weighs 1.5 of them) and quantized ranges start at a
+ * stage boundary of their row.  Fills item0[0 .. n] (caller-owned, `cap`
+ * entries) and returns n, or 0 for a null pointer, an unsupported
+ * configuration, n_groups < 0, r < 0, sms < 1 or cap < n + 1.  Host only: no
+ * CUDA call.  The decode entry points use this partition with the current
+ * GPU's multiprocessor count. */
+int32_t kvq_decode_partition(const kvq_config* cfg, int64_t n_groups, int32_t r, int32_t sms, int32_t* item0,
+                             int32_t cap, int32_t* n_items);
+
 #ifdef __cplusplus
 }
 #endif

@@ -52,6 +52,7 @@ _SIGS = {
     "kvq_launch_count": (ctypes.c_uint64, []),
     "kvq_cuda_error_string": (ctypes.c_char_p, []),
     "kvq_decode_splits": (ctypes.c_int32, [_P]),
+    "kvq_decode_partition": (ctypes.c_int32, [_P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32, _P]),
 }
 
 _lib = None

@@ -47,6 +47,18 @@ def workspace_bytes(cfg: L.KvqConfig) -> int:
     return int(L.load().kvq_workspace_bytes(ctypes.byref(cfg)))
 
 
+def decode_partition(cfg: L.KvqConfig, n_groups: int, r: int, sms: int):
+    """The decode launch's work partition (kvq_decode_partition): the first
+    global item of each CTA followed by the end, and the items per row.
+    Host only."""
+    buf = (ctypes.c_int32 * 161)()
+    n_items = ctypes.c_int32()
+    n = L.load().kvq_decode_partition(ctypes.byref(cfg), n_groups, r, sms, buf, 161, ctypes.byref(n_items))
+    if n <= 0:
+        raise ValueError("kvq_decode_partition: unsupported arguments")
+    return list(buf[:n + 1]), int(n_items.value)
+
+
 def layout(cfg: L.KvqConfig) -> L.KvqLayout:
     out = L.KvqLayout()
     L.check(L.load().kvq_get_layout(ctypes.byref(cfg), ctypes.byref(out)), "kvq_get_layout")

@@ -183,7 +183,8 @@ static int decode_stage_items(const kvq_config& c) {
 // and few enough that every CTA owns at least one chunk, so each CTA between a
 // row's first and last contributor has work in that row.  Returns the CTA
 // count (0 when the item indices would not fit in 32 bits).
-static int plan_decode(const kvq_config& c, int64_t n_groups, int r, int32_t* n_items, int32_t* item0) {
+static int plan_decode(const kvq_config& c, int64_t n_groups, int r, int sms_avail, int32_t* n_items,
+                       int32_t* item0) {
   // weights of a stage of quantized items and of a window chunk: a window
   // chunk's stage takes about 1.5 times a full stage of groups (measured)
   constexpr int64_t kWs = 2, kWw = 3;
@@ -194,7 +195,7 @@ static int plan_decode(const kvq_config& c, int64_t n_groups, int r, int32_t* n_
   if (rows * (n_groups + n_w) >= ((int64_t)1 << 31)) return 0;
   *n_items = (int32_t)(n_groups + n_w);
   const int64_t U = rows * (((n_groups + sg - 1) / sg) * kWs + n_w * kWw);
-  const int64_t sms = num_sms() < kMaxDecodeCtas ? num_sms() : kMaxDecodeCtas;
+  const int64_t sms = sms_avail < kMaxDecodeCtas ? sms_avail : kMaxDecodeCtas;
   int n = (int)std::max<int64_t>(1, std::min<int64_t>(sms, U / kWw));
   while (n > 1 && !partition_items(rows, n_groups, sg, n_w, kWs, kWw, n, item0)) --n;
   if (n == 1) partition_items(rows, n_groups, sg, n_w, kWs, kWw, 1, item0);
@@ -418,7 +419,7 @@ static kvq_status launch_attention(const kvq_cache* h, int r, const void* q, flo
   a.counters = reinterpret_cast<unsigned*>(h->base + h->lay.status_offset) + 1;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.n_groups = h->tq / c.group;
-  a.n_cta = plan_decode(c, a.n_groups, r, &a.n_items, a.item0);
+  a.n_cta = plan_decode(c, a.n_groups, r, num_sms(), &a.n_items, a.item0);
   if (a.n_cta <= 0) return KVQ_ERR_UNSUPPORTED;
   a.r = r;
   a.head = h->head;
@@ -520,7 +521,19 @@ const char* kvq_cuda_error_string(void) { return g_cuda_error; }
 int32_t kvq_decode_splits(const kvq_cache* h) {
   if (!h) return -1;
   int32_t n_items, item0[kMaxDecodeCtas + 1];
-  return plan_decode(h->cfg, h->tq / h->cfg.group, h->r, &n_items, item0);
+  return plan_decode(h->cfg, h->tq / h->cfg.group, h->r, num_sms(), &n_items, item0);
+}
+
+int32_t kvq_decode_partition(const kvq_config* cfg, int64_t n_groups, int32_t r, int32_t sms, int32_t* item0,
+                             int32_t cap, int32_t* n_items) {
+  if (!cfg || !item0 || !n_items || !config_ok(cfg) || n_groups < 0 || r < 0 || sms < 1) return 0;
+  int32_t tmp[kMaxDecodeCtas + 1];
+  int32_t ni = 0;
+  const int n = plan_decode(*cfg, n_groups, r, sms, &ni, tmp);
+  if (n <= 0 || cap < n + 1) return 0;
+  std::memcpy(item0, tmp, sizeof(int32_t) * (size_t)(n + 1));
+  *n_items = ni;
+  return n;
 }
 
 }  // extern "C"
