@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "quantized-KV decode attn: packed-KV GB/s (% of HBM peak), tokens/s"
 HBM_FALLBACK_GBS = 6650.0
-NORTH_STAR_HBM_GBS = 8000.0
+NOMINAL_HBM_GBS = 8000.0   # the B200 HBM3e peak as usually quoted (DGX figure)
 
 
 def _profiled_traffic(kernel: str, source: str, workload: str):
@@ -475,7 +475,7 @@ def main():
                   else "f16 mma (fp32 accumulate) over int2/int4 codes"),
         "data": "synthetic", "config": cfg_desc,
         "tokens_per_s": round(w.batch * world * args.steps / (res["ms"] * 1e-3), 1),
-        "pct_of_north_star_hbm": round(100 * value / world / NORTH_STAR_HBM_GBS, 2),
+        "pct_of_nominal_8tbs_hbm": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         "roofline": {"bound": "hbm", "kernel": kern_desc,
                      "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4),
