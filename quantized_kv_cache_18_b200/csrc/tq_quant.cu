@@ -11,8 +11,9 @@
 //
 // Readings: the residual is taken in rotated coordinates; a coordinate equal
 // to a threshold goes to the lower cell; a sketch value of exactly 0 gives bit
-// 1; the zero vector has u = 0.  Codes are decided on y computed in fp32 (Pi
-// in fp32, fp32 accumulation).
+// 1; the zero vector has u = 0.  Codes are decided on y computed to about
+// fp32 precision (Pi in fp32 and u, each split into fp16 hi + lo, fp32
+// accumulation; below).
 //
 // One persistent CTA per SM keeps 16 Pi^T and S^T in shared memory as
 // mma.sync B fragments, each split into fp16 hi + lo, and runs three (row,
