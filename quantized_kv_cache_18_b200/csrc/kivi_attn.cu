@@ -93,7 +93,7 @@ struct K {
 
 // ------------------------------------------------------------------ work partition
 // Items of a row: groups 0..n_g-1, then window chunks of kWinTok tokens.  The
-// host cuts the (row, item) sequence into byte-balanced CTA ranges (item0 in
+// host cuts the (row, item) sequence into stage-balanced CTA ranges (item0 in
 // the launch arguments, read from the grid-constant parameter space).
 struct Part {
   int n_g, n_items, n_cta;

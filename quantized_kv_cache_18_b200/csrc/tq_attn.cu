@@ -90,7 +90,7 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t w) {
 }
 
 // Work partition: items of a row are n_tb token blocks then n_wc window-type
-// chunks; the host cuts the (row, item) sequence into byte-balanced CTA ranges
+// chunks; the host cuts the (row, item) sequence into stage-balanced CTA ranges
 // (item0 in the launch arguments, read from the grid-constant parameter space).
 struct TPart {
   int n_tb, n_items, n_wc, n_cta;
