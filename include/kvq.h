@@ -296,7 +296,12 @@ kvq_status kvq_decode_attention_static(const kvq_cache* cache, const void* q, fl
 /*
  * Synchronises `stream`, reads the device status word into *bits (may be
  * NULL) and returns KVQ_ERR_DEVICE_STATUS if any bit is set, else KVQ_OK.
- * `clear` != 0 also zeroes the word.
+ * `clear` != 0 also zeroes the word and the per-row arrival counters of the
+ * decode merge (enqueued on `stream`).
+ * After KVQ_DEV_WAIT_TIMEOUT the outputs of the launch that set it are
+ * unspecified, and so is the window slot of the new token when that launch
+ * was a fused step (kvq_append_decode); the cache's other contents are
+ * unchanged, and after a clear the next call computes normally.
  */
 kvq_status kvq_get_status(kvq_cache* cache, uint32_t* bits, int32_t clear, void* stream);
 
@@ -326,6 +331,25 @@ const char* kvq_cuda_error_string(void);
 /* Kernels this library has launched since it was loaded (all handles). */
 uint64_t kvq_launch_count(void);
 
+/*
+ * Test hook for the decode kernels' bounded waits (no counterpart on the
+ * pages).  Every pipeline wait inside a decode launch gives up after a bound
+ * (default: about 1 s of SM clock cycles); a wait that gives up sets
+ * KVQ_DEV_WAIT_TIMEOUT and the launch finishes without writing outputs it
+ * cannot trust, leaving the GPU context usable.  This call lets a test reach
+ * that path without a GPU fault:
+ *   wait_cycles           the bound in SM clock cycles for later decode
+ *                         launches of this process (0 restores the default;
+ *                         values above the default are rejected);
+ *   withhold_first_stage  nonzero: CTA 0 of later decode launches does not
+ *                         issue the copy of its first pipeline stage, so the
+ *                         waits on that stage run out after `wait_cycles`.
+ * Waits for copies already in flight before a CTA exits keep the default
+ * bound.  Process-wide, not thread-safe against concurrent launches; for
+ * tests only.  Returns KVQ_ERR_INVALID_ARG for a bound above the default.
+ */
+kvq_status kvq_debug_set_wait_test(uint64_t wait_cycles, int32_t withhold_first_stage);
+
 /* Decode-attention split count the library picks for the current state. */
 int32_t kvq_decode_splits(const kvq_cache* cache);
 
@@ -337,7 +361,7 @@ int32_t kvq_decode_splits(const kvq_cache* cache);
  * CTA c of the decode launch owns the global items item0[c] .. item0[c+1]-1
  * (global item = row x n_items + item); item0[0] = 0, item0[n] = rows x
  * n_items, strictly increasing.  The ranges balance stages (a stage carries
- * up to 12, 8, 6 or 4 KIVI groups, by formulation and G, or 8 TURBO blocks;
+ * up to 12 KIVI groups for G = 32, 6 for G = 64, or 8 TURBO blocks;
  * a window chunk's stage weighs 1.5 of them) and quantized ranges start at a
  * stage boundary of their row.  Fills item0[0 .. n] (caller-owned, `cap`
  * entries) and returns n, or 0 for a null pointer, an unsupported

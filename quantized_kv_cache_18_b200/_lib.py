@@ -50,6 +50,7 @@ _SIGS = {
     "kvq_cache_destroy": (None, [_P]),
     "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvq_launch_count": (ctypes.c_uint64, []),
+    "kvq_debug_set_wait_test": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int32]),
     "kvq_cuda_error_string": (ctypes.c_char_p, []),
     "kvq_decode_splits": (ctypes.c_int32, [_P]),
     "kvq_decode_partition": (ctypes.c_int32, [_P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32, _P]),

@@ -54,18 +54,28 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* b, uint32_t parity
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false if the phase did not complete before the deadline or the
-// CTA is already aborting.
-// The deadline is checked on the SM cycle counter (cheap to read) every 64
-// polls; kWaitCycles is about 1 s at the B200's top clock.
-constexpr long long kWaitCycles = 2000000000ll;
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
+// Bounded wait: false if the phase did not complete within `limit` SM cycles
+// or the CTA is already aborting.  The default bound, kWaitCycles, is about
+// 1 s at the B200's top clock; the decode launches take theirs from the launch
+// arguments (a test may shorten it, see kvq_debug_set_wait_test).  Waits for
+// copies in flight before a CTA exits always use the default bound.
+constexpr long long kWaitCycles = kWaitCyclesDefault;
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                          long long limit = kWaitCycles) {
   if (mbar_try_wait(b, parity)) return true;
   const long long t0 = clock64();
+  const uint32_t ns = limit < 40000ll ? 0u : 20000u;   // a short bound polls instead of sleeping
   for (;;) {
-    if (mbar_try_wait_sleep(b, parity, 20000u)) return true;
+    if (mbar_try_wait_sleep(b, parity, ns)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
+  }
+}
+// Waits (bounded by the default limit) for a phase whose copy is in flight,
+// so that no bulk copy still writes this CTA's shared memory when it exits.
+__device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(b, parity) && clock64() - t0 < kWaitCycles) {
   }
 }
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

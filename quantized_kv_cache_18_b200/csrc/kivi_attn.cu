@@ -9,20 +9,24 @@
 // q~ = q (.) s (per group) and p~ = p (.) sv (per token) are split into fp16
 // hi + lo parts, and both contractions run on mma.sync with the exact
 // small-integer fp16 codes as the other operand.  Two formulations:
-//   head-major (GQA groups of 5..8 heads): the heads' hi | lo parts are the
-//     two 8-row halves of the m16 A operand and the codes are the B operand;
-//   token-major (groups of 1..4 heads): the codes are the A operand (tokens,
-//     resp. channels, are M) and the heads' hi | lo parts are the 8 columns
-//     of B, which halves the mma count and the accumulators of the
-//     head-major form for such groups and leaves room for 12 consumer warps.
+//   hybrid (GQA groups of 8 heads): scores head-major -- the heads' hi | lo
+//     parts are the two 8-row halves of the m16 A operand and the key codes
+//     are the B operand -- and P.V token-major -- the value codes are the A
+//     operand and p~ of the 8 heads the B operand, its hi and lo parts
+//     accumulated into one tile;
+//   token-major (groups of 1..4 heads): the codes are the A operand of both
+//     contractions (tokens, resp. channels, are M) and the heads' hi | lo
+//     parts are the 8 columns of B, half the mma's of the hybrid form for
+//     such groups.
 //
 // Structure (one CTA per SM, one launch per decode step):
 //   warp 0      producer: 1-D bulk copies (cp.async.bulk, no multicast) of whole
 //               group records / window rows into a ring of shared-memory stages
 //   warp 1      prep: the zero-point term beta = q . z for every group of a stage
 //               in batched mma's (columns = groups)
-//   warps 2..   consumers (8 head-major, 12 token-major): one 32-token block
-//               per warp per stage, online softmax
+//   warp 2      merge: the warp states of every segment but the CTA's last
+//   warps 3..   12 consumers: one 32-token block per warp per stage, online
+//               softmax
 // Work: the (row, item) sequence -- a row's groups then its 32-token window
 // chunks -- is cut on the host into ranges of equal stage count, one per CTA
 // (a window chunk's stage weighs 1.5 group stages).  A CTA writes one
@@ -134,11 +138,11 @@ __device__ __forceinline__ void for_each_chunk(const Part& P, int i0, int i1, FC
 }
 
 // ------------------------------------------------------------------ the kernel
-// The token-major variant runs 15 warps, the head-major one 11.  Declaring
-// 512 (384) threads caps them at 128 (168) registers, so that the four (three)
-// warps one SM sub-partition holds fit its 16,384-entry register file.
+// Both formulations run 15 warps.  Declaring 512 threads caps them at 128
+// registers, so that the four warps one SM sub-partition holds fit its
+// 16,384-entry register file.
 template <int BITS, int D, int G, bool TR>
-__global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __grid_constant__ AttnArgs a) {
+__global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_constant__ AttnArgs a) {
   using C = K<BITS, D, G, TR>;
   constexpr int P = D * BITS / 32;
   constexpr int J = BITS == 2 ? 4 : 2;
@@ -163,6 +167,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
   const Geom& gm = a.geom;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gr = lane >> 2, tc = lane & 3;
+  const long long wl = a.wait_cycles;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
@@ -247,15 +252,14 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
     // gpu-scope acq_rel atomic (release is cumulative), so one fenced atomic
     // publishes the whole partial; the last arriver's acquire plus the next
     // barrier make every partial visible to all the merging threads.
+    // An aborted CTA arrives as well (its partial is then unspecified), so the
+    // last arriver always resets the counter for the next launch; an aborted
+    // last arriver writes no output.
     sync();
     if (tid == 0) {
-      int last = 0;
-      if (!*abort_flag) {
-        unsigned old;
-        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;\n" : "=r"(old) : "l"(a.counters + row) : "memory");
-        last = old == (unsigned)(np - 1);
-      }
-      *s_last = last;
+      unsigned old;
+      asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;\n" : "=r"(old) : "l"(a.counters + row) : "memory");
+      *s_last = old == (unsigned)(np - 1);
     }
     sync();
     if (!*s_last) return;
@@ -286,17 +290,12 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
           bulk_g2s(smem, ws_row + (int64_t)j0 * g * DP, (uint32_t)(nj * PB), bar_merge);
           issued = true;
         }
-        const bool ok = !*abort_flag && mbar_wait(bar_merge, k & 1, abort_flag);
+        const bool ok = !*abort_flag && mbar_wait(bar_merge, k & 1, abort_flag, wl);
         if (!ok && !*abort_flag) {
           atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
           *abort_flag = 1;
         }
-        if (issued && !ok) {
-          // let the copy land before the CTA can exit (bounded)
-          const long long t0 = clock64();
-          while (!mbar_try_wait(bar_merge, k & 1) && clock64() - t0 < kWaitCycles) {
-          }
-        }
+        if (issued && !ok) mbar_drain(bar_merge, k & 1);   // the copy lands before the CTA can exit
         if (ok) {
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
@@ -346,7 +345,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
     // Last CTA of the row, merge warp: online log-sum-exp over the np partials,
     // the loads of up to kMB partials (o, m, l) in flight together.
     constexpr int kMB = 8;
-    for (int e4 = tid; e4 < g * D / 4; e4 += nth) {
+    for (int e4 = tid; e4 < g * D / 4 && !*abort_flag; e4 += nth) {
       const int h = e4 / (D / 4), c = 4 * (e4 - h * (D / 4));
       const float* col = ws_row + (int64_t)h * DP;
       float M = -INFINITY, L = 0.f;
@@ -402,7 +401,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
           const uint32_t par = (k >> 1) & 1;
           ++k;
           if (row == last_row) return;   // the consumer warps merge the CTA's last segment
-          const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[sbi], par, abort_flag));
+          const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[sbi], par, abort_flag, wl));
           if (!ok) {
             if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
             *abort_flag = 1;
@@ -421,7 +420,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued = 0, qseg = 0;
+      int issued = 0, qseg = 0, qissued = 0, withheld = -1;
       for_each_chunk<C::SG>(
           Pt, i0, i1,
           [&](int s, int row, bool win, int64_t first, int cnt) {
@@ -433,9 +432,17 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
             const bool paged = !win && gm.page_table != nullptr;
             RecordPages pages;
             if (paged) record_pages(gm, row, first, cnt, pages);
-            if (s >= C::NST && !mbar_wait(&bar_empty[slot], ((s / C::NST) - 1) & 1, abort_flag)) {
+            if (s >= C::NST && !mbar_wait(&bar_empty[slot], ((s / C::NST) - 1) & 1, abort_flag, wl)) {
               atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
               *abort_flag = 1;
+              return;
+            }
+            // consumers that gave up on this slot's previous copy set the flag
+            // before releasing the slot: that copy may still be in flight
+            if (*abort_flag) return;
+            if (s == 0 && cta == 0 && a.withhold_first_stage) {
+              withheld = 0;   // test hook: a stage whose wait nothing completes
+              issued = 1;
               return;
             }
             unsigned char* dst = smem + slot * C::STAGE;
@@ -477,25 +484,26 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
             if (*abort_flag) return;
             const int k = qseg++;
             const int qs = k & 1;
-            if (k >= 2 && !mbar_wait(&bar_qempty[qs], ((k >> 1) - 1) & 1, abort_flag)) {
+            if (k >= 2 && !mbar_wait(&bar_qempty[qs], ((k >> 1) - 1) & 1, abort_flag, wl)) {
               atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
               *abort_flag = 1;
               return;
             }
+            if (*abort_flag) return;
             const int b = row / gm.Hkv, hkv = row - b * gm.Hkv;
             const uint32_t bytes = (uint32_t)gm.g * D * 2;
             mbar_expect_tx(&bar_qfull[qs], bytes);
             bulk_g2s(sm_q + qs * 8 * D, a.q + ((int64_t)b * gm.Hq + (int64_t)hkv * gm.g) * D, bytes, &bar_qfull[qs]);
+            qissued = k + 1;
           },
           nop_seg);
-      if (*abort_flag) {
-        // let the copies already issued land before the CTA exits
-        for (int s = max(0, issued - C::NST); s < issued; ++s) {
-          const long long t0 = clock64();
-          while (!mbar_try_wait(&bar_full[s % C::NST], (s / C::NST) & 1) && clock64() - t0 < kWaitCycles) {
-          }
-        }
-      }
+      // Every copy issued lands before this warp exits (only the last NST
+      // stages and the last two q slots can still be in flight), so none can
+      // write shared memory after the CTA is gone, even when its consumers
+      // gave up waiting.
+      for (int s = max(0, issued - C::NST); s < issued; ++s)
+        if (s != withheld) mbar_drain(&bar_full[s % C::NST], (s / C::NST) & 1);
+      for (int k = max(0, qissued - 2); k < qissued; ++k) mbar_drain(&bar_qfull[k & 1], (k >> 1) & 1);
     }
     return;
   }
@@ -509,7 +517,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
         [&](int s, int row, bool win, int64_t first, int cnt) {
           const int slot = s % C::NST;
           // warp-uniform: every lane must take the mma below together
-          const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_full[slot], (s / C::NST) & 1, abort_flag));
+          const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_full[slot], (s / C::NST) & 1, abort_flag, wl));
           if (!ok) {
             if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
             *abort_flag = 1;
@@ -542,7 +550,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
           (void)row;
           const int k = qseg++;
           const int qs = k & 1;
-          const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_qfull[qs], (k >> 1) & 1, abort_flag));
+          const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_qfull[qs], (k >> 1) & 1, abort_flag, wl));
           if (!ok) {
             if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
             *abort_flag = 1;
@@ -566,7 +574,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
   // ------------------------------------------------------------------ consumers
   const int cw = warp - 3;
   // Head whose q this lane feeds to the score contraction: gr in the
-  // head-major formulation; gr >> 1 in the token-major one, where column gr of
+  // hybrid formulation; gr >> 1 in the token-major one, where column gr of
   // the q~ operand is the hi (even gr) or lo (odd gr) part of head gr >> 1.
   const int qhead = TR ? gr >> 1 : gr;
   const bool head_ok = qhead < gm.g;
@@ -574,10 +582,11 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
   int qseg = 0;
   const uint16_t* sq = sm_q;   // ring slot of the current segment
   uint32_t qh[NKT][2];   // q of head qhead at channels 16kt + 8rho + 2tc + {0, 1}, fp16x2
-  // Output accumulators.  Head-major: m16n8 tiles (rows = heads hi | lo,
-  // columns = 8 channels).  Token-major: m16n8 tiles (rows = 16 channels,
-  // columns = heads x {hi, lo}); this lane then holds head tc only.
-  constexpr int NO = TR ? D / 16 : NNT;
+  // Output accumulators, m16n8 tiles with rows = 16 channels.  Hybrid:
+  // columns = the 8 heads (hi and lo parts of p~ accumulate into the same
+  // tile).  Token-major: columns = heads x {hi, lo}; this lane then holds
+  // head tc only.
+  constexpr int NO = D / 16;
   float o[NO][4];
   float m = -INFINITY, l = 0.f, wz = 0.f;
   int seg_row = 0;
@@ -586,7 +595,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
     seg_row = row;
     const int k = qseg++;
     const int qs = k & 1;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_qfull[qs], (k >> 1) & 1, abort_flag));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_qfull[qs], (k >> 1) & 1, abort_flag, wl));
     if (!ok) {
       if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
       *abort_flag = 1;
@@ -821,11 +830,233 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
     __syncwarp();
   };
 
+  // ---------------------------------------------------------------- hybrid formulation (GQA groups of 8)
+  // Scores head-major: A = q~ of the 8 heads, hi parts in rows 0-7 and lo
+  // parts in rows 8-15; B = key codes (k16 channels x n8 tokens of the packed
+  // format).  Lane (gr, tc) then holds the scores of head gr for tokens
+  // 8 nt + 2 tc + {0, 1} -- which is exactly the B fragment of a token-major
+  // P.V (k16 tokens x n8 heads), so p~ never leaves registers.  P.V: A = value
+  // codes (m16 channels x k16 tokens: the B fragments of two adjacent 8-channel
+  // tiles of the packed format), B = p~ of the 8 heads, split hi + lo, both
+  // accumulated into one C tile [16 channels x 8 heads].  The output
+  // accumulators are then 32 registers (64 in a purely head-major P.V, whose
+  // lo rows are dead accumulator space), which leaves room for 12 consumer
+  // warps.  Lane (gr, tc) holds the softmax state of head gr and the output of
+  // heads 2 tc, 2 tc + 1.
+  auto hx_rescale = [&](float mt) {
+    // warp-uniform branch: lanes whose max did not grow scale by 1
+    if (__any_sync(0xffffffffu, mt > m)) {
+      const float mn = fmaxf(m, mt);
+      const float alpha = m == -INFINITY ? 0.f : fast_exp2(m - mn);
+      l *= alpha;
+      wz *= alpha;
+      m = mn;
+      // the output columns are heads 2 tc and 2 tc + 1: their factors come
+      // from quad 2 tc and quad 2 tc + 1
+      const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * tc);
+      const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * tc + 4);
+#pragma unroll
+      for (int i = 0; i < NO; ++i) {
+        o[i][0] *= a0;
+        o[i][1] *= a1;
+        o[i][2] *= a0;
+        o[i][3] *= a1;
+      }
+    }
+  };
+  auto hx_block = [&](const unsigned char* st, int slot) {
+    const int grp = cw / C::NTB, tbg = cw - grp * C::NTB;
+    const unsigned char* rec = st + grp * C::REC;
+    uint4 kc[P / 4];
+#pragma unroll
+    for (int p = 0; p < P / 4; ++p) kc[p] = lds128(rec + tbg * C::TBC + 16 * (32 * p + lane));
+    const float bs = sm_beta[(slot * C::SG + grp) * 8 + gr] * a.scale_log2;
+    // this lane's key scales: 16 bytes per k-tile pair kt2 at 64 kt2 + 16 tc
+    const unsigned char* psc = rec + C::KSOFF + 16 * tc;
+    float sc[4][4];   // [n-tile]
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+    for (int wi = 0; wi < WPN; ++wi)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pr[4][J];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          const int w = nt * WPN + wi;
+          const uint4 pc = kc[w >> 2];
+          const uint32_t word = (w & 3) == 0 ? pc.x : (w & 3) == 1 ? pc.y : (w & 3) == 2 ? pc.z : pc.w;
+          unpack_half<BITS>(half ? word >> 8 : word, pr[nt], magic);
+        }
+#pragma unroll
+        for (int m2 = 0; m2 < J / 2; ++m2) {
+          const int kt = (J / 2) * (2 * wi + half) + m2;
+          const uint2 s2 = *reinterpret_cast<const uint2*>(psc + 64 * (kt >> 1) + 8 * (kt & 1));
+          const __half2 hi0 = __hmul2(u32_as_h2(qh[kt][0]), u32_as_h2(s2.x));
+          const __half2 hi1 = __hmul2(u32_as_h2(qh[kt][1]), u32_as_h2(s2.y));
+          const uint32_t aq[4] = {h2_as_u32(hi0), h2_as_u32(__hfma2(u32_as_h2(qh[kt][0]), u32_as_h2(s2.x), __hneg2(hi0))),
+                                  h2_as_u32(hi1), h2_as_u32(__hfma2(u32_as_h2(qh[kt][1]), u32_as_h2(s2.y), __hneg2(hi1)))};
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) mma_f16_16816(sc[nt], aq, pr[nt][2 * m2], pr[nt][2 * m2 + 1]);
+        }
+      }
+    float x[4][2];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        x[nt][e] = fmaf(sc[nt][e] + sc[nt][2 + e], a.scale_log2, bs);
+        mx = fmaxf(mx, x[nt][e]);
+      }
+    hx_rescale(quad_max(mx));
+    uint32_t vm[8];
+    {
+      const uint4* pv = reinterpret_cast<const uint4*>(rec + C::VMOFF + 4 * (tbg * kTB + 8 * tc));
+      const uint4 v0 = lds128(pv), v1 = lds128(pv + 1);
+      vm[0] = v0.x; vm[1] = v0.y; vm[2] = v0.z; vm[3] = v0.w;
+      vm[4] = v1.x; vm[5] = v1.y; vm[6] = v1.z; vm[7] = v1.w;
+    }
+    // B fragments of P.V: k-tile kt, b0 = tokens 16 kt + 2 tc + {0, 1} (n-tile
+    // 2 kt), b1 = tokens 16 kt + 8 + 2 tc + {0, 1} (n-tile 2 kt + 1); column gr
+    uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int nt = 2 * kt + rr;
+        float pt[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float p = fast_exp2(x[nt][e] - m);
+          const float2 sz = __half22float2(u32_as_h2(vm[2 * nt + e]));
+          l += p;
+          wz = fmaf(p, sz.y, wz);
+          // value pair position j' of token 8 nt + 2 tc + e: nt (2-bit), nt & 1 (4-bit)
+          pt[e] = p * (sz.x * pos_comp_f(BITS, BITS == 2 ? nt : (nt & 1)));
+        }
+        const __half2 hi = __floats2half2_rn(pt[0], pt[1]);
+        const float2 hb = __half22float2(hi);
+        bh[kt][rr] = h2_as_u32(hi);
+        bl[kt][rr] = h2_as_u32(__floats2half2_rn(pt[0] - hb.x, pt[1] - hb.y));
+      }
+    uint4 vc[P / 4];
+#pragma unroll
+    for (int p = 0; p < P / 4; ++p) vc[p] = lds128(rec + (C::NTB + tbg) * C::TBC + 16 * (32 * p + lane));
+    auto vword = [&](int w) {
+      const uint4 pc = vc[w >> 2];
+      return (w & 3) == 0 ? pc.x : (w & 3) == 1 ? pc.y : (w & 3) == 2 ? pc.z : pc.w;
+    };
+    // k-tile-major: every m-tile's kt = 0 mma's before any kt = 1 mma, so the
+    // mma's into one accumulator are far apart (legacy mma.sync has a long latency)
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt)
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        uint32_t av[4];
+        if (BITS == 2) {
+          // channels 16mt + gr (low byte of each half word) and 16mt + 8 + gr (high byte)
+          const uint32_t w = vword(mt);
+          av[0] = kt ? unpack_pair<2, 2>(w, magic) : unpack_pair<2, 0>(w, magic);
+          av[1] = kt ? unpack_pair<2, 2>(w >> 8, magic) : unpack_pair<2, 0>(w >> 8, magic);
+          av[2] = kt ? unpack_pair<2, 3>(w, magic) : unpack_pair<2, 1>(w, magic);
+          av[3] = kt ? unpack_pair<2, 3>(w >> 8, magic) : unpack_pair<2, 1>(w >> 8, magic);
+        } else {
+          // words 2mt (channel 16mt + gr) and 2mt + 1 (16mt + 8 + gr); half word = kt
+          const uint32_t w0 = kt ? vword(2 * mt) >> 8 : vword(2 * mt);
+          const uint32_t w1 = kt ? vword(2 * mt + 1) >> 8 : vword(2 * mt + 1);
+          av[0] = unpack_pair<4, 0>(w0, magic);
+          av[1] = unpack_pair<4, 0>(w1, magic);
+          av[2] = unpack_pair<4, 1>(w0, magic);
+          av[3] = unpack_pair<4, 1>(w1, magic);
+        }
+        mma_f16_16816(o[mt], av, bh[kt][0], bh[kt][1]);
+        mma_f16_16816(o[mt], av, bl[kt][0], bl[kt][1]);
+      }
+  };
+  // Window chunk: warps 0 and 1 take tokens 16 cw .. 16 cw + 15 (exact 16-bit
+  // operands).  Scores head-major (A = q rows of the 8 heads, rows 8-15 zero;
+  // B = key rows by ldmatrix), P.V token-major (A = value rows transposed by
+  // ldmatrix; B = p split hi + lo in the input's format).
+  auto hx_window = [&](const unsigned char* st, int64_t first) {
+    const int n_tok = min(kWinTok, a.r - (int)first * kWinTok);
+    const int t0 = 16 * cw;
+    if (cw >= kWinTok / 16 || t0 >= n_tok) return;
+    const unsigned char* kb = st;
+    const unsigned char* vb = st + kWinTok * C::WROW;
+    const bool bf = gm.dtype == KVQ_BF16;
+    const int mi = lane >> 3, ri = lane & 7;   // ldmatrix: matrix and row this lane addresses
+    const uint16_t* qr = sq + gr * D;
+    float sw[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int krow = min(t0 + 8 * nt + ri, kWinTok - 1);
+#pragma unroll
+      for (int kt2 = 0; kt2 < NKT / 2; ++kt2) {
+        uint32_t bk[4];
+        ldsm_x4(bk, kb + krow * C::WROW + (16 * (2 * kt2 + (mi >> 1)) + 8 * (mi & 1)) * 2);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int kt = 2 * kt2 + h2;
+          const uint32_t aq[4] = {*reinterpret_cast<const uint32_t*>(qr + 16 * kt + 2 * tc), 0u,
+                                  *reinterpret_cast<const uint32_t*>(qr + 16 * kt + 8 + 2 * tc), 0u};
+          if (bf) mma_bf16_16816(sw[nt], aq, bk[2 * h2], bk[2 * h2 + 1]);
+          else mma_f16_16816(sw[nt], aq, bk[2 * h2], bk[2 * h2 + 1]);
+        }
+      }
+    }
+    float xv[2][2];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool valid = t0 + 8 * nt + 2 * tc + e < n_tok;
+        xv[nt][e] = valid ? sw[nt][e] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, xv[nt][e]);
+      }
+    hx_rescale(quad_max(mx));
+    uint32_t ph[2], pl[2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float pw[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        pw[e] = xv[nt][e] == -INFINITY ? 0.f : fast_exp2(xv[nt][e] - m);
+        l += pw[e];
+      }
+      ph[nt] = pack2_in16(pw[0], pw[1], gm.dtype);
+      const float2 pb = unpack2_in16(ph[nt], gm.dtype);
+      pl[nt] = pack2_in16(pw[0] - pb.x, pw[1] - pb.y, gm.dtype);
+    }
+    // rows past n_tok are zeroed so stale shared memory never meets the zero weights
+    const int vrow = min(t0 + 8 * (mi >> 1) + ri, kWinTok - 1);
+    const uint32_t m01 = (t0 + 2 * tc < n_tok ? 0x0000FFFFu : 0u) | (t0 + 2 * tc + 1 < n_tok ? 0xFFFF0000u : 0u);
+    const uint32_t m23 =
+        (t0 + 8 + 2 * tc < n_tok ? 0x0000FFFFu : 0u) | (t0 + 8 + 2 * tc + 1 < n_tok ? 0xFFFF0000u : 0u);
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      uint32_t av[4];
+      ldsm_x4_t(av, vb + vrow * C::WROW + (16 * mt + 8 * (mi & 1)) * 2);
+      av[0] &= m01;
+      av[1] &= m01;
+      av[2] &= m23;
+      av[3] &= m23;
+      if (bf) {
+        mma_bf16_16816(o[mt], av, ph[0], ph[1]);
+        mma_bf16_16816(o[mt], av, pl[0], pl[1]);
+      } else {
+        mma_f16_16816(o[mt], av, ph[0], ph[1]);
+        mma_f16_16816(o[mt], av, pl[0], pl[1]);
+      }
+    }
+  };
+
   auto chunk = [&](int s, int row, bool win, int64_t first, int cnt) {
     const int slot = s % C::NST;
     const uint32_t par = (s / C::NST) & 1;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_full[slot], par, abort_flag) &&
-                                                mbar_wait(&bar_ready[slot], par, abort_flag));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_full[slot], par, abort_flag, wl) &&
+                                                mbar_wait(&bar_ready[slot], par, abort_flag, wl));
     if (!ok) {
       if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
       *abort_flag = 1;
@@ -858,171 +1089,9 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
     if constexpr (TR) {
       if (ok && !win && cw < cnt * C::NTB) tr_block(st, slot);
       else if (ok && win) tr_window(st, first);
-    } else if (ok && !win && cw < cnt * C::NTB) {
-      // ---------------------------------------------------------- one quantized TB
-      const int grp = cw / C::NTB, tbg = cw - grp * C::NTB;
-      const unsigned char* rec = st + grp * C::REC;
-      uint4 kc[P / 4];
-#pragma unroll
-      for (int p = 0; p < P / 4; ++p) kc[p] = lds128(rec + tbg * C::TBC + 16 * (32 * p + lane));
-      const float bs = sm_beta[(slot * C::SG + grp) * 8 + gr] * a.scale_log2;
-      // this lane's key scales: 16 bytes per k-tile pair kt2 at 64 kt2 + 16 tc
-      const unsigned char* psc = rec + C::KSOFF + 16 * tc;
-      float sc[4][4];   // [n-tile]
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-#pragma unroll
-      for (int wi = 0; wi < WPN; ++wi)
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pr[4][J];
-#pragma unroll
-          for (int nt = 0; nt < 4; ++nt) {
-            const int w = nt * WPN + wi;
-            const uint4 pc = kc[w >> 2];
-            const uint32_t word = (w & 3) == 0 ? pc.x : (w & 3) == 1 ? pc.y : (w & 3) == 2 ? pc.z : pc.w;
-            unpack_half<BITS>(half ? word >> 8 : word, pr[nt], magic);
-          }
-#pragma unroll
-          for (int m2 = 0; m2 < J / 2; ++m2) {
-            const int kt = (J / 2) * (2 * wi + half) + m2;
-            const uint2 s2 = *reinterpret_cast<const uint2*>(psc + 64 * (kt >> 1) + 8 * (kt & 1));
-            const __half2 hi0 = __hmul2(u32_as_h2(qh[kt][0]), u32_as_h2(s2.x));
-            const __half2 hi1 = __hmul2(u32_as_h2(qh[kt][1]), u32_as_h2(s2.y));
-            const uint32_t aq[4] = {h2_as_u32(hi0), h2_as_u32(__hfma2(u32_as_h2(qh[kt][0]), u32_as_h2(s2.x), __hneg2(hi0))),
-                                    h2_as_u32(hi1), h2_as_u32(__hfma2(u32_as_h2(qh[kt][1]), u32_as_h2(s2.y), __hneg2(hi1)))};
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) mma_f16_16816(sc[nt], aq, pr[nt][2 * m2], pr[nt][2 * m2 + 1]);
-          }
-        }
-      float x[4][2];
-      float mt = -INFINITY;
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          x[nt][e] = fmaf(sc[nt][e] + sc[nt][2 + e], a.scale_log2, bs);
-          mt = fmaxf(mt, x[nt][e]);
-        }
-      rescale_to(quad_max(mt));
-      uint32_t vm[8];
-      {
-        const uint4* pv = reinterpret_cast<const uint4*>(rec + C::VMOFF + 4 * (tbg * kTB + 8 * tc));
-        const uint4 v0 = lds128(pv), v1 = lds128(pv + 1);
-        vm[0] = v0.x; vm[1] = v0.y; vm[2] = v0.z; vm[3] = v0.w;
-        vm[4] = v1.x; vm[5] = v1.y; vm[6] = v1.z; vm[7] = v1.w;
-      }
-      uint32_t apv[2][4];
-#pragma unroll
-      for (int kt = 0; kt < 2; ++kt)
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int nt = 2 * kt + rr;
-          float pt[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float p = fast_exp2(x[nt][e] - m);
-            const uint32_t meta = vm[2 * nt + e];
-            const float2 sz = __half22float2(u32_as_h2(meta));
-            l += p;
-            wz = fmaf(p, sz.y, wz);
-            // value pair position j' = 2kt + rho (2-bit) or rho (4-bit)
-            pt[e] = p * (sz.x * pos_comp_f(BITS, BITS == 2 ? 2 * kt + rr : rr));
-          }
-          const __half2 hi = __floats2half2_rn(pt[0], pt[1]);
-          const float2 hb = __half22float2(hi);
-          const __half2 lo = __floats2half2_rn(pt[0] - hb.x, pt[1] - hb.y);
-          apv[kt][2 * rr] = h2_as_u32(hi);
-          apv[kt][2 * rr + 1] = h2_as_u32(lo);
-        }
-      uint4 vc[P / 4];
-#pragma unroll
-      for (int p = 0; p < P / 4; ++p) vc[p] = lds128(rec + (C::NTB + tbg) * C::TBC + 16 * (32 * p + lane));
-      // k-tile-major: every n-tile's kt = 0 mma before any kt = 1 mma, so the two
-      // mma's into one accumulator are far apart (legacy mma.sync has a long latency)
-#pragma unroll
-      for (int kt = 0; kt < 2; ++kt)
-#pragma unroll
-        for (int w = 0; w < P; ++w) {
-          const uint4 pc = vc[w >> 2];
-          const uint32_t word = (w & 3) == 0 ? pc.x : (w & 3) == 1 ? pc.y : (w & 3) == 2 ? pc.z : pc.w;
-          if (BITS == 2) {
-            // pairs j' = 2kt, 2kt + 1 of both half words: n-tiles 2w (low half) and 2w + 1
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const uint32_t x = half ? word >> 8 : word;
-              const uint32_t b0 = kt ? unpack_pair<2, 2>(x, magic) : unpack_pair<2, 0>(x, magic);
-              const uint32_t b1 = kt ? unpack_pair<2, 3>(x, magic) : unpack_pair<2, 1>(x, magic);
-              mma_f16_16816(o[2 * w + half], apv[kt], b0, b1);
-            }
-          } else {
-            // 4-bit: half word = kt, pairs j' = 0, 1 = rho
-            const uint32_t x = kt ? word >> 8 : word;
-            mma_f16_16816(o[w], apv[kt], unpack_pair<4, 0>(x, magic), unpack_pair<4, 1>(x, magic));
-          }
-        }
-    } else if (ok && win) {
-      // ---------------------------------------------------------- window tokens 4cw..4cw+3 (exact 16-bit)
-      // scores: rows = heads (q, exact in its own format), columns = the 8 tokens
-      // from 4cw (the upper 4 belong to the next warp and are masked); P.V with
-      // p split hi + lo in the same format, one 16-token k-tile of which only the
-      // first 4 columns are non-zero
-      const int n_tok = min(kWinTok, a.r - (int)first * kWinTok);
-      const int t0 = 4 * cw;
-      const unsigned char* kb = st;
-      const unsigned char* vb = st + kWinTok * C::WROW;
-      const bool bf = gm.dtype == KVQ_BF16;
-      float sw[4] = {0.f, 0.f, 0.f, 0.f};
-      const int mi = lane >> 3, ri = lane & 7;   // ldmatrix: matrix and row this lane addresses
-      const int krow = min(t0 + ri, kWinTok - 1);
-#pragma unroll
-      for (int kt2 = 0; kt2 < NKT / 2; ++kt2) {
-        uint32_t bk[4];
-        ldsm_x4(bk, kb + krow * C::WROW + (16 * (2 * kt2 + (mi >> 1)) + 8 * (mi & 1)) * 2);
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int kt = 2 * kt2 + h2;
-          const uint32_t aq[4] = {head_ok ? *reinterpret_cast<const uint32_t*>(sq + gr * D + 16 * kt + 2 * tc) : 0u, 0u,
-                                  head_ok ? *reinterpret_cast<const uint32_t*>(sq + gr * D + 16 * kt + 8 + 2 * tc) : 0u,
-                                  0u};
-          if (bf) mma_bf16_16816(sw, aq, bk[2 * h2], bk[2 * h2 + 1]);
-          else mma_f16_16816(sw, aq, bk[2 * h2], bk[2 * h2 + 1]);
-        }
-      }
-      float xv[2];
-      float mt = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int t = t0 + 2 * tc + e;
-        const bool valid = head_ok && tc < 2 && t < n_tok;
-        xv[e] = valid ? sw[e] * a.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, xv[e]);
-      }
-      rescale_to(quad_max(mt));
-      float pw[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        pw[e] = xv[e] == -INFINITY ? 0.f : fast_exp2(xv[e] - m);
-        l += pw[e];
-      }
-      const uint32_t ph = pack2_in16(pw[0], pw[1], gm.dtype);
-      const float2 pb = unpack2_in16(ph, gm.dtype);
-      const uint32_t pl = pack2_in16(pw[0] - pb.x, pw[1] - pb.y, gm.dtype);
-      const uint32_t apw[4] = {ph, pl, 0u, 0u};
-      // value rows t0 + 2tc, t0 + 2tc + 1 of the k-tile: zero those past n_tok so
-      // stale shared memory never meets the zero weights
-      const uint32_t vmask = (t0 + 2 * tc < n_tok ? 0x0000FFFFu : 0u) | (t0 + 2 * tc + 1 < n_tok ? 0xFFFF0000u : 0u);
-      const int vrow = min(t0 + ri, kWinTok - 1);
-#pragma unroll
-      for (int n4 = 0; n4 < NNT / 4; ++n4) {
-        uint32_t bv[4];
-        ldsm_x4_t(bv, vb + vrow * C::WROW + 8 * (4 * n4 + mi) * 2);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (bf) mma_bf16_16816(o[4 * n4 + j], apw, bv[j] & vmask, 0u);
-          else mma_f16_16816(o[4 * n4 + j], apw, bv[j] & vmask, 0u);
-        }
-      }
+    } else {
+      if (ok && !win && cw < cnt * C::NTB) hx_block(st, slot);
+      else if (ok && win) hx_window(st, first);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar_empty[slot]);
@@ -1036,7 +1105,7 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
     const int sbi = k & 1;
     float* sb = sm_state + sbi * C::SBUF_F;
     if (k >= 2) {
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfree[sbi], ((k >> 1) - 1) & 1, abort_flag));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfree[sbi], ((k >> 1) - 1) & 1, abort_flag, wl));
       if (!ok) {
         if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
         *abort_flag = 1;
@@ -1063,15 +1132,22 @@ __global__ void __launch_bounds__(TR ? 512 : 384, 1) kivi_decode_kernel(const __
         s_o[(cw * C::HS + tc) * D + 16 * mt + 8 + gr] = o[mt][2] + o[mt][3] + wzs;
       }
     } else {
+      // softmax state of head gr; output columns heads 2 tc, 2 tc + 1
       const float ls = quad_sum(l), wzs = quad_sum(wz);
       if (tc == 0) {
         s_m[cw * C::HS + gr] = m;
         s_l[cw * C::HS + gr] = ls;
       }
+      const float wz0 = __shfl_sync(0xffffffffu, wzs, 8 * tc), wz1 = __shfl_sync(0xffffffffu, wzs, 8 * tc + 4);
+      float* o0 = s_o + (cw * C::HS + 2 * tc) * D;
+      float* o1 = o0 + D;
 #pragma unroll
-      for (int nt = 0; nt < NNT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) s_o[(cw * C::HS + gr) * D + 8 * nt + 2 * tc + e] = o[nt][e] + o[nt][2 + e] + wzs;
+      for (int mt = 0; mt < NO; ++mt) {
+        o0[16 * mt + gr] = o[mt][0] + wz0;
+        o1[16 * mt + gr] = o[mt][1] + wz1;
+        o0[16 * mt + 8 + gr] = o[mt][2] + wz0;
+        o1[16 * mt + 8 + gr] = o[mt][3] + wz1;
+      }
     }
     __syncwarp();
     if (lane == 0) {

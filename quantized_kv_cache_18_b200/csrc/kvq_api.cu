@@ -29,6 +29,9 @@ namespace kvq {
 
 static std::atomic<uint64_t> g_launches{0};
 static thread_local const char* g_cuda_error = "no error";
+// Test hook of the decode kernels' bounded waits (kvq_debug_set_wait_test).
+static std::atomic<long long> g_wait_cycles{0};   // 0: the default bound
+static std::atomic<int> g_withhold{0};
 
 // Records the failing CUDA call's message for kvq_cuda_error_string.
 static kvq_status cuda_failed(cudaError_t e) {
@@ -192,6 +195,8 @@ static int plan_decode(const kvq_config& c, int64_t n_groups, int r, int sms_ava
   const int A = c.scheme == KVQ_TURBO ? c.anchor_tokens : 0;
   const int64_t n_w = (r + kDecodeWinTok - 1) / kDecodeWinTok + A / kDecodeWinTok;
   const int sg = decode_stage_items(c);
+  // nothing to attend (an empty cache): no launch, and no partition to divide by
+  if (rows * (n_groups + n_w) == 0) return 0;
   if (rows * (n_groups + n_w) >= ((int64_t)1 << 31)) return 0;
   *n_items = (int32_t)(n_groups + n_w);
   const int64_t U = rows * (((n_groups + sg - 1) / sg) * kWs + n_w * kWw);
@@ -423,6 +428,9 @@ static kvq_status launch_attention(const kvq_cache* h, int r, const void* q, flo
   if (a.n_cta <= 0) return KVQ_ERR_UNSUPPORTED;
   a.r = r;
   a.head = h->head;
+  const long long wc = g_wait_cycles.load(std::memory_order_relaxed);
+  a.wait_cycles = wc > 0 ? wc : kWaitCyclesDefault;
+  a.withhold_first_stage = g_withhold.load(std::memory_order_relaxed);
   a.k_new = static_cast<const uint16_t*>(k_new);
   a.v_new = static_cast<const uint16_t*>(v_new);
   if (c.scheme == KVQ_TURBO) {
@@ -472,7 +480,9 @@ kvq_status kvq_get_status(kvq_cache* h, uint32_t* bits, int32_t clear, void* str
   cudaError_t e = cudaMemcpyAsync(&v, dev, sizeof(v), cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_failed(e);
-  if (clear) launch_clear_words(dev, 1, st);
+  // the clear also zeroes the rows' arrival counters, which a launch whose
+  // waits ran out may have left behind
+  if (clear) launch_clear_words(dev, 1 + h->cfg.batch * h->cfg.num_kv_heads, st);
   if (bits) *bits = v;
   return v ? KVQ_ERR_DEVICE_STATUS : KVQ_OK;
 }
@@ -516,10 +526,18 @@ const char* kvq_status_string(kvq_status s) {
 
 uint64_t kvq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+kvq_status kvq_debug_set_wait_test(uint64_t wait_cycles, int32_t withhold_first_stage) {
+  if (wait_cycles > (uint64_t)kWaitCyclesDefault) return KVQ_ERR_INVALID_ARG;
+  g_wait_cycles.store((long long)wait_cycles, std::memory_order_relaxed);
+  g_withhold.store(withhold_first_stage ? 1 : 0, std::memory_order_relaxed);
+  return KVQ_OK;
+}
+
 const char* kvq_cuda_error_string(void) { return g_cuda_error; }
 
 int32_t kvq_decode_splits(const kvq_cache* h) {
   if (!h) return -1;
+  if (h->seq_len <= 0) return 0;   // an empty cache launches nothing
   int32_t n_items, item0[kMaxDecodeCtas + 1];
   return plan_decode(h->cfg, h->tq / h->cfg.group, h->r, num_sms(), &n_items, item0);
 }

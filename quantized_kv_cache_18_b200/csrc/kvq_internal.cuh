@@ -40,8 +40,9 @@ constexpr int kFp8RowBytes = 144;   // FP8 token row: 128 E4M3 codes, fp16 scale
 constexpr int kMaxDecodeCtas = 160;   // decode launches use at most this many CTAs (one per SM)
 constexpr int kDecodeWinTok = 32;     // window tokens per decode work item
 constexpr int kKiviConsumersTM = 12;  // KIVI decode consumer warps, token-major formulation (GQA groups <= 4)
-constexpr int kKiviConsumersHM = 8;   // KIVI decode consumer warps, head-major formulation
+constexpr int kKiviConsumersHM = 12;  // KIVI decode consumer warps, hybrid formulation (GQA groups of 8)
 constexpr int kTqDecodeConsumers = 8; // TurboQuant decode consumer warps
+constexpr long long kWaitCyclesDefault = 2000000000ll;   // decode wait bound: about 1 s of SM cycles
 
 struct Geom {
   int scheme, d, bits, G, R, cap, B, Hkv, Hq, g, dtype;
@@ -249,6 +250,11 @@ struct AttnArgs {
   // item0[c] .. item0[c + 1] - 1 (strictly increasing), where a row's items
   // are its n_groups quantized items, then its window-type chunks.
   int32_t n_items;                        // items per row
+  // Bound of the kernel's waits in SM cycles (kWaitCycles unless a test set a
+  // shorter one) and, for tests of the timeout path, whether CTA 0 withholds
+  // the copy of its first stage (a wait that nothing completes).
+  long long wait_cycles;
+  int withhold_first_stage;
   int32_t item0[kMaxDecodeCtas + 1];
 };
 

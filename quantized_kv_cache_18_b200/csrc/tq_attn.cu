@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
   const Geom& gm = a.geom;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gr = lane >> 2, tc = lane & 3;
+  const long long wl = a.wait_cycles;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
     if (lane == 0) {
       mbar_expect_tx(bar_pi, D * D * 4);
       bulk_g2s(sm_pi, gm.params + kTqPi, D * D * 4, bar_pi);
-      int issued = 0, qseg = 0;
+      int issued = 0, qseg = 0, qissued = 0, withheld = -1;
       tq_for_each_chunk(
           Pt, i0, i1,
           [&](int s, int row, bool win, int64_t first, int cnt) {
@@ -206,9 +207,17 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
             const bool paged = !win && gm.page_table != nullptr;
             RecordPages pages;
             if (paged) record_pages(gm, row, first, cnt, pages);
-            if (s >= C::NST && !mbar_wait(&bar_empty[slot], ((s / C::NST) - 1) & 1, abort_flag)) {
+            if (s >= C::NST && !mbar_wait(&bar_empty[slot], ((s / C::NST) - 1) & 1, abort_flag, wl)) {
               atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
               *abort_flag = 1;
+              return;
+            }
+            // consumers that gave up on this slot's previous copy set the flag
+            // before releasing the slot: that copy may still be in flight
+            if (*abort_flag) return;
+            if (s == 0 && cta == 0 && a.withhold_first_stage) {
+              withheld = 0;   // test hook: a stage whose wait nothing completes
+              issued = 1;
               return;
             }
             unsigned char* dst = smem + slot * C::STAGE;
@@ -271,11 +280,13 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
             if (*abort_flag) return;
             const int k = qseg++;
             const int qs = k & 1;
-            if (k >= 2 && !mbar_wait(&bar_qempty[qs], ((k >> 1) - 1) & 1, abort_flag)) {
+            if (k >= 2 && !mbar_wait(&bar_qempty[qs], ((k >> 1) - 1) & 1, abort_flag, wl)) {
               atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
               *abort_flag = 1;
               return;
             }
+            if (*abort_flag) return;
+            qissued = k + 1;
             unsigned char* dq = sm_q + qs * C::QSLOT;
             if (part == 0) {
               mbar_expect_tx(&bar_qfull[qs], kTqQPrepBytes);
@@ -289,17 +300,14 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
             }
           },
           nop_seg);
-      if (*abort_flag) {
-        for (int s = max(0, issued - C::NST); s < issued; ++s) {
-          const long long t0 = clock64();
-          while (!mbar_try_wait(&bar_full[s % C::NST], (s / C::NST) & 1) && clock64() - t0 < kWaitCycles) {
-          }
-        }
-      }
-      // the Pi copy must land before the CTA exits
-      const long long t0 = clock64();
-      while (!mbar_try_wait(bar_pi, 0) && clock64() - t0 < kWaitCycles) {
-      }
+      // Every copy issued lands before this warp exits (only the last NST
+      // stages, the last two query slots and the Pi copy can still be in
+      // flight), so none can write shared memory after the CTA is gone, even
+      // when its consumers gave up waiting.
+      for (int s = max(0, issued - C::NST); s < issued; ++s)
+        if (s != withheld) mbar_drain(&bar_full[s % C::NST], (s / C::NST) & 1);
+      for (int k = max(0, qissued - 2); k < qissued; ++k) mbar_drain(&bar_qfull[k & 1], (k >> 1) & 1);
+      mbar_drain(bar_pi, 0);
     }
     return;
   }
@@ -331,7 +339,7 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
     (void)row;
     const int k = qseg++;
     const int qs = k & 1;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_qfull[qs], (k >> 1) & 1, abort_flag));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_qfull[qs], (k >> 1) & 1, abort_flag, wl));
     if (!ok) {
       if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
       *abort_flag = 1;
@@ -391,7 +399,7 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
   auto chunk = [&](int s, int row, bool win, int64_t first, int cnt) {
     const int slot = s % C::NST;
     const uint32_t par = (s / C::NST) & 1;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_full[slot], par, abort_flag));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_full[slot], par, abort_flag, wl));
     if (!ok) {
       if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
       *abort_flag = 1;
@@ -826,7 +834,7 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
     const float* fin = sm_o;
     if (part == 0) {
       if (!pi_ready) {
-        const bool ok = mbar_wait(bar_pi, 0, abort_flag);
+        const bool ok = mbar_wait(bar_pi, 0, abort_flag, wl);
         if (!ok && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
         if (!ok) *abort_flag = 1;
         pi_ready = true;
@@ -867,14 +875,13 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
         pslot[i] = c < D ? fin[h * D + c] : sm_hm[(c - D) * 8 + h];
       }
       tq_consumer_bar();
+      // An aborted CTA arrives as well (its partial is then unspecified), so
+      // the last arriver always resets the counter for the next launch; an
+      // aborted last arriver writes no output.
       if (ct == 0) {
-        int last = 0;
-        if (!*abort_flag) {
-          unsigned old;
-          asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;\n" : "=r"(old) : "l"(a.counters + row) : "memory");
-          last = old == (unsigned)(expected - 1);
-        }
-        *last_flag = last;
+        unsigned old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;\n" : "=r"(old) : "l"(a.counters + row) : "memory");
+        *last_flag = old == (unsigned)(expected - 1);
       }
       tq_consumer_bar();
       if (*last_flag) {
@@ -909,7 +916,7 @@ __global__ void __launch_bounds__(kTqThreads, 1) tq_decode_kernel(const __grid_c
           pw[i] = pm[i] == -INFINITY ? 0.f : exp2f(pm[i] - hm[h]) * hm[g + h];
         }
         tq_consumer_bar();
-        for (int e = ct; e < g * D; e += kTqConsumers * 32) {
+        for (int e = ct; e < g * D && !*abort_flag; e += kTqConsumers * 32) {
           const int h = e / D, c = e - h * D;
           float acc = 0.f;
           for (int j = 0; j < np; ++j) acc = fmaf(__ldcg(a.ws + (slot_of(j) * g + h) * (D + 2) + c), pw[j * g + h], acc);
