@@ -10,7 +10,7 @@ import pytest
 from scipy import integrate
 
 from oracle import turbo, turbo_cache
-from oracle.numerics import fp16_round
+from oracle.numerics import decode16, fp16_round
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -161,19 +161,93 @@ def test_zero_vector():
     assert np.all(out["codes"] == 3) and out["n"][0] == 0 and out["gamma"][0] == 0
 
 
-def test_codebook_points_round_trip():
-    """A vector whose rotated direction is a codebook point quantizes to that
-    point with a zero residual (gamma = 0 up to float64 rounding)."""
+def test_scaled_codebook_direction_has_closed_form_codes_gamma_and_signs():
+    """x = n Pi^T (c_k / ||c_k||) for a chosen code vector k: the rotated unit
+    vector is the codebook point c_k rescaled, so every coordinate stays in its
+    own cell (each is chosen at least 1e-3 from both thresholds of its cell),
+    the codes come back as k, the residual is e = c_k (1/||c_k|| - 1), gamma =
+    n |1 - ||c_k|||, and the sketch signs are those of (S c_k) (1/||c_k|| - 1).
+    A transposed Pi, a residual taken in the wrong space, a dropped norm or a
+    flipped sign convention each break one of these."""
     pi, s, lv, th = _params()
     rng = np.random.default_rng(4)
-    k = rng.integers(0, 8, (5, 128))
-    yv = lv[k] / np.linalg.norm(lv[k], axis=1, keepdims=True) * np.linalg.norm(lv[k], axis=1, keepdims=True)
+    edges = np.concatenate([[-np.inf], th, [np.inf]])
     n = np.array([0.5, 1.0, 3.0, 10.0, 100.0])
-    x = (yv / np.linalg.norm(yv, axis=1, keepdims=True) * n[:, None]) @ pi
-    out = turbo.quantize(x, pi, lv, th, s)
-    unit = lv[k] / np.linalg.norm(lv[k], axis=1, keepdims=True)
-    # the unit-norm codebook vector's codes are the nearest levels of unit coords
-    assert np.array_equal(out["codes"], turbo.codes_of(unit, th))
+    checked = 0
+    while checked < len(n):
+        k = rng.integers(0, 8, 128)
+        ck = lv[k]
+        norm = np.linalg.norm(ck)
+        y = ck / norm
+        # every coordinate at least 1e-3 inside its cell, away from ties
+        if np.any(y - edges[k] < 1e-3) or np.any(edges[k + 1] - y < 1e-3):
+            continue
+        x = n[checked] * (y @ pi)              # Pi^T y as a row vector
+        out = turbo.quantize(x[None, :], pi, lv, th, s)
+        assert np.array_equal(out["codes"][0], k.astype(np.uint8))
+        assert abs(out["n_exact"][0] - n[checked]) <= 1e-12 * n[checked]
+        gamma = n[checked] * abs(1.0 - norm)
+        assert abs(out["gamma_exact"][0] - gamma) <= 1e-9 * n[checked]
+        e_dir = (s @ ck) * (1.0 / norm - 1.0)
+        clear = np.abs(e_dir) > 1e-9
+        assert np.array_equal(out["signs"][0][clear], (e_dir[clear] >= 0).astype(np.uint8))
+        checked += 1
+
+
+def _turbo_scratch(kb, vb, S0, S, R, G, params):
+    """Closed-form state of a row after a prefill of S0 tokens and S - S0
+    appends: the window flushes G tokens each time it reaches R + G, so the
+    quantized length, window length and ring head follow from the counts, and
+    the quantized tokens are the first tq ones, quantized from scratch."""
+    pi, s, lv, th = params
+    tq0 = G * (max(0, S0 - R) // G)
+    r0 = S0 - tq0
+    n = S - S0
+    flushes = (r0 + n - R) // G if r0 + n >= R + G else 0
+    tq = tq0 + G * flushes
+    head = (G * flushes) % (R + G)
+    k = decode16(kb[:tq], "fp16")
+    v = decode16(vb[:tq], "fp16")
+    return tq, S - tq, head, turbo.quantize(k, pi, lv, th, s), turbo.quantize(v, pi, lv, th)
+
+
+@pytest.mark.parametrize("G,R,steps", [(4, 4, 14), (4, 8, 14), (32, 32, 70), (32, 128, 80)])
+def test_turbo_row_window_bookkeeping_brute_force(G, R, steps):
+    """Every prefill length up to ~R + 2G (and the boundary lengths) followed by
+    every append count up to `steps`, on d = m = 8 (the row model does not
+    depend on d): T_q, r, the ring head and the window tokens equal the closed
+    form, and the quantized tokens equal turbo.quantize applied from scratch to
+    the first T_q tokens."""
+    d = 8
+    rng = np.random.default_rng(7)
+    pi = turbo.rotation(rng.standard_normal((d, d)))
+    s = rng.standard_normal((d, d))
+    lv, th = turbo.deployed_codebook(d)
+    params = (pi, s, lv, th)
+    lens = sorted(set(list(range(0, R + 2 * G + 2, 1 if G == 4 else 7)) +
+                      [R - 1, R, R + 1, R + G - 1, R + G, R + G + 1, 2 * R + G + 5]))
+    for S0 in [x for x in lens if x >= 0]:
+        total = S0 + steps
+        kb = rng.standard_normal((total, d)).astype(np.float16).view(np.uint16)
+        vb = rng.standard_normal((total, d)).astype(np.float16).view(np.uint16)
+        row = turbo_cache.TurboRow(d, R, "fp16", pi, s, lv, th, G=G)
+        row.prefill(kb[:S0], vb[:S0])
+        for n in range(0, steps + 1):
+            if n:
+                row.append(kb[S0 + n - 1], vb[S0 + n - 1])
+            S = S0 + n
+            tq, r, head, kq, vq = _turbo_scratch(kb, vb, S0, S, R, G, params)
+            assert (row.tq, row.r, row.head) == (tq, r, head), (S0, n)
+            if S >= R:
+                assert R <= row.r < R + G
+            idx = (head + np.arange(r)) % (R + G)
+            assert np.array_equal(row.ring_k[idx], kb[tq:S]) and np.array_equal(row.ring_v[idx], vb[tq:S])
+            wk, wv = row.window_bits()
+            assert np.array_equal(wk, kb[tq:S]) and np.array_equal(wv, vb[tq:S])
+            for key in ("codes", "n", "gamma", "signs"):
+                assert np.array_equal(row.kq[key], kq[key]), (S0, n, key)
+            for key in ("codes", "n"):
+                assert np.array_equal(row.vq[key], vq[key]), (S0, n, key)
 
 
 def test_tie_goes_to_lower_index():
