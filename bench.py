@@ -5,17 +5,23 @@ A step is one decode step of the whole batch through kvq_append_decode: the
 new token enters the residual window (a flush quantizes G tokens when due) and
 the attention runs over the packed cache, in one kernel launch on steps that
 do not flush.  Metric: packed-KV bytes read by the decode attention per
-second (GB/s), with tokens/s alongside.
+second (GB/s), with tokens/s alongside.  The default workload is the
+Llama-3.1-70B-shaped 128K-token context at 2 bits.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 8b2] [--impl kivi|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 70b] [--impl kivi|reference]
 
 Timing: the K timed steps are captured into one CUDA graph (library calls
 through the C ABI) and replayed once between CUDA events on the launching
 stream, bracketed by a barrier and torch.cuda.synchronize(); the max over ranks
-is reported.  The e2e figure instead calls the public API step by step with
-host buffers.
-Each step targets the next of several identical cache replicas whose total
-size is over 3x the L2, so every step streams its cache from HBM.
+is reported.  Each step targets the next of several identical cache replicas
+whose total size is over 3x the L2, so every step streams its cache from HBM.
+The decode kernel is also timed launch by launch (at least 100 single-launch
+graph replays, replicas rotated: the cold-L2 median; the same replica again
+and again: the warm-L2 median), and the launch overhead is reported apart:
+the host cost of one library call and the device gap a separately launched
+graph adds.  The e2e figure calls the public API step by step with host
+buffers: one pinned host-to-device copy of the step's inputs and one
+device-to-host copy of its output per step.
 """
 from __future__ import annotations
 
@@ -267,7 +273,10 @@ def run_gpu(args, w, rank, world):
                                               c.ws.numel(), csp), "append_decode")
                 total_bytes += step_bytes(c)
     launches = launch_count() - launches0
-    # attention-only graph over the same replicas, for the per-launch kernel time
+    # attention-only graphs over the same replicas: one graph of K launches
+    # (the mean launch time) and one single-launch graph per replica (launch
+    # by launch medians); attention does not change the cache, so replays are
+    # idempotent
     agraph = torch.cuda.CUDAGraph()
     with torch.cuda.stream(cap_stream):
         with torch.cuda.graph(agraph, stream=cap_stream):
@@ -275,6 +284,15 @@ def run_gpu(args, w, rank, world):
                 c = caches[j % n_rep]
                 L.check(lib.kvq_decode_attention(c.handle, qp[j], outp, scale, ptr(c.ws), c.ws.numel(), csp),
                         "attention")
+    single = []
+    for i in range(n_rep):
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cap_stream):
+            with torch.cuda.graph(g1, stream=cap_stream):
+                c = caches[i]
+                L.check(lib.kvq_decode_attention(c.handle, qp[i], outp, scale, ptr(c.ws), c.ws.numel(), csp),
+                        "attention")
+        single.append(g1)
     attn_bytes = sum(step_bytes(caches[j % n_rep]) for j in range(args.steps))
     torch.cuda.synchronize()
     if world > 1:
@@ -306,19 +324,54 @@ def run_gpu(args, w, rank, world):
     a1.record(stream)
     torch.cuda.synchronize()
     attn_ms = [a0.elapsed_time(a1) / args.steps] * args.steps
-    del graph, agraph
+
+    def per_launch(order):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in order]
+        for (e0, e1), i in zip(ev, order):
+            e0.record(stream)
+            single[i].replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    n_med = max(100, args.steps)
+    cold = per_launch([j % n_rep for j in range(n_med)])
+    warm = per_launch([0] * (n_med + 1))[1:]   # the first launch brings replica 0 into L2
+    # host cost of one library call (argument checks, partition, launch), no graph
+    torch.cuda.synchronize()
+    h0 = time.perf_counter()
+    n_host = 100
+    for j in range(n_host):
+        c = caches[j % n_rep]
+        lib.kvq_decode_attention(c.handle, qp[j % steps_total], outp, scale, ptr(c.ws), c.ws.numel(), sp)
+    host_us = (time.perf_counter() - h0) / n_host * 1e6
+    torch.cuda.synchronize()
+    kernel = {"mean_us": statistics.mean(attn_ms) * 1e3, "median_cold_us": statistics.median(cold) * 1e3,
+              "median_warm_us": statistics.median(warm) * 1e3, "launches_timed": len(cold),
+              "host_call_us": host_us,
+              "graph_launch_gap_us": (statistics.median(cold) - statistics.mean(attn_ms)) * 1e3}
+    del graph, agraph, single
     for c in caches:
         if c.status():
             raise RuntimeError("device status word set during the bench")
     ms, total_bytes = combine_ranks(ms, total_bytes, world, device)
 
-    # end-to-end through the public API with host buffers: H2D of the step's
-    # inputs from pinned memory, append + attention, D2H of the output
-    h_q = q[args.warmup:].cpu().pin_memory()
-    h_kn = kn[args.warmup:].cpu().pin_memory()
-    h_vn = vn[args.warmup:].cpu().pin_memory()
+    # end-to-end through the public API with host buffers: each step's q,
+    # k_new and v_new sit in one pinned host row and cross in one host-to-device
+    # copy; the output comes back in one device-to-host copy
+    nq, nk = q[0].numel(), kn[0].numel()
+    row_elems = nq + 2 * nk
+    h_in = torch.empty((args.steps, row_elems), dtype=q.dtype).pin_memory()
+    for j in range(args.steps):
+        i = args.warmup + j
+        h_in[j, :nq].copy_(q[i].reshape(-1))
+        h_in[j, nq:nq + nk].copy_(kn[i].reshape(-1))
+        h_in[j, nq + nk:].copy_(vn[i].reshape(-1))
     h_out = torch.empty((args.steps,) + tuple(out.shape), dtype=torch.float32).pin_memory()
-    d_q, d_kn, d_vn = torch.empty_like(q[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
+    d_in = torch.empty(row_elems, dtype=q.dtype, device=device)
+    esz = d_in.element_size()
+    d_q, d_kn, d_vn = (ctypes.c_void_p(d_in.data_ptr()), ctypes.c_void_p(d_in.data_ptr() + nq * esz),
+                       ctypes.c_void_p(d_in.data_ptr() + (nq + nk) * esz))
     e_caches = [new_cache() for _ in range(n_rep)]
     K, V, _, _, _ = device_inputs(w, device, 1, rank)
     if turbo:
@@ -336,18 +389,17 @@ def run_gpu(args, w, rank, world):
     prefill_ms = p0.elapsed_time(p1) / n_rep
     prefill_bytes = int(K.numel() * 2 + V.numel() * 2) + step_bytes(e_caches[0])
     del K, V
-    torch.cuda.synchronize()
+    e_args = [(c.handle, ptr(c.ws), c.ws.numel()) for c in e_caches]
     e_bytes = 0
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for j in range(args.steps):
-        c = e_caches[j % n_rep]
-        d_q.copy_(h_q[j], non_blocking=True)
-        d_kn.copy_(h_kn[j], non_blocking=True)
-        d_vn.copy_(h_vn[j], non_blocking=True)
-        c.append_attention(d_kn, d_vn, d_q, out=out)
+        hnd, wsp, wsn = e_args[j % n_rep]
+        d_in.copy_(h_in[j], non_blocking=True)
+        L.check(lib.kvq_append_decode(hnd, d_kn, d_vn, d_q, outp, scale, wsp, wsn, sp), "append_decode")
         h_out[j].copy_(out, non_blocking=True)
-        e_bytes += step_bytes(c)
+        e_bytes += step_bytes(e_caches[j % n_rep])
     e1.record(stream)
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
@@ -355,17 +407,23 @@ def run_gpu(args, w, rank, world):
 
     res = dict(ms=ms, bytes=total_bytes, attn_ms=attn_ms, launches=launches, clocks=clk.summary(),
                e2e_ms=e_ms, e2e_bytes=e_bytes, n_rep=n_rep, splits=caches[0].decode_splits,
-               h2d=int(q[0].numel() * 2 + kn[0].numel() * 2 + vn[0].numel() * 2), d2h=int(out.numel() * 4),
+               h2d=int(row_elems * esz), d2h=int(out.numel() * 4), kernel=kernel,
                step_bytes_last=attn_bytes // args.steps, prefill_ms=prefill_ms, prefill_bytes=prefill_bytes)
     return res
 
 
 # ---------------------------------------------------------------- oracle (CPU) timing
 def oracle_sample(w, budget_s: float, steps: int = 1):
-    """Times the float64 oracle's decode step (append + attention over the
-    dequantized cache) on a bounded sample of (batch, kv-head) rows."""
+    """Times the float64 oracle on a bounded sample of (batch, kv-head) rows:
+    the prefill quantization of each sampled row, then its decode steps
+    (append + attention over the dequantized cache), the latter once with
+    numpy's thread pool as it is and once limited to one thread.  Rows are
+    processed one after another; a step's attention is numpy matrix products,
+    the only part the thread pool spreads over cores."""
+    import copy
+
     import numpy as np
-    from threadpoolctl import threadpool_info
+    from threadpoolctl import threadpool_info, threadpool_limits
     from oracle import attention as oatt
     from oracle import turbo, turbo_cache
     from oracle.cache import KiviRow
@@ -377,23 +435,16 @@ def oracle_sample(w, budget_s: float, steps: int = 1):
                      else turbo.rotation(W.gaussian_matrix(w, "rot", w.head_dim, w.head_dim)),
                      W.gaussian_matrix(w, "qjl", w.qjl_dim, w.head_dim).astype(np.float64),
                      *turbo.deployed_codebook(w.head_dim))
+        rec_bytes = turbo_cache.TB_BYTES
+    else:
+        rec_bytes = w.group * w.head_dim * w.bits // 4 + 4 * w.head_dim + 4 * w.group
 
-    t_total, bytes_total, rows = 0.0, 0, 0
-    g = w.gqa
-    b, h = 0, 0
-    wall0 = time.time()
-    while t_total < budget_s and time.time() - wall0 < 3 * budget_s + 15:
-        k, v = W.prefill_row(w, b, h)
-        if w.scheme == "turbo":
-            row = turbo_cache.TurboRow(w.head_dim, w.residual, w.dtype, *tq_params, G=w.group)
-            rec_bytes = turbo_cache.TB_BYTES
-        else:
-            row = KiviRow(w.head_dim, w.bits, w.group, w.residual, w.dtype)
-            rec_bytes = w.group * w.head_dim * w.bits // 4 + 4 * w.head_dim + 4 * w.group
-        row.prefill(k, v)
+    def decode_steps(row, b, h):
+        """Seconds and packed bytes of `steps` append + attention steps."""
+        t_sum, nbytes = 0.0, 0
         for s in range(1, steps + 1):
             kn, vn = W.decode_token(w, s)
-            q = W.query(w, s)[b, h * g:(h + 1) * g]
+            q = W.query(w, s)[b, h * w.gqa:(h + 1) * w.gqa]
             t = time.perf_counter()
             row.append(kn[b, h], vn[b, h])
             if w.scheme == "turbo":
@@ -401,14 +452,52 @@ def oracle_sample(w, budget_s: float, steps: int = 1):
             else:
                 Kd, Vd = row.dequantized()
                 oatt.attention(decode16(q, w.dtype), Kd, Vd, w.scale)
-            t_total += time.perf_counter() - t
-            bytes_total += (row.tq // w.group) * rec_bytes + row.r * 4 * w.head_dim
+            t_sum += time.perf_counter() - t
+            nbytes += (row.tq // w.group) * rec_bytes + row.r * 4 * w.head_dim
+        return t_sum, nbytes
+
+    acc = dict(pre_s=0.0, pre_bytes=0, multi_s=0.0, multi_bytes=0, single_s=0.0, single_bytes=0)
+    rows = 0
+    b, h = 0, 0
+    wall0 = time.time()
+    while acc["multi_s"] + acc["single_s"] + acc["pre_s"] < budget_s and time.time() - wall0 < 3 * budget_s + 15:
+        k, v = W.prefill_row(w, b, h)
+        if w.scheme == "turbo":
+            row = turbo_cache.TurboRow(w.head_dim, w.residual, w.dtype, *tq_params, G=w.group)
+        else:
+            row = KiviRow(w.head_dim, w.bits, w.group, w.residual, w.dtype)
+        t = time.perf_counter()
+        row.prefill(k, v)
+        acc["pre_s"] += time.perf_counter() - t
+        acc["pre_bytes"] += int(k.nbytes + v.nbytes) + (row.tq // w.group) * rec_bytes + row.r * 4 * w.head_dim
+        single_row = copy.deepcopy(row)
+        ts, nb = decode_steps(row, b, h)
+        acc["multi_s"] += ts
+        acc["multi_bytes"] += nb
+        with threadpool_limits(limits=1):
+            ts, nb = decode_steps(single_row, b, h)
+        acc["single_s"] += ts
+        acc["single_bytes"] += nb
         rows += 1
         h += 1
         if h == w.num_kv_heads:
             h, b = 0, (b + 1) % w.batch
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return dict(value=bytes_total / t_total / 1e9, seconds=t_total, rows=rows, steps=steps, cores=threads)
+    return dict(value=acc["multi_bytes"] / acc["multi_s"] / 1e9, seconds=acc["multi_s"], rows=rows, steps=steps,
+                cores=threads, single_value=acc["single_bytes"] / acc["single_s"] / 1e9,
+                single_seconds=acc["single_s"], prefill_value=acc["pre_bytes"] / acc["pre_s"] / 1e9,
+                prefill_seconds=acc["pre_s"])
+
+
+def cpu_baseline_obj(samp, w):
+    return {"value": round(samp["value"], 4), "unit": "GB/s", "cores": samp["cores"], "kind": "oracle",
+            "sample": f"{samp['rows']} (batch, kv-head) rows of {w.name}, {samp['steps']} append + attention "
+                      f"step(s) each after the row's prefill, {samp['seconds']:.1f} s; rows one after another, "
+                      f"numpy's {samp['cores']}-thread pool in the attention products",
+            "single_thread": {"value": round(samp["single_value"], 4), "unit": "GB/s", "cores": 1,
+                              "seconds": round(samp["single_seconds"], 2)},
+            "prefill_quantize": {"value": round(samp["prefill_value"], 4), "unit": "GB/s (inputs read + "
+                                 "records and window written)", "seconds": round(samp["prefill_seconds"], 2)}}
 
 
 def main():
@@ -416,7 +505,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="8b2")
+    ap.add_argument("--config", default="70b")
     ap.add_argument("--impl", default="kivi", choices=["kivi", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -455,8 +544,7 @@ def main():
                 "ms_per_step": round(full_bytes / (samp["value"] * 1e9) * 1e3, 3),
                 "ms_per_step_kind": "projected: one full step at the sampled rate", "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg_desc,
-                "cpu_baseline": {"value": samp["value"], "unit": "GB/s", "cores": samp["cores"], "kind": "oracle",
-                                 "sample": f"{samp['rows']} (batch, kv-head) rows x {samp['steps']} steps"},
+                "cpu_baseline": cpu_baseline_obj(samp, w),
                 "e2e": {"value": samp["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return
@@ -493,6 +581,7 @@ def main():
                      "bytes_per_launch": res["step_bytes_last"], "mean_launch_us": round(attn_mean * 1e3, 2)},
         "e2e": {"value": round(res["e2e_bytes"] / (res["e2e_ms"] * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+        "kernel_timing": {k: round(v, 2) if isinstance(v, float) else v for k, v in res["kernel"].items()},
         "gpu_launches": res["launches"], "clocks": res["clocks"], "replicas": res["n_rep"],
         "decode_splits": res["splits"],
         # secondary: the prefill (quantize kernel + window copy) of one replica,
@@ -503,10 +592,7 @@ def main():
                     "kernel": "tq_quantize_kernel" if w.scheme == "turbo" else "kivi_quantize_kernel"},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        samp = oracle_sample(w, args.cpu_budget)
-        line["cpu_baseline"] = {"value": round(samp["value"], 4), "unit": "GB/s", "cores": samp["cores"],
-                                "kind": "oracle", "sample": f"{samp['rows']} (batch, kv-head) rows of {w.name}, "
-                                                            f"one append + attention each, {samp['seconds']:.1f} s"}
+        line["cpu_baseline"] = cpu_baseline_obj(oracle_sample(w, args.cpu_budget), w)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:

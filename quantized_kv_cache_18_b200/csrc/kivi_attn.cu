@@ -76,7 +76,11 @@ struct K {
   // then o[NC][HS][D]
   static constexpr int SO = (2 * NC * HS + 1 + 3) / 4 * 4;
   static constexpr int SBUF_F = SO + NC * HS * D;
-  static constexpr int FIXED = 2 * SBUF_F * 4 + (TR ? NC * 512 : 0) + 2 * 8 * D * 2 + 8 * 8 + 16;
+  // warp-state buffers: two let the merge warp merge one segment while the
+  // consumers fill the next; the hybrid formulation's 8-head states are twice
+  // as large, so it keeps one and spends the room on a deeper stage ring
+  static constexpr int NSB = TR ? 2 : 1;
+  static constexpr int FIXED = NSB * SBUF_F * 4 + (TR ? NC * 512 : 0) + 2 * 8 * D * 2 + 8 * 8 + 16;
   static constexpr int NST_FIT = (227 * 1024 - FIXED) / (STAGE + SG * 8 * 4 + 3 * 8);
   static constexpr int NST = (STAGE > 48 * 1024 ? 3 : 4) < NST_FIT ? (STAGE > 48 * 1024 ? 3 : 4) : NST_FIT;
   static constexpr int KSOFF = G * D * BITS / 4;
@@ -85,7 +89,7 @@ struct K {
   // shared memory map (bytes)
   static constexpr int OFF_BETA = NST * STAGE;
   static constexpr int OFF_S = OFF_BETA + NST * SG * 8 * 4;      // two warp-state buffers
-  static constexpr int OFF_PW = OFF_S + 2 * SBUF_F * 4;          // per-warp P tile (TR): 32 tokens x 8 fp16
+  static constexpr int OFF_PW = OFF_S + NSB * SBUF_F * 4;        // per-warp P tile (TR): 32 tokens x 8 fp16
   static constexpr int OFF_Q = OFF_PW + (TR ? NC * 512 : 0);     // q ring: 2 slots x raw 16-bit q of 8 heads
   static constexpr int OFF_BAR = OFF_Q + 2 * 8 * D * 2;
   static constexpr int OFF_FLAG = OFF_BAR + (3 * NST + 9) * 8;
@@ -147,12 +151,11 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
   constexpr int P = D * BITS / 32;
   constexpr int J = BITS == 2 ? 4 : 2;
   constexpr int NKT = D / 16;
-  constexpr int NNT = D / 8;
   constexpr int WPN = P / 4;
 
   extern __shared__ __align__(128) unsigned char smem[];
   float* sm_beta = reinterpret_cast<float*>(smem + C::OFF_BETA);
-  float* sm_state = reinterpret_cast<float*>(smem + C::OFF_S);   // [2][SBUF_F]
+  float* sm_state = reinterpret_cast<float*>(smem + C::OFF_S);   // [NSB][SBUF_F]
   uint16_t* sm_q = reinterpret_cast<uint16_t*>(smem + C::OFF_Q);
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_ready = bar_full + C::NST;
@@ -397,8 +400,8 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
     for_each_chunk<C::SG>(
         Pt, i0, i1, [](int, int, bool, int64_t, int) {}, nop_seg,
         [&](int row) {
-          const int sbi = k & 1;
-          const uint32_t par = (k >> 1) & 1;
+          const int sbi = k % C::NSB;
+          const uint32_t par = (k / C::NSB) & 1;
           ++k;
           if (row == last_row) return;   // the consumer warps merge the CTA's last segment
           const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[sbi], par, abort_flag, wl));
@@ -864,9 +867,8 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
       }
     }
   };
-  auto hx_block = [&](const unsigned char* st, int slot) {
-    const int grp = cw / C::NTB, tbg = cw - grp * C::NTB;
-    const unsigned char* rec = st + grp * C::REC;
+  // scores of one block (log2 domain, zero-point term included) -> x
+  auto hx_qk = [&](const unsigned char* rec, int tbg, int slot, int grp, float (&x)[4][2]) {
     uint4 kc[P / 4];
 #pragma unroll
     for (int p = 0; p < P / 4; ++p) kc[p] = lds128(rec + tbg * C::TBC + 16 * (32 * p + lane));
@@ -900,15 +902,16 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
           for (int nt = 0; nt < 4; ++nt) mma_f16_16816(sc[nt], aq, pr[nt][2 * m2], pr[nt][2 * m2 + 1]);
         }
       }
-    float x[4][2];
-    float mx = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        x[nt][e] = fmaf(sc[nt][e] + sc[nt][2 + e], a.scale_log2, bs);
-        mx = fmaxf(mx, x[nt][e]);
-      }
+      for (int e = 0; e < 2; ++e) x[nt][e] = fmaf(sc[nt][e] + sc[nt][2 + e], a.scale_log2, bs);
+  };
+  // online softmax and P.V of a block whose scores are x (record rec, token block tbg)
+  auto hx_finish = [&](const unsigned char* rec, int tbg, const float (&x)[4][2]) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) mx = fmaxf(mx, fmaxf(x[nt][0], x[nt][1]));
     hx_rescale(quad_max(mx));
     uint32_t vm[8];
     {
@@ -1089,9 +1092,14 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
     if constexpr (TR) {
       if (ok && !win && cw < cnt * C::NTB) tr_block(st, slot);
       else if (ok && win) tr_window(st, first);
-    } else {
-      if (ok && !win && cw < cnt * C::NTB) hx_block(st, slot);
-      else if (ok && win) hx_window(st, first);
+    } else if (ok && !win && cw < cnt * C::NTB) {
+      const int grp = cw / C::NTB, tbg = cw - grp * C::NTB;
+      const unsigned char* rec = st + grp * C::REC;
+      float x[4][2];
+      hx_qk(rec, tbg, slot, grp, x);
+      hx_finish(rec, tbg, x);
+    } else if (ok && win) {
+      hx_window(st, first);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar_empty[slot]);
@@ -1100,12 +1108,12 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
   int final_row = -1;
   float* final_sb = nullptr;
   auto seg_end = [&](int row) {
-    // warp state -> state buffer k & 1, once the merge warp is done with segment k - 2
+    // warp state -> state buffer k % NSB, once the merge warp is done with segment k - NSB
     const int k = qseg - 1;
-    const int sbi = k & 1;
+    const int sbi = k % C::NSB;
     float* sb = sm_state + sbi * C::SBUF_F;
-    if (k >= 2) {
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfree[sbi], ((k >> 1) - 1) & 1, abort_flag, wl));
+    if (k >= C::NSB) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfree[sbi], ((k / C::NSB) - 1) & 1, abort_flag, wl));
       if (!ok) {
         if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
         *abort_flag = 1;

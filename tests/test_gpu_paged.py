@@ -1,11 +1,15 @@
 """Paged caches (a pool of record pages and a per-row block table) against
-contiguous caches of the same workload.
+contiguous caches of the same workload and against the float64 oracle.
 
 Same inputs, same calls: a paged cache must hold bit-identical records (read
 through its block table) and window, and return bit-identical attention.  The
 block tables are random permutations of the pool, so no row's pages are
-adjacent or in order.  A table entry outside the pool must raise
-KVQ_DEV_BAD_PAGE and be skipped, never dereferenced."""
+adjacent or in order.  After the prefill, at the first step that flushes the
+window and at the last step, every row of the paged cache is also checked
+against the oracle: records and window bit-exact (TurboQuant blocks under the
+ambiguity rule of test_gpu_turbo) and attention within max-abs 2e-3 and rel-L2
+1e-3.  A table entry outside the pool must raise KVQ_DEV_BAD_PAGE and be
+skipped, never dereferenced."""
 import ctypes
 import math
 
@@ -13,7 +17,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import to_dev
+from gpu_util import check_row_attention, oracle_row, to_dev
 from quantized_kv_cache_18_b200 import _lib as L
 from quantized_kv_cache_18_b200 import workloads as W
 from quantized_kv_cache_18_b200.cache import QuantizedKVCache, config_from_workload, turbo_setup_from_workload
@@ -54,6 +58,67 @@ def _same(paged, flat, w):
     assert torch.equal(paged.ring_view()[:, :, idx], flat.ring_view()[:, :, idx])
 
 
+class _OracleRows:
+    """The oracle's rows of a workload, advanced with the same appends, and the
+    paged cache's records and window checked against them."""
+
+    def __init__(self, w, K, V):
+        self.w = w
+        self.rows = [(b, h) for b in range(w.batch) for h in range(w.num_kv_heads)]
+        if w.scheme == "turbo":
+            from test_gpu_turbo import oracle_params
+            from test_gpu_turbo import oracle_row as tq_row
+            self.params = oracle_params(w)
+            self.o = {bh: tq_row(w, self.params, K[bh[0], bh[1]], V[bh[0], bh[1]]) for bh in self.rows}
+            self.toks = {bh: ([K[bh[0], bh[1]]], [V[bh[0], bh[1]]]) for bh in self.rows}
+        else:
+            self.o = {bh: oracle_row(w, K[bh[0], bh[1]], V[bh[0], bh[1]]) for bh in self.rows}
+
+    def append(self, kn, vn):
+        for (b, h), row in self.o.items():
+            row.append(kn[b, h], vn[b, h])
+            if self.w.scheme == "turbo":
+                self.toks[(b, h)][0].append(kn[b, h][None])
+                self.toks[(b, h)][1].append(vn[b, h][None])
+
+    def check_state(self, cache):
+        """Records (through the block table) and window of every row; returns
+        the number of TurboQuant keys whose codes took the other neighbour."""
+        w = self.w
+        any_row = next(iter(self.o.values()))
+        assert (cache.quantized_len, cache.window_len, cache.window_head) == (any_row.tq, any_row.r, any_row.head)
+        n = any_row.tq // _unit(w)
+        ring = cache.ring_view().cpu().numpy().view(np.uint16)
+        flips = 0
+        for (b, h), row in self.o.items():
+            ri = b * w.num_kv_heads + h
+            if n:
+                got = cache.row_records(ri, n).cpu().numpy()
+                if w.scheme == "turbo":
+                    from test_gpu_turbo import check_blocks
+                    kall = np.concatenate(self.toks[(b, h)][0])[:row.tq]
+                    vall = np.concatenate(self.toks[(b, h)][1])[:row.tq]
+                    flips += check_blocks(got, w, self.params, kall, vall)[1]
+                else:
+                    assert np.array_equal(got, row.records()), f"row {ri}: records differ from the oracle"
+            idx = (row.head + np.arange(row.r)) % row.cap
+            assert np.array_equal(ring[ri, 0][idx], row.ring_k[idx]), f"row {ri}: key window differs"
+            assert np.array_equal(ring[ri, 1][idx], row.ring_v[idx]), f"row {ri}: value window differs"
+        return flips
+
+    def check_attention(self, out, q, flips):
+        w, g = self.w, self.w.gqa
+        out = out.cpu().numpy()
+        for (b, h), row in self.o.items():
+            got = out[b, h * g:(h + 1) * g]
+            if w.scheme == "turbo":
+                if flips == 0:   # same codes on both sides
+                    from test_gpu_turbo import check_attention
+                    check_attention(got, row.attention(q[b, h * g:(h + 1) * g], w.scale))
+            else:
+                check_row_attention(got, row, q[b, h * g:(h + 1) * g], w)
+
+
 @pytest.mark.parametrize("name,kw,S,steps,page_records", [
     ("tiny", dict(), 300, 70, 1),                     # one group per page; flushes
     ("8b2", dict(batch=2), 1500, 40, 4),              # token-major kernel; a stage spans pages
@@ -73,14 +138,27 @@ def test_paged_cache_matches_contiguous(name, kw, S, steps, page_records):
             turbo_setup_from_workload(c, w)
         c.prefill(to_dev(K), to_dev(V))
     _same(paged, flat, w)
+    orc = _OracleRows(w, K, V)
+    flips = orc.check_state(paged)
+    q0 = W.query(w, 0)
+    orc.check_attention(paged.attention(to_dev(q0)), q0, flips)
+    first_flush = None
     for i in range(1, steps + 1):
         kn, vn = W.decode_token(w, i)
-        qd = to_dev(W.query(w, i))
+        q = W.query(w, i)
+        qd = to_dev(q)
         kd, vd = to_dev(kn), to_dev(vn)
+        tq_before = paged.quantized_len
         out_p = paged.append_attention(kd, vd, qd)
         out_f = flat.append_attention(kd, vd, qd)
+        orc.append(kn, vn)
         torch.cuda.synchronize()
         assert torch.equal(out_p, out_f), f"step {i}: outputs differ"
+        flushed = paged.quantized_len != tq_before
+        if (flushed and first_flush is None) or i == steps:
+            first_flush = first_flush or (i if flushed else None)
+            orc.check_attention(out_p, q, orc.check_state(paged))
+    assert first_flush is not None, "the case must cross a flush"
     _same(paged, flat, w)
     assert paged.status() == 0 and flat.status() == 0
 

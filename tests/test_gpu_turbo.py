@@ -11,9 +11,18 @@ boundary that covers the GPU's rounding error:
   * a token with a code that took the other neighbour has a different
     residual e, so its gamma and signs are not compared (only counted);
   * sign bit: |(S e)_i| < EPS_SE;
-  * fp16 n or gamma: exact value within a relative 1e-5 of an fp16 rounding
-    midpoint.
-The fraction of ambiguous decisions must stay under 0.5 %.  Attention is
+  * fp16 n: both sides compute the norm in fp64 from the 16-bit inputs
+    (relative error below 128 * 2^-53, about 1.4e-14), so n must be
+    bit-exact unless the exact norm lies within EPS_N = 1e-12 (relative) of
+    an fp16 rounding midpoint;
+  * fp16 gamma = n ||y - c_hat||: the GPU's y has an error below EPS_Y per
+    coordinate, so ||e|| is off by at most sqrt(d) EPS_Y (triangle
+    inequality); a gamma may differ from the oracle's only as the other fp16
+    neighbour of the exact value, when the exact value lies within
+    n sqrt(d) EPS_Y of the midpoint between the two.
+Every code and sign inside its window, and every norm or gamma that actually
+differs, counts as ambiguous; the ambiguous fraction of all these decisions
+must stay under 0.5 %.  Attention is
 compared on a cache whose packed blocks are the oracle's own (written into the
 buffer), so both sides read the same codes, within max-abs 2e-3 and rel-L2
 1e-3; with no code decided differently the GPU's own cache is compared too.
@@ -36,7 +45,7 @@ pytestmark = pytest.mark.gpu
 
 EPS_Y = 1e-5
 EPS_SE = 1e-4
-EPS_MID = 1e-5
+EPS_N = 1e-12
 
 TQ = W.WORKLOADS["tq"]
 SMALL = W.with_sizes(TQ, batch=1, num_kv_heads=2, num_q_heads=8, seq_len=480, decode_steps=72)
@@ -64,15 +73,22 @@ def oracle_row(w, params, kb, vb):
     return row
 
 
-def _near_fp16_midpoint(x):
-    """True where float64 x lies within EPS_MID (relative) of a midpoint between
-    two adjacent fp16 values."""
+def _near_fp16_midpoint(x, tol):
+    """True where float64 x lies within `tol` (absolute, scalar or per value)
+    of a midpoint between two adjacent fp16 values."""
     x = np.abs(np.asarray(x, np.float64))
     h = x.astype(np.float16).astype(np.float64)
     nxt = np.nextafter(h.astype(np.float16), np.float16(np.inf)).astype(np.float64)
     prv = np.nextafter(h.astype(np.float16), np.float16(0)).astype(np.float64)
     mids = np.stack([0.5 * (h + nxt), 0.5 * (h + prv)])
-    return np.any(np.abs(mids - x) <= EPS_MID * np.maximum(x, 1e-30), axis=0)
+    return np.any(np.abs(mids - x) <= tol, axis=0)
+
+
+def _fp16_neighbours(a, b):
+    """True where fp16 values a and b (float64 arrays) are equal or adjacent."""
+    ua = np.abs(fp16_bits(a).astype(np.int64))
+    ub = np.abs(fp16_bits(b).astype(np.int64))
+    return np.abs(ua - ub) <= 1
 
 
 def check_blocks(got_rec, w, params, k_bits, v_bits):
@@ -103,11 +119,17 @@ def check_blocks_values(got_rec, w, params, k, v):
     # norms: fp16 of an fp64 norm on both sides
     for got, q in ((kn, kq), (vn, vq)):
         bad = fp16_bits(got) != fp16_bits(q["n"])
-        assert not np.any(bad & ~_near_fp16_midpoint(q["n_exact"])), "norm differs"
+        assert not np.any(bad & ~_near_fp16_midpoint(q["n_exact"], EPS_N * q["n_exact"])), "norm differs"
+        n_amb += int(bad.sum())
+        n_dec += bad.size
     # gamma and signs of the tokens whose key codes all agree
     ok = ~flipped_tok
     badg = (fp16_bits(kg) != fp16_bits(kq["gamma"])) & ok
-    assert not np.any(badg & ~_near_fp16_midpoint(kq["gamma_exact"])), "gamma differs"
+    g_tol = kq["n_exact"] * math.sqrt(w.head_dim) * EPS_Y
+    assert not np.any(badg & ~(_near_fp16_midpoint(kq["gamma_exact"], g_tol) &
+                               _fp16_neighbours(kg, kq["gamma"]))), "gamma differs"
+    n_amb += int(badg.sum())
+    n_dec += int(ok.sum())
     amb_s = np.abs(kq["se"]) < EPS_SE
     bads = (ks != kq["signs"]) & ok[:, None]
     assert not np.any(bads & ~amb_s), f"{int(np.sum(bads & ~amb_s))} sign bits differ away from 0"
