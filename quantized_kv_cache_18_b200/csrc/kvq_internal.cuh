@@ -97,7 +97,8 @@ constexpr int kTqLevels = kTqST + kTqD * kTqM * 4; // float [8] codebook levels
 constexpr int kTqThr = kTqLevels + 32;             // float [8] thresholds (7 used, [7] = +inf)
 constexpr int kTqLevels16 = kTqThr + 32;           // fp16 [8] levels
 constexpr int kTqLut = kTqLevels + 128;            // uint32 [64]: fp16x2 (level[lo], level[hi]) of index lo + 8 hi
-constexpr int kTqParamBytes = kTqLut + 256;
+constexpr int kTqSPiT = kTqLut + 256;              // float [d][m], transpose of S Pi (the sketch of a rotated query)
+constexpr int kTqParamBytes = kTqSPiT + kTqD * kTqM * 4;
 constexpr int kTqQPrepBytes = 2 * (kTqD / 16) * 32 * 16;   // rotated query fragments of one row
 
 __host__ __device__ inline int64_t rec_kscale_off(const Geom& g) { return (int64_t)g.G * g.d * g.bits / 4; }

@@ -13,9 +13,10 @@
 //
 // turbo_setup_kernel   one CTA: Householder QR in fp64 in shared memory, the
 //                      Lloyd-Max fixed point in fp64, then the fp32 tables.
-// tq_query_prep_kernel one CTA per (batch, kv head): q' = Pi q and q'' = S q'
-//                      for the row's query heads, split into fp16 hi + lo and
-//                      stored in the A-fragment order of the decode kernel.
+// tq_query_prep_kernel four CTAs per (batch, kv head): q' = Pi q and
+//                      q'' = (S Pi) q for the row's query heads, split into
+//                      fp16 hi + lo and stored in the A-fragment order of the
+//                      decode kernel.
 #include <cuda_runtime.h>
 
 #include "kvq_internal.cuh"
@@ -187,13 +188,33 @@ __global__ void __launch_bounds__(kSetupThreads, 1)
     const uint16_t h_hi2 = __shfl_sync(0xffffffffu, __half_as_ushort(h), 4 + ((lane >> 3) & 3));
     lut[32 + lane] = (uint32_t)h_lo | ((uint32_t)h_hi2 << 16);
   }
+  // ---------------------------------------------------------------- (S Pi)^T, fp64 sums of the fp32 tables
+  // q'' = S Pi q is then one product with q, like q' = Pi q
+  __syncthreads();   // Pi and S^T are in the parameter block
+  {
+    const float* PiG = reinterpret_cast<const float*>(params + kTqPi);
+    float* SPiT = reinterpret_cast<float*>(params + kTqSPiT);
+    for (int e = tid; e < D * M; e += kSetupThreads) {
+      const int j = e / M, i = e - j * M;   // SPiT[j][i] = sum_k S[i][k] Pi[k][j]
+      double acc = 0.0;
+      for (int k = 0; k < D; ++k) acc += (double)ST[k * M + i] * (double)PiG[k * D + j];
+      SPiT[e] = (float)acc;
+    }
+  }
   if (flags) atomicOr(&s_flags, flags);
   __syncthreads();
   if (tid == 0 && s_flags) atomicOr(status, s_flags);
 }
 
 // ---------------------------------------------------------------- query rotation
+// q' = Pi q and q'' = (S Pi) q of every query head of a row, split into fp16
+// hi + lo in the A-fragment order of the decode kernel.  The 256 outputs of a
+// head (128 of q', 128 of q'') are cut into four quarters, one CTA each, so a
+// row takes four CTAs and each stages only its 64 columns of Pi^T or (S Pi)^T
+// (32 KB): every output is one 128-term fp32 dot product, no product waits
+// for another.
 constexpr int kPrepThreads = 256;
+constexpr int kPrepCols = 64;   // outputs per CTA
 
 __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
   return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
@@ -201,79 +222,64 @@ __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
 
 __global__ void __launch_bounds__(kPrepThreads)
     tq_query_prep_kernel(Geom gm, const uint16_t* __restrict__ q, unsigned char* __restrict__ qprep) {
-  constexpr int D = kTqD, M = kTqM;
-  extern __shared__ __align__(16) float sW[];   // [D][D]: Pi^T, then S^T
-  __shared__ float qf[8][D];    // raw q of the row's heads
-  __shared__ float qr[8][D];    // Pi q
-  __shared__ float qs[8][M];    // S Pi q
-  const int row = blockIdx.x;
+  constexpr int D = kTqD;
+  __shared__ __align__(16) float sW[D][kPrepCols];   // column slice of Pi^T or (S Pi)^T
+  __shared__ float qf[8][D];                          // raw q of the row's heads
+  __shared__ float y[8][kPrepCols + 1];               // this quarter of Pi q or S Pi q
+  const int row = blockIdx.x, k = blockIdx.y;         // quarter k: outputs 64 k .. 64 k + 63 of [q' | q'']
   const int b = row / gm.Hkv, hkv = row - b * gm.Hkv;
   const int g = gm.g;
   const int tid = threadIdx.x;
+  const int vec = k >> 1, c0 = kPrepCols * (k & 1);
+  const float* W = reinterpret_cast<const float*>(gm.params + (vec == 0 ? kTqPiT : kTqSPiT));
+  // the slice is requested at once (8 x 16-byte loads per thread)
+  uint4 v[D * kPrepCols / 4 / kPrepThreads];
+#pragma unroll
+  for (int u = 0; u < D * kPrepCols / 4 / kPrepThreads; ++u) {
+    const int e = tid + u * kPrepThreads;   // float4 index in the slice: row e / 16, column 4 (e % 16)
+    v[u] = __ldg(reinterpret_cast<const uint4*>(W + (e >> 4) * D + c0) + (e & 15));
+  }
   const uint16_t* qrow = q + ((int64_t)b * gm.Hq + (int64_t)hkv * g) * D;
-  // the whole matrix is requested at once (16 x 16-byte loads per thread), so
-  // its latency is paid once rather than once per row of the product
-  auto stage = [&](int off) {
-    const uint4* src = reinterpret_cast<const uint4*>(gm.params + off);
-    uint4 v[D * D / 4 / kPrepThreads];
-#pragma unroll
-    for (int k = 0; k < D * D / 4 / kPrepThreads; ++k) v[k] = __ldg(src + tid + k * kPrepThreads);
-#pragma unroll
-    for (int k = 0; k < D * D / 4 / kPrepThreads; ++k) reinterpret_cast<uint4*>(sW)[tid + k * kPrepThreads] = v[k];
-  };
-  stage(kTqPiT);
   for (int e = tid; e < 8 * D; e += kPrepThreads) {
     const int h = e / D;
     qf[h][e - h * D] = h < g ? in16_to_float(qrow[e], gm.dtype) : 0.f;
   }
-  __syncthreads();
-  const int i = tid & (D - 1), h0 = tid / D;   // two head slots per column
-  {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int j = 0; j < D; ++j) {
-      const float w = sW[j * D + i];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] = fmaf(w, qf[h0 + 2 * u][j], acc[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) qr[h0 + 2 * u][i] = acc[u];
+  for (int u = 0; u < D * kPrepCols / 4 / kPrepThreads; ++u) {
+    const int e = tid + u * kPrepThreads;
+    reinterpret_cast<uint4*>(&sW[e >> 4][0])[e & 15] = v[u];
   }
   __syncthreads();
-  stage(kTqST);
-  __syncthreads();
   {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int i = tid & (kPrepCols - 1), h0 = tid / kPrepCols;   // heads h0 and h0 + 4
+    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll 8
     for (int j = 0; j < D; ++j) {
-      const float w = sW[j * M + i];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] = fmaf(w, qr[h0 + 2 * u][j], acc[u]);
+      const float w = sW[j][i];
+      acc0 = fmaf(w, qf[h0][j], acc0);
+      acc1 = fmaf(w, qf[h0 + 4][j], acc1);
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) qs[h0 + 2 * u][i] = acc[u];
+    y[h0][i] = acc0;
+    y[h0 + 4][i] = acc1;
   }
   __syncthreads();
   // fragments: [vector (q', q'')][kt][lane] uint4 =
-  //   {hi(gr, c0..c0+1), lo(gr, c0..c0+1), hi(gr, c0+8..c0+9), lo(gr, c0+8..c0+9)}, c0 = 16 kt + 2 tc
-  uint4* out = reinterpret_cast<uint4*>(qprep + (int64_t)row * kTqQPrepBytes);
-  for (int e = tid; e < 2 * (D / 16) * 32; e += kPrepThreads) {
-    const int vec = e / ((D / 16) * 32);
-    const int kt = (e / 32) % (D / 16);
-    const int lane = e & 31;
+  //   {hi(gr, c..c+1), lo(gr, c..c+1), hi(gr, c+8..c+9), lo(gr, c+8..c+9)}, c = 16 kt + 2 tc
+  if (tid < 4 * 32) {
+    const int ktl = tid >> 5, lane = tid & 31, kt = (c0 >> 4) + ktl;
     const int gr = lane >> 2, tc = lane & 3;
-    const float* src = vec == 0 ? qr[gr] : qs[gr];
     uint32_t w[4];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      const int c = 16 * kt + 8 * half + 2 * tc;
-      const float x0 = src[c], x1 = src[c + 1];
+      const int c = 16 * ktl + 8 * half + 2 * tc;   // column of this quarter
+      const float x0 = y[gr][c], x1 = y[gr][c + 1];
       const __half h0v = __float2half_rn(x0), h1v = __float2half_rn(x1);
       const __half l0 = __float2half_rn(x0 - __half2float(h0v)), l1 = __float2half_rn(x1 - __half2float(h1v));
       w[2 * half] = pack_h2(h0v, h1v);
       w[2 * half + 1] = pack_h2(l0, l1);
     }
-    out[e] = make_uint4(w[0], w[1], w[2], w[3]);
+    uint4* out = reinterpret_cast<uint4*>(qprep + (int64_t)row * kTqQPrepBytes);
+    out[(vec * (D / 16) + kt) * 32 + lane] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -291,13 +297,7 @@ void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_
 }
 
 void launch_tq_query_prep(const Geom& g, const uint16_t* q, unsigned char* qprep, cudaStream_t st) {
-  const int smem = kTqD * kTqD * (int)sizeof(float);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(tq_query_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    attr_set = true;
-  }
-  tq_query_prep_kernel<<<g.B * g.Hkv, kPrepThreads, smem, st>>>(g, q, qprep);
+  tq_query_prep_kernel<<<dim3(g.B * g.Hkv, 4), kPrepThreads, 0, st>>>(g, q, qprep);
   count_launch(1);
 }
 

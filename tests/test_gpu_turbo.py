@@ -236,6 +236,9 @@ def test_setup_tables_match_the_oracle():
     idx = np.arange(64)
     want = fp16_bits(lv)[idx & 7].astype(np.uint32) | (fp16_bits(lv)[idx >> 3].astype(np.uint32) << 16)
     assert np.array_equal(lut, want)
+    # (S Pi)^T: fp64 sums of the fp32 tables, then fp32 -- within a few fp32 ulps of the oracle's S Pi
+    spit = p[off + 384:off + 384 + d * d * 4].view(np.float32).reshape(d, d)
+    assert np.abs(spit.T.astype(np.float64) - S @ Pi).max() < 2e-5
 
 
 # ------------------------------------------------------------------ Walsh-Hadamard rotation

@@ -62,6 +62,38 @@ def test_static_entry_point_matches_workspace_entry_point(name, kw, S):
     assert cache.status() == 0
 
 
+def test_static_entry_point_on_a_turboquant_cache():
+    """The TurboQuant workspace is the rotated-query prefix followed by the
+    partial slots; the static array holds both.  Two calls in a row against
+    kvq_decode_attention and against the float64 oracle over the same codes."""
+    from test_gpu_turbo import SMALL, check_attention, gpu_cache, oracle_params
+    from test_gpu_turbo import oracle_row as tq_row
+    w = W.with_sizes(SMALL, batch=3, num_kv_heads=2, num_q_heads=8, seq_len=1500)
+    params = oracle_params(w)
+    K, V = W.prefill(w, seq_len=1500)
+    cache = gpu_cache(w)
+    cache.prefill(to_dev(K), to_dev(V))
+    assert workspace_bytes(cache.cfg) <= 4 * 1024 * 1024
+    rows = {(b, h): tq_row(w, params, K[b, h], V[b, h]) for b in range(w.batch) for h in range(w.num_kv_heads)}
+    n_tb = cache.quantized_len // 32
+    rec = cache.records_view()
+    for (b, h), row in rows.items():   # the oracle's blocks, so both sides read the same codes
+        rec[b * w.num_kv_heads + h, :n_tb].copy_(torch.from_numpy(row.records()))
+    qh = W.query(w, 2)
+    q = to_dev(qh)
+    ref = cache.attention(q)
+    g = w.gqa
+    for _ in range(2):
+        out = torch.full_like(ref, float("nan"))
+        assert _static_call(cache, q, out) == L.KVQ_OK
+        torch.cuda.synchronize()
+        _agree(out, ref)
+        o = out.cpu().numpy()
+        for (b, h), row in rows.items():
+            check_attention(o[b, h * g:(h + 1) * g], row.attention(qh[b, h * g:(h + 1) * g], w.scale))
+    assert cache.status() == 0
+
+
 def test_static_entry_point_rejects_configs_over_the_limit():
     # (rows + SMs) * g * (d + 4) * 4 bytes of scratch > 4 MiB for 2048 rows of GQA 4, d 128
     cfg = make_config("kivi", 2, 32, 32, 128, 8, 32, 256, 64, "bf16")
