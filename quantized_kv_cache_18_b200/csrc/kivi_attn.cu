@@ -54,6 +54,28 @@ namespace {
 
 constexpr int kWinTok = kDecodeWinTok;                     // tokens per window item
 
+// Code operands as fp16 subnormals: (x & field) is the fp16 bit pattern of
+// code * 2^(b j') * 2^-24 (exponent field zero), one LOP3 per pair instead of
+// LOP3 + HSUB2.  The mma.sync products of such operands keep about 2^-17 of
+// the sum of |products| (measured against exact sums; normal operands keep
+// about 2^-21), well inside the attention tolerance.  The 2^24 goes back in
+// fp32: into the score scale, and into the output at the end of a segment.
+constexpr float kSubScale = 16777216.f;   // 2^24
+template <int BITS, int JP>
+__device__ __forceinline__ uint32_t code_pair(uint32_t x) {
+  constexpr uint32_t M = (BITS == 2 ? 0x00030003u : 0x000F000Fu) << (BITS * JP);
+  return x & M;
+}
+template <int BITS>
+__device__ __forceinline__ void code_half(uint32_t x, uint32_t* out) {
+  out[0] = code_pair<BITS, 0>(x);
+  out[1] = code_pair<BITS, 1>(x);
+  if (BITS == 2) {
+    out[2] = code_pair<BITS, 2>(x);
+    out[3] = code_pair<BITS, 3>(x);
+  }
+}
+
 template <int NC>
 __device__ __forceinline__ void consumer_bar() { named_bar_sync<NC * 32>(); }
 
@@ -581,7 +603,6 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
   // the q~ operand is the hi (even gr) or lo (odd gr) part of head gr >> 1.
   const int qhead = TR ? gr >> 1 : gr;
   const bool head_ok = qhead < gm.g;
-  const uint32_t magic = kMagic;
   int qseg = 0;
   const uint16_t* sq = sm_q;   // ring slot of the current segment
   uint32_t qh[NKT][2];   // q of head qhead at channels 16kt + 8rho + 2tc + {0, 1}, fp16x2
@@ -593,6 +614,23 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
   float o[NO][4];
   float m = -INFINITY, l = 0.f, wz = 0.f;
   int seg_row = 0;
+  // The code contractions accumulate 2^-24 of their value (subnormal code
+  // operands); o_sub: o is still on that scale (the segment's window chunks,
+  // which come after its quantized blocks, bring it to 1 first).
+  const float sl_code = a.scale_log2 * kSubScale;
+  bool o_sub = true;
+  auto o_to_unit = [&]() {
+    if (o_sub) {
+#pragma unroll
+      for (int i = 0; i < NO; ++i) {
+        o[i][0] *= kSubScale;
+        o[i][1] *= kSubScale;
+        o[i][2] *= kSubScale;
+        o[i][3] *= kSubScale;
+      }
+      o_sub = false;
+    }
+  };
 
   auto seg_begin = [&](int row) {
     seg_row = row;
@@ -620,6 +658,7 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
       }
 #pragma unroll
     for (int i = 0; i < NO; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    o_sub = true;
     m = -INFINITY;
     l = 0.f;
     wz = 0.f;
@@ -684,7 +723,7 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
           const int w = nt * WPN + wi;
           const uint4 pc = kc[w >> 2];
           const uint32_t word = (w & 3) == 0 ? pc.x : (w & 3) == 1 ? pc.y : (w & 3) == 2 ? pc.z : pc.w;
-          unpack_half<BITS>(half ? word >> 8 : word, pr[nt], magic);
+          code_half<BITS>(half ? word >> 8 : word, pr[nt]);
         }
 #pragma unroll
         for (int m2 = 0; m2 < J / 2; ++m2) {
@@ -711,7 +750,7 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
       for (int e2 = 0; e2 < 2; ++e2) {
         const int i = 2 * mt + e2;
         x[i] = fmaf((sc[0][mt][2 * e2] + sc[1][mt][2 * e2]) + (sc[0][mt][2 * e2 + 1] + sc[1][mt][2 * e2 + 1]),
-                    a.scale_log2, bs);
+                    sl_code, bs);
         mx = fmaxf(mx, x[i]);
       }
     rescale_to(tr_head_max(mx));
@@ -747,18 +786,18 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
         if (BITS == 2) {
           // channels 16mt + gr (low byte of each half word) and 16mt + 8 + gr (high byte)
           const uint32_t w = vword(mt);
-          av[0] = kt ? unpack_pair<2, 2>(w, magic) : unpack_pair<2, 0>(w, magic);
-          av[1] = kt ? unpack_pair<2, 2>(w >> 8, magic) : unpack_pair<2, 0>(w >> 8, magic);
-          av[2] = kt ? unpack_pair<2, 3>(w, magic) : unpack_pair<2, 1>(w, magic);
-          av[3] = kt ? unpack_pair<2, 3>(w >> 8, magic) : unpack_pair<2, 1>(w >> 8, magic);
+          av[0] = kt ? code_pair<2, 2>(w) : code_pair<2, 0>(w);
+          av[1] = kt ? code_pair<2, 2>(w >> 8) : code_pair<2, 0>(w >> 8);
+          av[2] = kt ? code_pair<2, 3>(w) : code_pair<2, 1>(w);
+          av[3] = kt ? code_pair<2, 3>(w >> 8) : code_pair<2, 1>(w >> 8);
         } else {
           // words 2mt (channel 16mt + gr) and 2mt + 1 (16mt + 8 + gr); half word = kt
           const uint32_t w0 = kt ? vword(2 * mt) >> 8 : vword(2 * mt);
           const uint32_t w1 = kt ? vword(2 * mt + 1) >> 8 : vword(2 * mt + 1);
-          av[0] = unpack_pair<4, 0>(w0, magic);
-          av[1] = unpack_pair<4, 0>(w1, magic);
-          av[2] = unpack_pair<4, 1>(w0, magic);
-          av[3] = unpack_pair<4, 1>(w1, magic);
+          av[0] = code_pair<4, 0>(w0);
+          av[1] = code_pair<4, 0>(w1);
+          av[2] = code_pair<4, 1>(w0);
+          av[3] = code_pair<4, 1>(w1);
         }
         mma_f16_16816(o[mt], av, bp[2 * kt], bp[2 * kt + 1]);
       }
@@ -770,6 +809,7 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
     const int n_tok = min(kWinTok, a.r - (int)first * kWinTok);
     const int t0 = 16 * cw;
     if (cw >= kWinTok / 16 || t0 >= n_tok) return;
+    o_to_unit();
     const unsigned char* kb = st;
     const unsigned char* vb = st + kWinTok * C::WROW;
     const bool bf = gm.dtype == KVQ_BF16;
@@ -888,7 +928,7 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
           const int w = nt * WPN + wi;
           const uint4 pc = kc[w >> 2];
           const uint32_t word = (w & 3) == 0 ? pc.x : (w & 3) == 1 ? pc.y : (w & 3) == 2 ? pc.z : pc.w;
-          unpack_half<BITS>(half ? word >> 8 : word, pr[nt], magic);
+          code_half<BITS>(half ? word >> 8 : word, pr[nt]);
         }
 #pragma unroll
         for (int m2 = 0; m2 < J / 2; ++m2) {
@@ -905,7 +945,7 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) x[nt][e] = fmaf(sc[nt][e] + sc[nt][2 + e], a.scale_log2, bs);
+      for (int e = 0; e < 2; ++e) x[nt][e] = fmaf(sc[nt][e] + sc[nt][2 + e], sl_code, bs);
   };
   // online softmax and P.V of a block whose scores are x (record rec, token block tbg)
   auto hx_finish = [&](const unsigned char* rec, int tbg, const float (&x)[4][2]) {
@@ -960,18 +1000,18 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
         if (BITS == 2) {
           // channels 16mt + gr (low byte of each half word) and 16mt + 8 + gr (high byte)
           const uint32_t w = vword(mt);
-          av[0] = kt ? unpack_pair<2, 2>(w, magic) : unpack_pair<2, 0>(w, magic);
-          av[1] = kt ? unpack_pair<2, 2>(w >> 8, magic) : unpack_pair<2, 0>(w >> 8, magic);
-          av[2] = kt ? unpack_pair<2, 3>(w, magic) : unpack_pair<2, 1>(w, magic);
-          av[3] = kt ? unpack_pair<2, 3>(w >> 8, magic) : unpack_pair<2, 1>(w >> 8, magic);
+          av[0] = kt ? code_pair<2, 2>(w) : code_pair<2, 0>(w);
+          av[1] = kt ? code_pair<2, 2>(w >> 8) : code_pair<2, 0>(w >> 8);
+          av[2] = kt ? code_pair<2, 3>(w) : code_pair<2, 1>(w);
+          av[3] = kt ? code_pair<2, 3>(w >> 8) : code_pair<2, 1>(w >> 8);
         } else {
           // words 2mt (channel 16mt + gr) and 2mt + 1 (16mt + 8 + gr); half word = kt
           const uint32_t w0 = kt ? vword(2 * mt) >> 8 : vword(2 * mt);
           const uint32_t w1 = kt ? vword(2 * mt + 1) >> 8 : vword(2 * mt + 1);
-          av[0] = unpack_pair<4, 0>(w0, magic);
-          av[1] = unpack_pair<4, 0>(w1, magic);
-          av[2] = unpack_pair<4, 1>(w0, magic);
-          av[3] = unpack_pair<4, 1>(w1, magic);
+          av[0] = code_pair<4, 0>(w0);
+          av[1] = code_pair<4, 0>(w1);
+          av[2] = code_pair<4, 1>(w0);
+          av[3] = code_pair<4, 1>(w1);
         }
         mma_f16_16816(o[mt], av, bh[kt][0], bh[kt][1]);
         mma_f16_16816(o[mt], av, bl[kt][0], bl[kt][1]);
@@ -985,6 +1025,7 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
     const int n_tok = min(kWinTok, a.r - (int)first * kWinTok);
     const int t0 = 16 * cw;
     if (cw >= kWinTok / 16 || t0 >= n_tok) return;
+    o_to_unit();
     const unsigned char* kb = st;
     const unsigned char* vb = st + kWinTok * C::WROW;
     const bool bf = gm.dtype == KVQ_BF16;
@@ -1119,6 +1160,7 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
         *abort_flag = 1;
       }
     }
+    o_to_unit();
     float* s_m = sb;
     float* s_l = sb + C::NC * C::HS;
     float* s_o = sb + C::SO;
