@@ -1105,13 +1105,14 @@ __global__ void __launch_bounds__(512, 1) kivi_decode_kernel(const __grid_consta
       if (lane == 0 && !*abort_flag) atomicOr(gm.status, KVQ_DEV_WAIT_TIMEOUT);
       *abort_flag = 1;
     }
-    if (s == 0 && cw >= 4) {
-      // The consumer warps of one SM sub-partition (cw, cw + 4, cw + 8) start
-      // a fraction of a block apart, so that one's softmax overlaps another's
-      // mma's instead of all of them alternating in step (the stage waits
-      // never resynchronise them: the ring runs ahead of the consumers).
+    if (TR && s == 0 && cw >= 4) {
+      // Token-major formulation: the consumer warps of one SM sub-partition
+      // (cw, cw + 4, cw + 8) start a fraction of a block apart, so that one's
+      // softmax overlaps another's mma's instead of all of them alternating in
+      // step.  (In the hybrid formulation the warps drift into the same phase
+      // whatever the start offsets; measured on 70b, no offset was fastest.)
       const long long t0 = clock64();
-      const long long d = (cw >> 2) * (TR ? 800 : 1300);
+      const long long d = (cw >> 2) * 800;
       while (clock64() - t0 < d) {
       }
     }
