@@ -46,12 +46,18 @@ __device__ __forceinline__ CodeParams code_params(float s, float z, int levels) 
   p.eb = 2.384185791015625e-7f * (2.f * (float)levels + 2.f + fabsf(p.zinv));   // 2^-22 (...)
   return p;
 }
+// The exact decision, out of line: it runs for a small fraction of the
+// elements, and inlining it at every call site bloated the kernel's code
+// (instruction-cache misses were its top stall).
+__device__ __noinline__ uint32_t code_exact(float x, float z, float s, int levels) {
+  return (uint32_t)exact_code((double)x, (double)z, (double)s, s > 0.f ? 1.0 / (double)s : 0.0, levels);
+}
 __device__ __forceinline__ uint32_t code_of(float x, const CodeParams& p, int levels) {
   float r = fmaf(x, p.inv, -p.zinv);
   r = fminf(fmaxf(r, 0.f), (float)levels);   // also maps NaN to 0
   const float k = rintf(r);
   if (fabsf(fabsf(r - k) - 0.5f) > p.eb) return (uint32_t)k;
-  return (uint32_t)exact_code((double)x, (double)p.z, (double)p.s, p.s > 0.f ? 1.0 / (double)p.s : 0.0, levels);
+  return code_exact(x, p.z, p.s, levels);
 }
 
 template <bool BF>
@@ -134,8 +140,13 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
       }
     }
   } else {
+    // one token per step; lane k keeps step k's extremes, so the fp64
+    // parameter arithmetic runs on one lane per token at the end
     const int warp = (tid >> 5) - 2, lane = tid & 31;
-    for (int t = warp; t < G; t += 2) {
+    float my_mn = 0.f, my_mx = 0.f;
+    int my_t = -1;
+    static_assert(G / 2 <= 32, "value parameter split");
+    for (int t = warp, k = 0; t < G; t += 2, ++k) {
       float mn = INFINITY, mx = -INFINITY, nf = 0.f;
 #pragma unroll
       for (int c2 = lane; c2 < D / 2; c2 += 32) {
@@ -151,16 +162,21 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       }
       if (__any_sync(0xffffffffu, nf != 0.f)) flags |= KVQ_DEV_NONFINITE_INPUT;
-      if (lane == 0) {
-        const __half hs = __double2half(((double)mx - (double)mn) / (double)LEVELS);
-        const __half hz = __double2half((double)mn);
-        const float sc = __half2float(hs), z = __half2float(hz);
-        if (!isfinite(sc) || !isfinite(z)) flags |= KVQ_DEV_PARAM_OVERFLOW;
-        v_s[t] = sc;
-        v_z[t] = z;
-        v_sb[t] = __half_as_ushort(hs);
-        v_zb[t] = __half_as_ushort(hz);
+      if (lane == k) {
+        my_mn = mn;
+        my_mx = mx;
+        my_t = t;
       }
+    }
+    if (my_t >= 0) {
+      const __half hs = __double2half(((double)my_mx - (double)my_mn) / (double)LEVELS);
+      const __half hz = __double2half((double)my_mn);
+      const float sc = __half2float(hs), z = __half2float(hz);
+      if (!isfinite(sc) || !isfinite(z)) flags |= KVQ_DEV_PARAM_OVERFLOW;
+      v_s[my_t] = sc;
+      v_z[my_t] = z;
+      v_sb[my_t] = __half_as_ushort(hs);
+      v_zb[my_t] = __half_as_ushort(hz);
     }
   }
   __syncthreads();
