@@ -14,6 +14,7 @@
 // pair's parameters in registers), pack 16-byte pieces of the record.
 #include <cuda_runtime.h>
 
+#include "decode_common.cuh"
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -60,232 +61,407 @@ __device__ __forceinline__ uint32_t code_of(float x, const CodeParams& p, int le
   return code_exact(x, p.z, p.s, levels);
 }
 
+// ------------------------------------------------------------------ per-unit parameters
+// A unit is one key channel of the group or one value token.  mn and mx are its
+// extremes as floats (exact); mx propagates a nan input.
+template <int BITS, bool BF>
+struct UnitOut {
+  uint16_t sb, zb;          // fp16 scale and zero-point (record metadata)
+  float s, z;
+  uint16_t c[3];            // 2-bit: 16-bit code thresholds
+  float inv, zinv, thr;     // 4-bit: code estimate constants
+  uint32_t flags;
+};
+
 template <bool BF>
-__device__ __forceinline__ float in16f(uint16_t bits) {
-  return BF ? __uint_as_float((uint32_t)bits << 16) : __half2float(__ushort_as_half(bits));
+__device__ __forceinline__ uint16_t to16_rn(double x) {
+  if (BF) return __bfloat16_as_ushort(__double2bfloat16(x));
+  return __half_as_ushort(__double2half(x));
+}
+template <bool BF>
+__device__ __forceinline__ double from16(uint16_t b) {
+  return BF ? (double)__uint_as_float((uint32_t)b << 16) : (double)__half2float(__ushort_as_half(b));
+}
+// The next larger value of the 16-bit input format (nan and +inf stay).
+template <bool BF>
+__device__ __forceinline__ uint16_t next_up16(uint16_t b) {
+  constexpr uint16_t kInf = BF ? 0x7F80 : 0x7C00;
+  if ((b & 0x7FFF) >= kInf && b != (uint16_t)(kInf | 0x8000)) return b;
+  if (b == 0x8000) return 1;
+  return (b & 0x8000) ? (uint16_t)(b - 1) : (uint16_t)(b + 1);
+}
+// The smallest input value v with v >= X (strict: v > X); X is exact in double.
+// Then "x >= v" for an input x says exactly "x >= X" (or "x > X").
+template <bool BF>
+__device__ __forceinline__ uint16_t threshold16(double X, bool strict) {
+  uint16_t c = to16_rn<BF>(X);
+  const double cd = from16<BF>(c);
+  if (cd < X || (strict && cd == X)) c = next_up16<BF>(c);
+  return c;
+}
+
+// Parameters s = fp16((max - min) / L) (the quotient rounded once in double,
+// then to fp16) and z = fp16(min).  2-bit codes count the thresholds
+// X_k = z + (k + 1/2) s that x passes: x > X_k for even k, x >= X_k for odd k,
+// which is round half to even of (x - z) / s clamped to [0, 3]; X_k is exact
+// in double, so each test becomes "x >= c_k" for one 16-bit constant.  s == 0
+// gives code 0 (thresholds +inf).  4-bit codes use the fp32 estimate described
+// at code_of, with thr = 0.5 - eb, or -1 (every code decided exactly) when z is
+// far enough from min, or s small enough against max - z, that an estimate
+// could leave [0, 15].
+template <int BITS, bool BF>
+__device__ __forceinline__ UnitOut<BITS, BF> unit_params(float mn, float mx) {
+  constexpr int L = (1 << BITS) - 1;
+  UnitOut<BITS, BF> u;
+  u.flags = (isfinite(mn) && isfinite(mx)) ? 0u : (uint32_t)KVQ_DEV_NONFINITE_INPUT;
+  const double dmn = mn, dmx = mx;
+  const __half hs = __double2half((dmx - dmn) / (double)L), hz = __double2half(dmn);
+  u.sb = __half_as_ushort(hs);
+  u.zb = __half_as_ushort(hz);
+  u.s = __half2float(hs);
+  u.z = __half2float(hz);
+  if (isinf(u.s) || isinf(u.z)) u.flags |= KVQ_DEV_PARAM_OVERFLOW;
+  if constexpr (BITS == 2) {
+    constexpr uint16_t kInf = BF ? 0x7F80 : 0x7C00;
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+      u.c[k] = u.s == 0.f ? kInf : threshold16<BF>((double)u.z + (k + 0.5) * (double)u.s, (k & 1) == 0);
+  } else {
+    u.inv = u.s > 0.f ? 1.f / u.s : 0.f;
+    u.zinv = u.z * u.inv;
+    const bool safe = ((double)u.z - dmn <= 0.5 * (double)u.s) && (dmx - (double)u.z <= (L + 0.5) * (double)u.s);
+    u.thr = safe ? 0.5f - 2.384185791015625e-7f * (2.f * (float)L + 2.f + fabsf(u.zinv)) : -1.f;
+  }
+  return u;
+}
+
+template <bool BF> struct Pair16;
+template <> struct Pair16<false> {
+  using T = __half2;
+  static __device__ __forceinline__ T of(uint32_t u) { return u32_as_h2(u); }
+  static __device__ __forceinline__ float lo(T v) { return __low2float(v); }
+  static __device__ __forceinline__ float hi(T v) { return __high2float(v); }
+};
+template <> struct Pair16<true> {
+  using T = __nv_bfloat162;
+  static __device__ __forceinline__ T of(uint32_t u) { return *reinterpret_cast<__nv_bfloat162*>(&u); }
+  static __device__ __forceinline__ float lo(T v) { return __low2float(v); }
+  static __device__ __forceinline__ float hi(T v) { return __high2float(v); }
+};
+
+// 2-bit: the two codes of a pair from three 16-bit threshold pairs.  The masks
+// m0 >= m1 >= m2 (0xFFFF per passing half) are a thermometer code; its count in
+// binary is b1 = m1, b0 = m0 ^ m1 ^ m2.  Pair j lands at bits (2j, 16 + 2j).
+template <bool BF>
+__device__ __forceinline__ uint32_t code_pair2(uint32_t x, uint32_t c0, uint32_t c1, uint32_t c2, int j) {
+  using P = Pair16<BF>;
+  const uint32_t m0 = __hge2_mask(P::of(x), P::of(c0));
+  const uint32_t m1 = __hge2_mask(P::of(x), P::of(c1));
+  const uint32_t m2 = __hge2_mask(P::of(x), P::of(c2));
+  return ((m0 ^ m1 ^ m2) & (0x00010001u << (2 * j))) | (m1 & (0x00020002u << (2 * j)));
+}
+
+// 4-bit: fp32 estimates of the codes of a pair, accumulated as k * 16^j into
+// the low bits of 2^23-offset floats; ok turns false when a code is undecided.
+template <bool BF>
+__device__ __forceinline__ void code_pair4(uint32_t x, float inv0, float zinv0, float inv1, float zinv1, float thr,
+                                           float& acc0, float& acc1, bool& ok, int j) {
+  using P = Pair16<BF>;
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23: adding it rounds to an integer
+  const float kPos = (float)(1 << (4 * j));
+  const float x0 = P::lo(P::of(x)), x1 = P::hi(P::of(x));
+  const float r0 = fmaf(x0, inv0, -zinv0), r1 = fmaf(x1, inv1, -zinv1);
+  const float k0 = (r0 + kRound) - kRound, k1 = (r1 + kRound) - kRound;
+  ok = ok && fabsf(r0 - k0) < thr && fabsf(r1 - k1) < thr;
+  acc0 = fmaf(k0, kPos, acc0);
+  acc1 = fmaf(k1, kPos, acc1);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem));
 }
 
 // One CTA quantizes one group record (G tokens of one row); BF: bf16 inputs
 // (else fp16).
+//
+// 1. The key and value tiles are copied to shared memory (rows padded by 16
+//    bytes, so the 8 rows of an 8x8 ldmatrix tile fall in distinct banks).
+// 2. Parameters: warps 0-1 reduce key channel pairs over the G tokens, warps
+//    2-3 value tokens over the d channels, with 16-bit pair min/max.
+// 3. Codes: a thread builds whole 32-bit words of the packed format for its own
+//    lane.  ldmatrix hands lane (gr, tc) exactly a word's pairs: a key tile
+//    (tokens x channels) gives token gr, channels 2tc and 2tc + 1; the same
+//    tile transposed gives channel gr, tokens 2tc and 2tc + 1 for the values.
+//    Warps 0-1 code keys (a thread keeps the thresholds of its channels across
+//    token blocks), warps 2-3 values (a thread keeps its eight tokens').
+// 4. The record, assembled in shared memory, is stored in 16-byte pieces.
 template <int BITS, int D, int G, bool BF>
 __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs a) {
-  constexpr int LEVELS = (1 << BITS) - 1;
+  constexpr int L = (1 << BITS) - 1;
   constexpr int NTB = G / kTB;
-  constexpr int P = D * BITS / 32;              // words per lane per TB
   constexpr int PAIRS = 16 / BITS;              // pairs per word
-  constexpr int J = BITS == 2 ? 4 : 2;          // pairs per half word
-  constexpr int PITCH = D + 8;                  // staged row pitch (halves): rows 8 apart land 4 banks apart
-  // key codes: thread = (channel pair, token range); value codes: thread = (token pair, channel range)
-  constexpr int KCP = D / 2, KTR = kQuantThreads / KCP, KTOK = G / KTR;
-  constexpr int VTP = G / 2, VCR = kQuantThreads / VTP, VCH = D / VCR;
-  static_assert(kQuantThreads % KCP == 0 && G % KTR == 0, "key code split");
-  static_assert(kQuantThreads % VTP == 0 && D % VCR == 0 && VCH % 8 == 0, "value code split");
+  constexpr int P = D * BITS / 32;              // words per lane per TB (keys or values)
+  constexpr int WPT = D * BITS / 128;           // key words per (lane, 8-token block)
+  constexpr int CPW = PAIRS / 4;                // 8-channel blocks per value word
+  constexpr int TBB = kTB * D * BITS / 8;       // code bytes of one TB
+  constexpr int REC = 2 * NTB * TBB + 4 * D + NTB * kTB * 4;
+  constexpr int PITCH = D + 8;                  // staged row pitch (halves)
+  constexpr int KS = 128 / D;                   // key parameter threads per channel pair
+  constexpr int VS = 64 / G;                    // value parameter threads per token
+  static_assert(REC % 16 == 0 && PAIRS % 4 == 0 && (D / 2) * KS == 64 && VS >= 1, "shape");
   extern __shared__ __align__(16) unsigned char smem[];
-  uint16_t* sk = reinterpret_cast<uint16_t*>(smem);            // [G][PITCH] staged keys
-  uint16_t* sv = sk + G * PITCH;                               // [G][PITCH] staged values
-  uint8_t* ck = reinterpret_cast<uint8_t*>(sv + G * PITCH);    // [G][D] key codes
-  uint8_t* cvt = ck + G * D;                                   // [D][G] value codes (channel-major)
-  __shared__ float k_s[D], k_z[D];
-  __shared__ float v_s[G], v_z[G];
-  __shared__ uint16_t k_sb[D], k_zb[D], v_sb[G], v_zb[G];
+  uint16_t* sk = reinterpret_cast<uint16_t*>(smem);           // [G][PITCH]
+  uint16_t* sv = sk + G * PITCH;                              // [G][PITCH]
+  unsigned char* srec = reinterpret_cast<unsigned char*>(sv + G * PITCH);   // record image
+  // 2-bit: thresholds, 16-bit per unit, adjacent units share a word
+  // 4-bit: (inv, zinv, thr, -) and (s, z) per unit
+  __shared__ __align__(16) uint16_t kc[BITS == 2 ? 3 : 1][D], vc[BITS == 2 ? 3 : 1][G];
+  __shared__ __align__(16) float4 kp[BITS == 4 ? D : 1], vp[BITS == 4 ? G : 1];
+  __shared__ __align__(16) float2 ksz[BITS == 4 ? D : 1], vsz[BITS == 4 ? G : 1];
   __shared__ uint32_t s_flags;
 
-  const Geom& gm = a.geom;
   const int row = blockIdx.y;
   const int grp = blockIdx.x;
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   if (tid == 0) s_flags = 0;
 
-  // 1. stage the key and value tiles
-  const uint16_t* gk = a.src_k + (int64_t)row * a.src_row_stride + (int64_t)grp * G * D;
-  const uint16_t* gv = a.src_v + (int64_t)row * a.src_row_stride + (int64_t)grp * G * D;
-  for (int i = tid; i < G * D / 8; i += kQuantThreads) {
-    const int t = i / (D / 8), c8 = i - t * (D / 8);
-    *reinterpret_cast<uint4*>(sk + t * PITCH + 8 * c8) = ldg_nc_v4(reinterpret_cast<const uint4*>(gk) + i);
-    *reinterpret_cast<uint4*>(sv + t * PITCH + 8 * c8) = ldg_nc_v4(reinterpret_cast<const uint4*>(gv) + i);
+  // 1. stage
+  {
+    const uint16_t* gk = a.src_k + (int64_t)row * a.src_row_stride + (int64_t)grp * G * D;
+    const uint16_t* gv = a.src_v + (int64_t)row * a.src_row_stride + (int64_t)grp * G * D;
+#pragma unroll 4
+    for (int i = tid; i < G * D / 8; i += kQuantThreads) {
+      const int t = i / (D / 8), c8 = i - t * (D / 8);
+      cp_async16(sk + t * PITCH + 8 * c8, gk + 8 * i);
+      cp_async16(sv + t * PITCH + 8 * c8, gv + 8 * i);
+    }
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
   }
   __syncthreads();
 
+  using PT = Pair16<BF>;
+  using T2 = typename PT::T;
   uint32_t flags = 0;
-  // 2. parameters.  Warps 0-1: keys, one channel pair per thread over the G
-  // tokens; warps 2-3: values, one token per warp at a time.  An input that is
-  // inf or NaN turns the running fma(x, 0, .) into NaN.
-  static_assert(D / 2 <= 64, "key parameter split");
-  if (tid < 64) {
-    for (int cp = tid; cp < D / 2; cp += 64) {
-      const int c = 2 * cp;
-      float mn0 = INFINITY, mx0 = -INFINITY, mn1 = INFINITY, mx1 = -INFINITY, nf = 0.f;
-#pragma unroll 8
-      for (int t = 0; t < G; ++t) {
-        const uint32_t x2 = *reinterpret_cast<const uint32_t*>(sk + t * PITCH + c);
-        const float x0 = in16f<BF>((uint16_t)(x2 & 0xFFFFu)), x1 = in16f<BF>((uint16_t)(x2 >> 16));
-        nf = fmaf(x0, 0.f, fmaf(x1, 0.f, nf));
-        mn0 = fminf(mn0, x0);
-        mx0 = fmaxf(mx0, x0);
-        mn1 = fminf(mn1, x1);
-        mx1 = fmaxf(mx1, x1);
-      }
-      if (nf != 0.f) flags |= KVQ_DEV_NONFINITE_INPUT;
+  uint16_t* ksc = reinterpret_cast<uint16_t*>(srec + 2 * NTB * TBB);   // key scales, then zeros
+  uint32_t* vmeta = reinterpret_cast<uint32_t*>(srec + 2 * NTB * TBB + 4 * D);
+  auto put_key = [&](int c, const UnitOut<BITS, BF>& u) {
+    const int kt = c >> 4, rho = (c >> 3) & 1, tc = (c >> 1) & 3, e = c & 1;
+    const int pos = 8 * (4 * (kt >> 1) + tc) + 4 * (kt & 1) + 2 * rho + e;
+    ksc[pos] = u.sb;
+    ksc[D + pos] = u.zb;
+    if constexpr (BITS == 2) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float mn = e ? mn1 : mn0, mx = e ? mx1 : mx0;
-        const __half hs = __double2half(((double)mx - (double)mn) / (double)LEVELS);
-        const __half hz = __double2half((double)mn);
-        const float sc = __half2float(hs), z = __half2float(hz);
-        if (!isfinite(sc) || !isfinite(z)) flags |= KVQ_DEV_PARAM_OVERFLOW;
-        k_s[c + e] = sc;
-        k_z[c + e] = z;
-        k_sb[c + e] = __half_as_ushort(hs);
-        k_zb[c + e] = __half_as_ushort(hz);
+      for (int k = 0; k < 3; ++k) kc[k][c] = u.c[k];
+    } else {
+      kp[c] = make_float4(u.inv, u.zinv, u.thr, 0.f);
+      ksz[c] = make_float2(u.s, u.z);
+    }
+    flags |= u.flags;
+  };
+  auto put_value = [&](int t, const UnitOut<BITS, BF>& u) {
+    const int tb = t / kTB, tt = t % kTB;
+    const int kt = tt >> 4, rho = (tt >> 3) & 1, tc = (tt >> 1) & 3, e = tt & 1;
+    vmeta[tb * kTB + 8 * tc + 4 * kt + 2 * rho + e] = (uint32_t)u.sb | ((uint32_t)u.zb << 16);
+    if constexpr (BITS == 2) {
+#pragma unroll
+      for (int k = 0; k < 3; ++k) vc[k][t] = u.c[k];
+    } else {
+      vp[t] = make_float4(u.inv, u.zinv, u.thr, 0.f);
+      vsz[t] = make_float2(u.s, u.z);
+    }
+    flags |= u.flags;
+  };
+
+  // 2. parameters
+  if (tid < 64) {
+    // channel pair pc over tokens ks, ks + KS, ... (rows 1 apart: 4 banks apart)
+    const int pc = tid / KS, ks = tid % KS;
+    T2 mn = PT::of(BF ? 0x7F807F80u : 0x7C007C00u), mx = PT::of(BF ? 0xFF80FF80u : 0xFC00FC00u);
+#pragma unroll 8
+    for (int t = ks; t < G; t += KS) {
+      const T2 x = PT::of(*reinterpret_cast<const uint32_t*>(sk + t * PITCH + 2 * pc));
+      mn = __hmin2(mn, x);
+      mx = __hmax2_nan(mx, x);
+    }
+    if (KS == 2) {
+      uint32_t a0 = *reinterpret_cast<uint32_t*>(&mn), a1 = *reinterpret_cast<uint32_t*>(&mx);
+      mn = __hmin2(mn, PT::of(__shfl_xor_sync(0xffffffffu, a0, 1)));
+      mx = __hmax2_nan(mx, PT::of(__shfl_xor_sync(0xffffffffu, a1, 1)));
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      if (KS == 2 && e != ks) continue;
+      const float fmn = e ? PT::hi(mn) : PT::lo(mn), fmx = e ? PT::hi(mx) : PT::lo(mx);
+      put_key(2 * pc + e, unit_params<BITS, BF>(fmn, fmx));
+    }
+  } else {
+    // token t over channel pairs [v D/(2 VS), (v + 1) D/(2 VS)), four at a time
+    const int u = tid - 64, t = u / VS, v = u % VS;
+    constexpr int PPV = D / (2 * VS);
+    T2 mn = PT::of(BF ? 0x7F807F80u : 0x7C007C00u), mx = PT::of(BF ? 0xFF80FF80u : 0xFC00FC00u);
+#pragma unroll 4
+    for (int p4 = 0; p4 < PPV / 4; ++p4) {
+      const uint4 q = *reinterpret_cast<const uint4*>(sv + t * PITCH + 2 * (v * PPV + 4 * p4));
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        mn = __hmin2(mn, PT::of(w[i]));
+        mx = __hmax2_nan(mx, PT::of(w[i]));
+      }
+    }
+    float fmn = fminf(PT::lo(mn), PT::hi(mn));
+    float fmx = PT::lo(mx), fmx1 = PT::hi(mx);
+    fmx = (isnan(fmx) || isnan(fmx1)) ? __int_as_float(0x7fc00000) : fmaxf(fmx, fmx1);
+    if (VS == 2) {
+      const float omn = __shfl_xor_sync(0xffffffffu, fmn, 1), omx = __shfl_xor_sync(0xffffffffu, fmx, 1);
+      fmn = fminf(fmn, omn);
+      fmx = (isnan(fmx) || isnan(omx)) ? __int_as_float(0x7fc00000) : fmaxf(fmx, omx);
+    }
+    if (v == 0) put_value(t, unit_params<BITS, BF>(fmn, fmx));
+  }
+  __syncthreads();
+
+  // 3. codes
+  const int tc = lane & 3;
+  auto word_at = [&](bool is_v, int tb, int w) -> uint32_t* {
+    return reinterpret_cast<uint32_t*>(srec + (is_v ? NTB + tb : tb) * TBB + 16 * (32 * (w >> 2) + lane) + 4 * (w & 3));
+  };
+  if (warp < 2) {
+    // keys: word (nt, sub) of token 8 nt + gr holds channels 8 PAIRS sub + 8 j + 2 tc (+1)
+    constexpr int SUBS_PER_WARP = WPT >= 2 ? WPT / 2 : 1;
+    for (int si = 0; si < SUBS_PER_WARP; ++si) {
+      const int sub = WPT >= 2 ? 2 * si + warp : 0;
+      const int cbase = 8 * PAIRS * sub + 2 * tc;
+      if constexpr (BITS == 2) {
+        uint32_t c0[PAIRS], c1[PAIRS], c2[PAIRS];
+#pragma unroll
+        for (int j = 0; j < PAIRS; ++j) {
+          c0[j] = *reinterpret_cast<const uint32_t*>(&kc[0][cbase + 8 * j]);
+          c1[j] = *reinterpret_cast<const uint32_t*>(&kc[1][cbase + 8 * j]);
+          c2[j] = *reinterpret_cast<const uint32_t*>(&kc[2][cbase + 8 * j]);
+        }
+#pragma unroll 1
+        for (int it = (WPT >= 2 ? 0 : warp); it < NTB * 4; it += (WPT >= 2 ? 1 : 2)) {
+          const int tb = it >> 2, nt = it & 3;
+          const uint16_t* rowp = sk + (tb * kTB + 8 * nt + (lane & 7)) * PITCH + 8 * PAIRS * sub + 8 * (lane >> 3);
+          uint32_t x[PAIRS];
+#pragma unroll
+          for (int i = 0; i < PAIRS / 4; ++i) ldsm_x4(x + 4 * i, rowp + 32 * i);
+          uint32_t wd = 0;
+#pragma unroll
+          for (int j = 0; j < PAIRS; ++j) wd |= code_pair2<BF>(x[j], c0[j], c1[j], c2[j], j);
+          *word_at(false, tb, nt * WPT + sub) = wd;
+        }
+      } else {
+        float inv[2 * PAIRS], zinv[2 * PAIRS], thr = 0.5f;
+#pragma unroll
+        for (int j = 0; j < PAIRS; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float4 q = kp[cbase + 8 * j + e];
+            inv[2 * j + e] = q.x;
+            zinv[2 * j + e] = q.y;
+            thr = fminf(thr, q.z);
+          }
+#pragma unroll 1
+        for (int it = (WPT >= 2 ? 0 : warp); it < NTB * 4; it += (WPT >= 2 ? 1 : 2)) {
+          const int tb = it >> 2, nt = it & 3;
+          const uint16_t* rowp = sk + (tb * kTB + 8 * nt + (lane & 7)) * PITCH + 8 * PAIRS * sub + 8 * (lane >> 3);
+          uint32_t x[PAIRS];
+#pragma unroll
+          for (int i = 0; i < PAIRS / 4; ++i) ldsm_x4(x + 4 * i, rowp + 32 * i);
+          float acc0 = 8388608.f, acc1 = 8388608.f;
+          bool ok = true;
+#pragma unroll
+          for (int j = 0; j < PAIRS; ++j)
+            code_pair4<BF>(x[j], inv[2 * j], zinv[2 * j], inv[2 * j + 1], zinv[2 * j + 1], thr, acc0, acc1, ok, j);
+          uint32_t wd = __byte_perm(__float_as_uint(acc0), __float_as_uint(acc1), 0x5410);
+          if (!ok) {
+            wd = 0;
+            for (int j = 0; j < PAIRS; ++j)
+              for (int e = 0; e < 2; ++e) {
+                const int c = cbase + 8 * j + e;
+                const float xv = e ? PT::hi(PT::of(x[j])) : PT::lo(PT::of(x[j]));
+                wd |= code_of(xv, code_params(ksz[c].x, ksz[c].y, L), L) << (16 * e + BITS * j);
+              }
+          }
+          *word_at(false, tb, nt * WPT + sub) = wd;
+        }
       }
     }
   } else {
-    // one token per step; lane k keeps step k's extremes, so the fp64
-    // parameter arithmetic runs on one lane per token at the end
-    const int warp = (tid >> 5) - 2, lane = tid & 31;
-    float my_mn = 0.f, my_mx = 0.f;
-    int my_t = -1;
-    static_assert(G / 2 <= 32, "value parameter split");
-    for (int t = warp, k = 0; t < G; t += 2, ++k) {
-      float mn = INFINITY, mx = -INFINITY, nf = 0.f;
+    // values: word w holds channels 8 (CPW w + j / 4) + gr, tokens 8 (j % 4) + 2 tc (+1)
+    const int vw = warp - 2;
+    for (int tb = 0; tb < NTB; ++tb) {
+      if constexpr (BITS == 2) {
+        uint32_t c0[4], c1[4], c2[4];
 #pragma unroll
-      for (int c2 = lane; c2 < D / 2; c2 += 32) {
-        const uint32_t x2 = *reinterpret_cast<const uint32_t*>(sv + t * PITCH + 2 * c2);
-        const float x0 = in16f<BF>((uint16_t)(x2 & 0xFFFFu)), x1 = in16f<BF>((uint16_t)(x2 >> 16));
-        nf = fmaf(x0, 0.f, fmaf(x1, 0.f, nf));
-        mn = fminf(mn, fminf(x0, x1));
-        mx = fmaxf(mx, fmaxf(x0, x1));
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      }
-      if (__any_sync(0xffffffffu, nf != 0.f)) flags |= KVQ_DEV_NONFINITE_INPUT;
-      if (lane == k) {
-        my_mn = mn;
-        my_mx = mx;
-        my_t = t;
-      }
-    }
-    if (my_t >= 0) {
-      const __half hs = __double2half(((double)my_mx - (double)my_mn) / (double)LEVELS);
-      const __half hz = __double2half((double)my_mn);
-      const float sc = __half2float(hs), z = __half2float(hz);
-      if (!isfinite(sc) || !isfinite(z)) flags |= KVQ_DEV_PARAM_OVERFLOW;
-      v_s[my_t] = sc;
-      v_z[my_t] = z;
-      v_sb[my_t] = __half_as_ushort(hs);
-      v_zb[my_t] = __half_as_ushort(hz);
-    }
-  }
-  __syncthreads();
-
-  // 4. codes.  Keys: channels (2 cp, 2 cp + 1) of tokens [tr * KTOK, +KTOK);
-  // the two codes of a token land side by side in ck.
-  {
-    const int cp = tid % KCP, tr = tid / KCP;
-    const int c = 2 * cp;
-    const CodeParams p0 = code_params(k_s[c], k_z[c], LEVELS), p1 = code_params(k_s[c + 1], k_z[c + 1], LEVELS);
-#pragma unroll 4
-    for (int t = tr * KTOK; t < (tr + 1) * KTOK; ++t) {
-      const uint32_t x2 = *reinterpret_cast<const uint32_t*>(sk + t * PITCH + c);
-      const uint32_t q0 = code_of(in16f<BF>((uint16_t)(x2 & 0xFFFFu)), p0, LEVELS);
-      const uint32_t q1 = code_of(in16f<BF>((uint16_t)(x2 >> 16)), p1, LEVELS);
-      *reinterpret_cast<uint16_t*>(ck + t * D + c) = (uint16_t)(q0 | (q1 << 8));
-    }
-  }
-  // Values: tokens (2 tp, 2 tp + 1), channels [cr * VCH, +VCH); the two codes of
-  // a channel land side by side in the channel-major cvt.
-  {
-    const int tp = tid % VTP, cr = tid / VTP;
-    const int t = 2 * tp;
-    const CodeParams p0 = code_params(v_s[t], v_z[t], LEVELS), p1 = code_params(v_s[t + 1], v_z[t + 1], LEVELS);
-#pragma unroll 2
-    for (int c8 = cr * VCH; c8 < (cr + 1) * VCH; c8 += 8) {
-      const uint4 x0 = *reinterpret_cast<const uint4*>(sv + t * PITCH + c8);
-      const uint4 x1 = *reinterpret_cast<const uint4*>(sv + (t + 1) * PITCH + c8);
-      const uint32_t w0[4] = {x0.x, x0.y, x0.z, x0.w}, w1[4] = {x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint16_t h0 = (uint16_t)(w0[e >> 1] >> (16 * (e & 1))), h1 = (uint16_t)(w1[e >> 1] >> (16 * (e & 1)));
-        const uint32_t q0 = code_of(in16f<BF>(h0), p0, LEVELS);
-        const uint32_t q1 = code_of(in16f<BF>(h1), p1, LEVELS);
-        *reinterpret_cast<uint16_t*>(cvt + (c8 + e) * G + t) = (uint16_t)(q0 | (q1 << 8));
-      }
-    }
-  }
-  __syncthreads();
-
-  // 5. packing: one 16-byte piece (4 words of one lane) per iteration; a pair
-  // is the codes of two adjacent channels of a token (keys) or of two adjacent
-  // tokens of a channel (values), one 16-bit load either way
-  char* rec = record_ptr(gm, row, a.dst_group0 + grp);
-  if (rec == nullptr) flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
-  constexpr int PIECES = NTB * 32 * (P / 4);   // per key (or value) part
-  for (int i = rec != nullptr ? tid : 2 * PIECES; i < 2 * PIECES; i += kQuantThreads) {
-    const bool is_v = i >= PIECES;
-    const int pi = is_v ? i - PIECES : i;
-    const int tb = pi / (32 * (P / 4));
-    const int rem = pi - tb * 32 * (P / 4);
-    const int p = rem / 32, lane = rem & 31;
-    const int gr = lane >> 2, tc = lane & 3;
-    uint32_t wv[4];
-#pragma unroll
-    for (int e4 = 0; e4 < 4; ++e4) {
-      const int w = 4 * p + e4;
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < PAIRS; ++j) {
-        const int half = j / J, jp = j % J;
-        const int slot = 2 * w + half;
-        uint32_t pr;
-        if (!is_v) {
-          constexpr int SPN = BITS == 2 ? D / 32 : D / 16;   // slots per key n-tile
-          const int nt = slot / SPN;
-          const int u = BITS == 2 ? 4 * (slot % SPN) + jp : 2 * (slot % SPN) + jp;
-          const int kt = u >> 1, rho = u & 1;
-          pr = *reinterpret_cast<const uint16_t*>(ck + (tb * kTB + 8 * nt + gr) * D + 16 * kt + 8 * rho + 2 * tc);
-        } else {
-          int nt, u;
-          if (BITS == 2) {
-            nt = slot;
-            u = jp;
-          } else {
-            nt = slot >> 1;
-            u = 2 * (slot & 1) + jp;
-          }
-          const int kt = u >> 1, rho = u & 1;
-          pr = *reinterpret_cast<const uint16_t*>(cvt + (8 * nt + gr) * G + tb * kTB + 16 * kt + 8 * rho + 2 * tc);
+        for (int m = 0; m < 4; ++m) {
+          const int t = tb * kTB + 8 * m + 2 * tc;
+          c0[m] = *reinterpret_cast<const uint32_t*>(&vc[0][t]);
+          c1[m] = *reinterpret_cast<const uint32_t*>(&vc[1][t]);
+          c2[m] = *reinterpret_cast<const uint32_t*>(&vc[2][t]);
         }
-        // pr = lo | hi << 8  ->  lo at bit b j, hi at bit 16 + b j
-        word |= ((pr | (pr << 8)) & 0x00FF00FFu) << (BITS * j);
+#pragma unroll 1
+        for (int w = vw; w < P; w += 2) {
+          uint32_t x[PAIRS];
+#pragma unroll
+          for (int i = 0; i < PAIRS / 4; ++i)
+            ldsm_x4_t(x + 4 * i, sv + (tb * kTB + 8 * (lane >> 3) + (lane & 7)) * PITCH + 8 * (CPW * w + i));
+          uint32_t wd = 0;
+#pragma unroll
+          for (int j = 0; j < PAIRS; ++j) wd |= code_pair2<BF>(x[j], c0[j & 3], c1[j & 3], c2[j & 3], j);
+          *word_at(true, tb, w) = wd;
+        }
+      } else {
+        float inv[8], zinv[8], thr = 0.5f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float4 q = vp[tb * kTB + 8 * m + 2 * tc + e];
+            inv[2 * m + e] = q.x;
+            zinv[2 * m + e] = q.y;
+            thr = fminf(thr, q.z);
+          }
+#pragma unroll 1
+        for (int w = vw; w < P; w += 2) {
+          uint32_t x[PAIRS];
+          ldsm_x4_t(x, sv + (tb * kTB + 8 * (lane >> 3) + (lane & 7)) * PITCH + 8 * w);
+          float acc0 = 8388608.f, acc1 = 8388608.f;
+          bool ok = true;
+#pragma unroll
+          for (int j = 0; j < PAIRS; ++j)
+            code_pair4<BF>(x[j], inv[2 * j], zinv[2 * j], inv[2 * j + 1], zinv[2 * j + 1], thr, acc0, acc1, ok, j);
+          uint32_t wd = __byte_perm(__float_as_uint(acc0), __float_as_uint(acc1), 0x5410);
+          if (!ok) {
+            wd = 0;
+            for (int j = 0; j < PAIRS; ++j)
+              for (int e = 0; e < 2; ++e) {
+                const int t = tb * kTB + 8 * j + 2 * tc + e;
+                const float xv = e ? PT::hi(PT::of(x[j])) : PT::lo(PT::of(x[j]));
+                wd |= code_of(xv, code_params(vsz[t].x, vsz[t].y, L), L) << (16 * e + BITS * j);
+              }
+          }
+          *word_at(true, tb, w) = wd;
+        }
       }
-      wv[e4] = word;
     }
-    char* dst = rec + (is_v ? (NTB + tb) : tb) * (int64_t)(kTB * D * BITS / 8) + 16 * (32 * p + lane);
-    *reinterpret_cast<uint4*>(dst) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-  }
-
-  // 6. metadata
-  uint16_t* ksc = reinterpret_cast<uint16_t*>(rec + rec_kscale_off(gm));
-  uint16_t* kzr = reinterpret_cast<uint16_t*>(rec + rec_kzero_off(gm));
-  for (int c = rec != nullptr ? tid : D; c < D; c += kQuantThreads) {
-    const int kt = c >> 4, rho = (c >> 3) & 1, tc = (c >> 1) & 3, e = c & 1;
-    const int pos = 8 * (4 * (kt >> 1) + tc) + 4 * (kt & 1) + 2 * rho + e;
-    ksc[pos] = k_sb[c];
-    kzr[pos] = k_zb[c];
-  }
-  uint32_t* vm = reinterpret_cast<uint32_t*>(rec + rec_vmeta_off(gm));
-  for (int t = rec != nullptr ? tid : G; t < G; t += kQuantThreads) {
-    const int tb = t / kTB, tt = t % kTB;
-    const int kt = tt >> 4, rho = (tt >> 3) & 1, tc = (tt >> 1) & 3, e = tt & 1;
-    vm[tb * kTB + 8 * tc + 4 * kt + 2 * rho + e] = (uint32_t)v_sb[t] | ((uint32_t)v_zb[t] << 16);
   }
 
   if (flags) atomicOr(&s_flags, flags);
   __syncthreads();
-  if (tid == 0) flag_status(gm.status, s_flags);
+
+  // 4. store the record
+  char* rec = record_ptr(a.geom, row, a.dst_group0 + grp);
+  if (rec != nullptr) {
+    for (int i = tid; i < REC / 16; i += kQuantThreads)
+      reinterpret_cast<uint4*>(rec)[i] = reinterpret_cast<const uint4*>(srec)[i];
+  } else if (tid == 0) {
+    s_flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
+  }
+  if (tid == 0 && s_flags) flag_status(a.geom.status, s_flags);
 }
 
 // Copies window tokens [t0, t0 + n) of every row of a [B][Hkv][S][d] input into
@@ -322,7 +498,7 @@ __global__ void clear_words_kernel(uint32_t* words, int n) {
 
 template <int BITS, int D, int G, bool BF>
 void launch_q_dtype(const QuantArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)G * (D + 8) * 2 * 2 + (size_t)G * D * 2;
+  const size_t smem = (size_t)G * (D + 8) * 2 * 2 + (size_t)(2 * G * D * BITS / 8 + 4 * D + G * 4);
   auto kern = kivi_quantize_kernel<BITS, D, G, BF>;
   static bool attr_set = false;   // per template instance; the attribute is per device function
   if (!attr_set) {

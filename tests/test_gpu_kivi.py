@@ -123,6 +123,21 @@ def test_code_decisions_on_large_offsets_and_ties(dtype, bits):
     _run_prefill_bits(w, k, v)
 
 
+@pytest.mark.parametrize("dtype,bits", [("fp16", 2), ("fp16", 4), ("bf16", 2), ("bf16", 4)])
+def test_code_decisions_on_tiny_inputs(dtype, bits):
+    """Inputs around 1e-6: fp16 subnormals, and for bf16 zero-points and scales
+    that fall into fp16's subnormal range (z then differs from the minimum, so
+    codes below z and above the top level are clamped).  Bit-exact like the
+    oracle."""
+    w = W.with_sizes(W.WORKLOADS["tiny"], dtype=dtype, bits=bits)
+    rng = np.random.default_rng(13)
+    S = 300
+    x = rng.normal(0.0, 1.5e-6, (1, 2, S, 64))
+    x[0, 1] += 4e-6
+    k, v = W.to_bits(x, dtype), W.to_bits(x[..., ::-1].copy(), dtype)
+    _run_prefill_bits(w, k, v)
+
+
 def _run_prefill_bits(w, K, V):
     cache = gpu_prefill(w, K, V)
     for b in range(w.batch):
@@ -131,10 +146,12 @@ def _run_prefill_bits(w, K, V):
     assert cache.status() == 0
 
 
-def test_nonfinite_input_sets_status_bit():
+@pytest.mark.parametrize("bad", [0x7C00, 0x7E00])   # fp16 +inf, nan
+def test_nonfinite_input_sets_status_bit(bad):
     w = W.WORKLOADS["tiny"]
     K, V = W.prefill(w, seq_len=256)
-    K[0, 1, 3, 5] = 0x7C00          # fp16 +inf inside the first quantized group
+    K[0, 1, 3, 5] = bad             # inside the first quantized group
+    V[0, 0, 40, 7] = bad            # inside the second
     cache = gpu_prefill(w, K, V)
     bits = cache.status(clear=True)
     assert bits & 1
