@@ -98,7 +98,14 @@ constexpr int kTqThr = kTqLevels + 32;             // float [8] thresholds (7 us
 constexpr int kTqLevels16 = kTqThr + 32;           // fp16 [8] levels
 constexpr int kTqLut = kTqLevels + 128;            // uint32 [64]: fp16x2 (level[lo], level[hi]) of index lo + 8 hi
 constexpr int kTqSPiT = kTqLut + 256;              // float [d][m], transpose of S Pi (the sketch of a rotated query)
-constexpr int kTqParamBytes = kTqSPiT + kTqD * kTqM * 4;
+// Tensor-core operand images of the quantizer's products y = Pi u and S e: four
+// fp16 [128][128] matrices B[n][k] (16 Pi hi, 16 Pi lo, S hi, S lo; hi + lo is
+// the fp32 value), each in the no-swizzle K-major layout of tcgen05.mma: the
+// 8 x 8 core matrix (n / 8, k / 8) at byte 2048 (k / 8) + 128 (n / 8), row n % 8
+// at 16-byte steps.
+constexpr int kTqBImg = kTqSPiT + kTqD * kTqM * 4;
+constexpr int kTqBImgBytes = 32768;                // one image
+constexpr int kTqParamBytes = kTqBImg + 4 * kTqBImgBytes;
 constexpr int kTqQPrepBytes = 2 * (kTqD / 16) * 32 * 16;   // rotated query fragments of one row
 
 __host__ __device__ inline int64_t rec_kscale_off(const Geom& g) { return (int64_t)g.G * g.d * g.bits / 4; }
@@ -272,6 +279,8 @@ void launch_kivi_attention(const AttnArgs& a, cudaStream_t st);
 void launch_clear_words(uint32_t* words, int n, cudaStream_t st);
 void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_gauss, bool wht, cudaStream_t st);
 void launch_tq_quantize(const QuantArgs& a, cudaStream_t st);
+// the tensor-core quantizer (dense rotation, 16-bit sources); launch_tq_quantize routes to it
+void launch_tq_quantize_tc(const QuantArgs& a, cudaStream_t st);
 void launch_tq_query_prep(const Geom& g, const uint16_t* q, unsigned char* qprep, cudaStream_t st);
 void launch_tq_attention(const AttnArgs& a, cudaStream_t st);
 size_t cache_workspace_bytes(const kvq_cache* cache);   // kvq_workspace_bytes of the cache's config

@@ -455,6 +455,10 @@ __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) 
 void launch_tq_quantize(const QuantArgs& a, cudaStream_t st) {
   const int64_t tasks = (int64_t)a.geom.B * a.geom.Hkv * a.n_groups;
   if (tasks <= 0) return;
+  if (!a.geom.rot_wht && a.src_fp8 == nullptr) {   // dense rotation, 16-bit rows: the tensor-core kernel
+    launch_tq_quantize_tc(a, st);
+    return;
+  }
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(tq_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QSmem::BYTES);

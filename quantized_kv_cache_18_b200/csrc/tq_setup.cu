@@ -200,6 +200,22 @@ __global__ void __launch_bounds__(kSetupThreads, 1)
       for (int k = 0; k < D; ++k) acc += (double)ST[k * M + i] * (double)PiG[k * D + j];
       SPiT[e] = (float)acc;
     }
+    // ---------------------------------------------------------------- tcgen05 operand images of 16 Pi and S
+    // (the quantizer scales u by 16 as well, so the lo parts of both stay
+    // clear of fp16 subnormals)
+    __half* img = reinterpret_cast<__half*>(params + kTqBImg);
+    constexpr int kHalves = kTqBImgBytes / 2;
+    for (int e = tid; e < D * D; e += kSetupThreads) {
+      const int n = e / D, k = e - n * D;
+      const int off = ((k >> 3) * 2048 + (n >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) / 2;
+      const float p = 16.f * PiG[n * D + k];   // B[n][k] = 16 Pi[n][k]
+      const float q = ST[k * M + n];           // B[n][k] = S[n][k]
+      const __half ph = __float2half_rn(p), qh = __float2half_rn(q);
+      img[off] = ph;
+      img[kHalves + off] = __float2half_rn(p - __half2float(ph));
+      img[2 * kHalves + off] = qh;
+      img[3 * kHalves + off] = __float2half_rn(q - __half2float(qh));
+    }
   }
   if (flags) atomicOr(&s_flags, flags);
   __syncthreads();
