@@ -19,18 +19,25 @@
 //   D  fp32 in tensor memory: 256 y, then 64 S e.
 // The scalings keep the lo parts clear of fp16 subnormals.
 //
-// Warp roles (288 threads, one persistent CTA per SM):
-//   warps 0-3  keys; thread (w, l) owns token 32 w + l of the tile: norm and
-//              split u; after y its codes, e, ||e||^2 and split e; after S e
-//              its sign bits and (n, gamma)
-//   warps 4-7  values, the same rows: norm, split u, codes, n
-//   warp 8     lane 0 issues the mma chains and commits them to mbarriers
+// Warp roles (544 threads, one persistent CTA per SM):
+//   warps 0-15  token warps: warp w serves the tensor-memory lane quadrant
+//               q = w % 4, so thread (w, l) owns token 32 q + l of the tile,
+//               and r = w / 4 picks keys (r < 2) or values and the half of
+//               the 128 coordinates it handles (r % 2).  The two halves of a
+//               token meet in shared memory for its norm, ||e||^2 and sign
+//               words (a 64-thread named barrier per kind and quadrant).
+//   warp 16     lane 0 issues the mma chains and commits them to mbarriers
+// Keys: norm and split u; after y the codes, e, ||e||^2 and split e; after
+// S e the sign bits and (n, gamma).  Values: norm, split u, codes, n.
 // Tensor memory (512 columns): keys D 0-127, A hi 128-191, A lo 192-255 (e
 // reuses A, S e reuses D); values D 256-383, A hi 384-447, A lo 448-511.  The
 // value chain runs while the key warps code y, the S e chain while the value
-// warps code theirs.  The eight token warps then pack the tile's code words.
-// Every wait is bounded; a wait that gives up sets KVQ_DEV_WAIT_TIMEOUT and
-// the CTA stops at the next tile boundary, after its issued chains complete.
+// warps code theirs.  Key threads write their 6-bit pair indices in record
+// slot order; value threads combine their codes with the next token's (the
+// next lane) into pair indices; the token warps then pack the tile's words.
+// Every wait is bounded and idles with a short sleep instead of spinning; a
+// wait that gives up sets KVQ_DEV_WAIT_TIMEOUT and the CTA stops at the next
+// tile boundary, after its issued chains complete.
 #include <cuda_runtime.h>
 
 #include "kvq_internal.cuh"
@@ -41,17 +48,26 @@ namespace kvq {
 namespace {
 
 constexpr int kTcTok = 128;
-constexpr int kTcThreads = 288;
+constexpr int kTokWarps = 16;
+constexpr int kTokThreads = kTokWarps * 32;
+constexpr int kTcThreads = kTokThreads + 32;
 constexpr int kTcCols = 512;
-constexpr int kCodeRow = 144;   // code tile row stride (bytes): 16-byte aligned rows, 4 banks apart
 
 struct TcSmem {
-  static constexpr int B = 0;                               // 16 Pi hi, 16 Pi lo, S hi, S lo
-  static constexpr int CK = B + 4 * kTqBImgBytes;           // uint8 [128][kCodeRow] key codes
-  static constexpr int CV = CK + kTcTok * kCodeRow;         // uint8 [128][kCodeRow] value codes
-  static constexpr int BYTES = CV + kTcTok * kCodeRow;
+  static constexpr int B = 0;                          // 16 Pi hi, 16 Pi lo, S hi, S lo
+  static constexpr int IK = B + 4 * kTqBImgBytes;      // uint8 [4 blocks][32 lanes][64 slots] key pair indices
+  static constexpr int IV = IK + 4 * 32 * 64;          // uint8 [64 token pairs][128 coordinates] value pair indices
+  static constexpr int NP = IV + 64 * 128;             // double [2 kinds][2 halves][128] partial sums of squares
+  static constexpr int EP = NP + 2 * 2 * 128 * 8;      // float [128] partial ||64 e||^2 of the low half
+  static constexpr int SW = EP + 128 * 4;              // uint32 [128][4] sign words of the low half
+  static constexpr int BYTES = SW + 128 * 16;
 };
 static_assert(TcSmem::BYTES <= 227 * 1024, "TurboQuant tensor-core quantizer exceeds shared memory");
+
+template <bool BF>
+__device__ __forceinline__ float in16f(uint32_t bits16) {
+  return BF ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((uint16_t)bits16));
+}
 
 // fp16 hi + lo split of two fp32 values, packed as fp16x2 pairs
 __device__ __forceinline__ void split_pair(float v0, float v1, uint32_t& hi, uint32_t& lo) {
@@ -60,6 +76,23 @@ __device__ __forceinline__ void split_pair(float v0, float v1, uint32_t& hi, uin
   hi = h2_as_u32(h);
   lo = h2_as_u32(__floats2half2_rn(v0 - hf.x, v1 - hf.y));
 }
+
+// Bounded wait that sleeps between polls (the waits here last microseconds;
+// polling would take issue slots from the warps that work meanwhile).
+__device__ __forceinline__ bool mbar_wait_nap(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(b, parity)) return true;
+  const long long t0 = clock64();
+  uint32_t ns = 32;
+  for (;;) {
+    __nanosleep(ns);
+    if (mbar_try_wait(b, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) return false;
+    if (ns < 256) ns <<= 1;
+  }
+}
+
+__device__ __forceinline__ void bar_pair(int id) { asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory"); }
 
 // The chain D = A_hi B_hi + A_hi B_lo + A_lo B_hi over K = 128.
 __device__ __forceinline__ void issue_product(uint32_t d, uint32_t a_hi, uint32_t a_lo, const unsigned char* b_hi,
@@ -75,74 +108,42 @@ __device__ __forceinline__ void issue_product(uint32_t d, uint32_t a_hi, uint32_
   }
 }
 
-// Loads the thread's token (128 16-bit coordinates; zeros when src is null),
-// returns n = ||x|| and writes (16 u) split hi | lo into its tensor-memory lane.
-__device__ __forceinline__ double load_split_unit(const uint16_t* src, int dtype, uint32_t t_hi, uint32_t t_lo,
-                                                  uint32_t& flags) {
-  uint4 raw[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) raw[i] = src != nullptr ? ldg_nc_v4(src + 8 * i) : make_uint4(0, 0, 0, 0);
-  double s0 = 0.0, s1 = 0.0;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const double x0 = in16_to_float((uint16_t)(w[q] & 0xFFFFu), dtype);
-      const double x1 = in16_to_float((uint16_t)(w[q] >> 16), dtype);
-      s0 = fma(x0, x0, s0);
-      s1 = fma(x1, x1, s1);
-    }
-  }
-  const double s = s0 + s1;
-  if (!isfinite(s)) flags |= KVQ_DEV_NONFINITE_INPUT;
-  const double n = sqrt(s);
-  const float f = n > 0.0 ? (float)(1.0 / n) * 16.f : 0.f;
-#pragma unroll
-  for (int h = 0; h < 4; ++h) {   // 32 coordinates = 16 columns at a time
-    uint32_t hi[16], lo[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 r = raw[4 * h + i];
-      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        split_pair(in16_to_float((uint16_t)(w[q] & 0xFFFFu), dtype) * f, in16_to_float((uint16_t)(w[q] >> 16), dtype) * f,
-                   hi[4 * i + q], lo[4 * i + q]);
-    }
-    tmem_st16(t_hi + 16 * h, hi);
-    tmem_st16(t_lo + 16 * h, lo);
-  }
-  return n;
+__device__ __forceinline__ uint32_t gt_mask(float a, float b) {   // 0xFFFFFFFF if a > b, else 0
+  uint32_t r;
+  asm("set.gt.u32.f32 %0, %1, %2;\n" : "=r"(r) : "f"(a), "f"(b));
+  return r;
 }
-
-// code of 256 y against the thresholds scaled by 256 (ascending; the cell
-// count of thresholds strictly below)
+// code of 256 y against the thresholds scaled by 256 (ascending; the count of
+// thresholds strictly below)
 __device__ __forceinline__ uint32_t cell_of(float acc, const float* t) {
-  uint32_t c = 0;
-#pragma unroll
-  for (int k = 0; k < 7; ++k) c += acc > t[k] ? 1u : 0u;
-  return c;
+  const uint32_t s = (gt_mask(acc, t[0]) + gt_mask(acc, t[1]) + gt_mask(acc, t[2])) +
+                     (gt_mask(acc, t[3]) + gt_mask(acc, t[4]) + gt_mask(acc, t[5])) + gt_mask(acc, t[6]);
+  return 0u - s;
 }
 
+template <bool BF>
 __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ __align__(8) uint64_t bar_b, bar_fin, bar_a[2], bar_d[2];
   __shared__ uint32_t s_tmem, s_flags;
   __shared__ int s_abort;
   __shared__ float s_t256[8], s_lv64[8];
+  __shared__ uint32_t* s_rec[4];   // records of the tile's four tasks (null: none or outside the pool)
 
   const Geom& gm = a.geom;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   unsigned char* sB = smem + TcSmem::B;
-  uint8_t* sCK = smem + TcSmem::CK;
-  uint8_t* sCV = smem + TcSmem::CV;
+  uint8_t* sIK = smem + TcSmem::IK;
+  uint8_t* sIV = smem + TcSmem::IV;
+  double* sNP = reinterpret_cast<double*>(smem + TcSmem::NP);
+  float* sEP = reinterpret_cast<float*>(smem + TcSmem::EP);
+  uint32_t* sSW = reinterpret_cast<uint32_t*>(smem + TcSmem::SW);
 
   if (tid == 0) {
     mbar_init(&bar_b, 1);
     mbar_init(&bar_fin, 1);
-    mbar_init(&bar_a[0], 128);
-    mbar_init(&bar_a[1], 128);
+    mbar_init(&bar_a[0], 256);
+    mbar_init(&bar_a[1], 256);
     mbar_init(&bar_d[0], 1);
     mbar_init(&bar_d[1], 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -164,28 +165,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
   const int64_t n_tiles = (n_tasks + 3) / 4;
   uint32_t flags = 0;
 
-  if (warp == 8) {
+  if (warp == kTokWarps) {
     // ------------------------------------------------------------ mma issue
     if (lane == 0) {
       mbar_expect_tx(&bar_b, 4 * kTqBImgBytes);
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         bulk_g2s(sB + i * kTqBImgBytes, gm.params + kTqBImg + i * kTqBImgBytes, kTqBImgBytes, &bar_b);
-      bool ok = mbar_wait(&bar_b, 0, &s_abort);
+      bool ok = mbar_wait_nap(&bar_b, 0, &s_abort);
       if (!ok) mbar_drain(&bar_b, 0);
       const unsigned char *pi_hi = sB, *pi_lo = sB + kTqBImgBytes;
       const unsigned char *s_hi = sB + 2 * kTqBImgBytes, *s_lo = sB + 3 * kTqBImgBytes;
       int64_t it = 0;
       for (int64_t tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
-        if (!(ok = mbar_wait(&bar_a[0], 0, &s_abort))) break;
+        if (!(ok = mbar_wait_nap(&bar_a[0], 0, &s_abort))) break;
         tc_fence_after();
         issue_product(tbase, tbase + 128, tbase + 192, pi_hi, pi_lo);
         umma_commit(&bar_d[0]);
-        if (!(ok = mbar_wait(&bar_a[1], (uint32_t)(it & 1), &s_abort))) break;
+        if (!(ok = mbar_wait_nap(&bar_a[1], (uint32_t)(it & 1), &s_abort))) break;
         tc_fence_after();
         issue_product(tbase + 256, tbase + 384, tbase + 448, pi_hi, pi_lo);
         umma_commit(&bar_d[1]);
-        if (!(ok = mbar_wait(&bar_a[0], 1, &s_abort))) break;
+        if (!(ok = mbar_wait_nap(&bar_a[0], 1, &s_abort))) break;
         tc_fence_after();
         issue_product(tbase, tbase + 128, tbase + 192, s_hi, s_lo);
         umma_commit(&bar_d[0]);
@@ -200,154 +201,229 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
     }
   } else {
     // ------------------------------------------------------------ token warps
-    const int wg = warp >> 2;                       // 0 keys, 1 values
-    const int m = 32 * (warp & 3) + lane;           // token row of the tile
-    const uint32_t t_d = tbase + ((uint32_t)(32 * (warp & 3)) << 16) + (wg ? 256u : 0u);
+    const int q = warp & 3, r = warp >> 2;
+    const int kind = r >> 1, h = r & 1;           // kind 0 keys, 1 values; coordinate half h
+    const int m = 32 * q + lane;                  // token row of the tile
+    const int tt = m & 31, tbm = m >> 5;          // token of its block, block of the tile
+    const int pair_bar = 1 + 4 * kind + q;        // the two halves of these 32 tokens
+    const uint32_t t_d = tbase + ((uint32_t)(32 * q) << 16) + (kind ? 256u : 0u);
     const uint32_t t_hi = t_d + 128, t_lo = t_d + 192;
     float thr[7];
 #pragma unroll
     for (int k = 0; k < 7; ++k) thr[k] = s_t256[k];
-    const int tt = m & 31;                          // token of its block
     const int entry = 8 * ((tt >> 1) & 3) + 4 * (tt >> 4) + 2 * ((tt >> 3) & 1) + (tt & 1);
+    const double rng = recip(a.n_groups);
     int64_t it = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
-      const int64_t task = tile * 4 + (m >> 5);
+      const int64_t task = tile * 4 + tbm;
       const bool valid = task < n_tasks;
       int row = 0;
       int64_t blk = 0;
       if (valid) {
-        row = (int)(task / a.n_groups);
+        row = (int)div_floor(task, a.n_groups, rng);
         blk = task - (int64_t)row * a.n_groups;
       }
-      const uint16_t* src =
-          valid ? (wg ? a.src_v : a.src_k) + (int64_t)row * a.src_row_stride + (blk * kTB + tt) * kTqD
-                : nullptr;
       unsigned char* dst = valid ? reinterpret_cast<unsigned char*>(record_ptr(gm, row, a.dst_group0 + blk)) : nullptr;
+      if (kind == 0 && h == 0 && tt == 0) {
+        s_rec[tbm] = reinterpret_cast<uint32_t*>(dst);
+        if (valid && dst == nullptr) flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
+      }
 
-      // y: the unit vector into the A operand
-      const double n = load_split_unit(src, gm.dtype, t_hi, t_lo, flags);
+      // ---------------------------------------------------------- u = x / ||x||, split, into the A operand
+      // the token's 64 coordinates are read twice: for the norm, then (from L1) for the split
+      const uint4* src = reinterpret_cast<const uint4*>((kind ? a.src_v : a.src_k) + (int64_t)row * a.src_row_stride +
+                                                        (blk * kTB + tt) * kTqD + 64 * h);
+      double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 rv = valid ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const double x0 = in16f<BF>(w[k] & 0xFFFFu), x1 = in16f<BF>(w[k] >> 16);
+          s0 = fma(x0, x0, s0);
+          s1 = fma(x1, x1, s1);
+        }
+      }
+      sNP[(2 * kind + h) * 128 + m] = s0 + s1;
+      bar_pair(pair_bar);
+      const double ss = sNP[(2 * kind) * 128 + m] + sNP[(2 * kind + 1) * 128 + m];
+      if (h == 0 && !isfinite(ss)) flags |= KVQ_DEV_NONFINITE_INPUT;
+      const double n = sqrt(ss);
+      {
+        const float f = n > 0.0 ? (float)(1.0 / n) * 16.f : 0.f;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {   // 16 coordinates = 8 columns at a time
+          uint32_t hi[8], lo[8];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const uint4 rv = valid ? __ldg(src + 2 * g + i) : make_uint4(0, 0, 0, 0);
+            const uint32_t w[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              split_pair(in16f<BF>(w[k] & 0xFFFFu) * f, in16f<BF>(w[k] >> 16) * f, hi[4 * i + k], lo[4 * i + k]);
+          }
+          tmem_st8(t_hi + 32 * h + 8 * g, hi);
+          tmem_st8(t_lo + 32 * h + 8 * g, lo);
+        }
+      }
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar_a[wg]);
+      mbar_arrive(&bar_a[kind]);
 
-      bool ok = mbar_wait(&bar_d[wg], wg ? (uint32_t)(it & 1) : 0u, &s_abort);
-      if (ok) {
-        tc_fence_after();
-        uint8_t* crow = (wg ? sCV : sCK) + m * kCodeRow;
-        float es0 = 0.f, es1 = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_d + 32 * c, r);
-          tc_wait_ld();
-          uint32_t cw[8], eh[16], el[16];
+      // ---------------------------------------------------------- y: codes (keys also e)
+      // (ok is made warp-uniform: tcgen05.ld / st and the shuffle below are warp-collective)
+      bool ok = __all_sync(0xffffffffu, mbar_wait_nap(&bar_d[kind], kind ? (uint32_t)(it & 1) : 0u, &s_abort));
+      if (!ok) s_abort = 1;
+      if (kind == 0) {
+        float es = 0.f;
+        if (ok) {
+          tc_fence_after();
+          uint32_t kx[4][2];   // pair indices of slots 8 h .. 8 h + 7 of quad lane tc, one byte each
 #pragma unroll
-          for (int p = 0; p < 16; ++p) {
-            const float y0 = __uint_as_float(r[2 * p]), y1 = __uint_as_float(r[2 * p + 1]);
-            const uint32_t c0 = cell_of(y0, thr), c1 = cell_of(y1, thr);
-            const uint32_t pr = c0 | (c1 << 8);
-            if (p & 1) cw[p >> 1] |= pr << 16;
-            else cw[p >> 1] = pr;
-            if (wg == 0) {
+          for (int c = 0; c < 4; ++c) {   // 16 coordinates (8 pairs) at a time
+            uint32_t rr[16];
+            tmem_ld16(t_d + 64 * h + 16 * c, rr);
+            tc_wait_ld();
+            uint32_t eh[8], el[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+              const float y0 = __uint_as_float(rr[2 * p]), y1 = __uint_as_float(rr[2 * p + 1]);
+              const uint32_t c0 = cell_of(y0, thr), c1 = cell_of(y1, thr);
+              // pair 32 h + 8 c + p: quad lane p & 3, slot 8 h + 2 c + p / 4
+              const uint32_t idx = (c0 + 8u * c1) << (8 * (2 * (c & 1) + (p >> 2)));
+              if ((c & 1) == 0 && (p >> 2) == 0) kx[p & 3][c >> 1] = idx;
+              else kx[p & 3][c >> 1] |= idx;
               const float e0 = fmaf(y0, 0.25f, -s_lv64[c0]), e1 = fmaf(y1, 0.25f, -s_lv64[c1]);   // 64 e
-              es0 = fmaf(e0, e0, es0);
-              es1 = fmaf(e1, e1, es1);
+              es = fmaf(e0, e0, es);
+              es = fmaf(e1, e1, es);
               split_pair(e0, e1, eh[p], el[p]);
             }
+            tmem_st8(t_hi + 32 * h + 8 * c, eh);
+            tmem_st8(t_lo + 32 * h + 8 * c, el);
           }
-          *reinterpret_cast<uint4*>(crow + 32 * c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          *reinterpret_cast<uint4*>(crow + 32 * c + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-          if (wg == 0) {
-            tmem_st16(t_hi + 16 * c, eh);
-            tmem_st16(t_lo + 16 * c, el);
-          }
-        }
-        if (wg == 0) {
+          // key pair indices: lane 4 gr + tc of the block, slots 16 nt + 8 h .. + 7
+          uint8_t* ik = sIK + tbm * 2048 + 16 * (tt >> 3) + 8 * h;
+#pragma unroll
+          for (int tc = 0; tc < 4; ++tc)
+            *reinterpret_cast<uint2*>(ik + (4 * (tt & 7) + tc) * 64) = make_uint2(kx[tc][0], kx[tc][1]);
+          if (h == 0) sEP[m] = es;
           // S e: the residual into the A operand, then the signs
           tc_wait_st();
           tc_fence_before();
           mbar_arrive(&bar_a[0]);
-          ok = mbar_wait(&bar_d[0], 1u, &s_abort);
-          if (ok) {
-            tc_fence_after();
-            uint32_t sw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              uint32_t r[32];
-              tmem_ld32(t_d + 32 * c, r);
-              tc_wait_ld();
+          ok = __all_sync(0xffffffffu, mbar_wait_nap(&bar_d[0], 1u, &s_abort));
+          if (!ok) s_abort = 1;
+        }
+        uint32_t sw[4] = {0u, 0u, 0u, 0u};
+        if (ok) {
+          tc_fence_after();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int i = 32 * c + j;   // sketch row: lane tc = (i >> 1) & 3 of the quad, bit 2 kt + rho (+ 16)
-                const uint32_t bit = 1u << (2 * (i >> 4) + ((i >> 3) & 1) + 16 * (i & 1));
-                if (__uint_as_float(r[j]) >= 0.f) sw[(i >> 1) & 3] |= bit;
-              }
-            }
-            const __half hn = __double2half(n);
-            const __half hg = __double2half(n * sqrt((double)(es0 + es1) * (1.0 / 4096.0)));
-            if (isinf(__half2float(hn)) || isinf(__half2float(hg))) flags |= KVQ_DEV_PARAM_OVERFLOW;
-            if (dst != nullptr) {
-              const int nt = tt >> 3, gr = tt & 7;
-              uint32_t* sg = reinterpret_cast<uint32_t*>(dst + kTqSigns);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t rr[16];
+            tmem_ld16(t_d + 64 * h + 16 * c, rr);
+            tc_wait_ld();
 #pragma unroll
-              for (int q = 0; q < 4; ++q) sg[4 * (4 * gr + q) + nt] = sw[q];
-              reinterpret_cast<uint32_t*>(dst + kTqKMeta)[entry] =
-                  (uint32_t)__half_as_ushort(hn) | ((uint32_t)__half_as_ushort(hg) << 16);
+            for (int j = 0; j < 16; ++j) {
+              const int i = 64 * h + 16 * c + j;   // sketch row: quad lane (i >> 1) & 3, bit 2 kt + rho (+ 16)
+              const uint32_t bit = 1u << (2 * (i >> 4) + ((i >> 3) & 1) + 16 * (i & 1));
+              if (__uint_as_float(rr[j]) >= 0.f) sw[(i >> 1) & 3] |= bit;
             }
           }
-        } else {
+        }
+        if (h == 0) *reinterpret_cast<uint4*>(sSW + 4 * m) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+        bar_pair(pair_bar);   // both halves reach it, whatever their waits returned
+        // a half whose wait gave up set s_abort before the barrier: its words are then incomplete
+        const bool both = ok && !s_abort;
+        if (both && h == 1) {
+          const uint4 o = *reinterpret_cast<const uint4*>(sSW + 4 * m);
+          const __half hn = __double2half(n);
+          const __half hg = __double2half(n * sqrt((double)(sEP[m] + es) * (1.0 / 4096.0)));
+          if (isinf(__half2float(hn)) || isinf(__half2float(hg))) flags |= KVQ_DEV_PARAM_OVERFLOW;
+          if (dst != nullptr) {
+            uint32_t* sg = reinterpret_cast<uint32_t*>(dst + kTqSigns) + 4 * (4 * (tt & 7)) + (tt >> 3);
+            sg[0] = sw[0] | o.x;
+            sg[4] = sw[1] | o.y;
+            sg[8] = sw[2] | o.z;
+            sg[12] = sw[3] | o.w;
+            reinterpret_cast<uint32_t*>(dst + kTqKMeta)[entry] =
+                (uint32_t)__half_as_ushort(hn) | ((uint32_t)__half_as_ushort(hg) << 16);
+          }
+        }
+      } else if (ok) {
+        tc_fence_after();
+        uint32_t cw[16];   // codes of coordinates 64 h + 4 k .. + 3, one byte each
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rr[16];
+          tmem_ld16(t_d + 64 * h + 16 * c, rr);
+          tc_wait_ld();
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            const uint32_t pr =
+                cell_of(__uint_as_float(rr[2 * p]), thr) | (cell_of(__uint_as_float(rr[2 * p + 1]), thr) << 8);
+            if (p & 1) cw[4 * c + (p >> 1)] |= pr << 16;
+            else cw[4 * c + (p >> 1)] = pr;
+          }
+        }
+        // value pair indices: this token's codes plus 8 x the next token's (the next lane)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) cw[k] += __shfl_down_sync(0xffffffffu, cw[k], 1) << 3;
+        if ((lane & 1) == 0) {
+          uint4* iv = reinterpret_cast<uint4*>(sIV + (m >> 1) * 128 + 64 * h);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) iv[k] = make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
+        }
+        if (h == 0) {
           const __half hv = __double2half(n);
           if (isinf(__half2float(hv))) flags |= KVQ_DEV_PARAM_OVERFLOW;
           if (dst != nullptr) reinterpret_cast<uint16_t*>(dst + kTqVMeta)[entry] = __half_as_ushort(hv);
         }
       }
-      if (!ok) s_abort = 1;
-      // all 256 token threads agree on stopping before the code tiles are packed
-      if (bar_red_or(1, 256, !ok)) {
+      // all token threads agree on stopping before the tile's words are packed
+      if (bar_red_or(9, kTokThreads, !ok)) {
         flags |= KVQ_DEV_WAIT_TIMEOUT;
         break;
       }
 
       // ---------------------------------------------------------- pack the tile's code words
-      for (int item = tid; item < 4 * 2 * 416; item += 256) {
-        const int tb = item / (2 * 416);
-        const int qw = item - tb * (2 * 416);
-        const int64_t tb_task = tile * 4 + tb;
-        if (tb_task >= n_tasks) continue;
-        const int trow = (int)(tb_task / a.n_groups);
-        const int64_t tblk = tb_task - (int64_t)trow * a.n_groups;
-        uint32_t* out = reinterpret_cast<uint32_t*>(record_ptr(gm, trow, a.dst_group0 + tblk));
-        if (out == nullptr) {
-          flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
-          continue;
-        }
-        const int vblk = qw >= 416;
-        const int q = qw - 416 * vblk;
-        const int ln = q < 384 ? (q >> 2) & 31 : q - 384;
-        const int w = q < 384 ? 4 * (q >> 7) + (q & 3) : 12;
-        const int gr = ln >> 2, tc = ln & 3;
-        const uint8_t* ct = (vblk ? sCV : sCK) + 32 * tb * kCodeRow;
+      // word i of a block's key (value) codes: i < 384 is word 4 (i / 128) + i % 4
+      // of lane (i / 4) % 32, i >= 384 word 12 of lane i - 384
+#pragma unroll 1
+      for (int item = tid; item < 4 * 2 * 416; item += kTokThreads) {
+        const int tb = item / 832, rest = item - 832 * tb;
+        uint32_t* out = s_rec[tb];
+        if (out == nullptr) continue;
+        const int vblk = rest >= 416;
+        const int i = rest - 416 * vblk;
+        const int ln = i < 384 ? (i >> 2) & 31 : i - 384;
+        const int w = i < 384 ? 4 * (i >> 7) + (i & 3) : 12;
         uint32_t word = 0;
+        if (!vblk) {
+          // slots 5 w .. 5 w + 4 of the lane's 64 index bytes
+          const uint8_t* ib = sIK + tb * 2048 + ln * 64;
+          const int b0 = 5 * w;
+          const uint32_t lo = *reinterpret_cast<const uint32_t*>(ib + (b0 & ~3));
+          const uint32_t hi = (b0 & ~3) + 4 < 64 ? *reinterpret_cast<const uint32_t*>(ib + (b0 & ~3) + 4) : 0u;
+          const uint64_t v = ((uint64_t)hi << 32 | lo) >> (8 * (b0 & 3));
 #pragma unroll
-        for (int f = 0; f < 5; ++f) {
-          const int slot = 5 * w + f;
-          if (slot < 64) {
-            uint32_t idx;
-            if (!vblk) {   // key pair (nt, kt, rho): token 8 nt + gr, coordinates 16 kt + 8 rho + 2 tc (+1)
-              const int nt = slot >> 4, kt = (slot >> 1) & 7, rho = slot & 1;
-              const uint8_t* cp = ct + (8 * nt + gr) * kCodeRow + 16 * kt + 8 * rho + 2 * tc;
-              idx = cp[0] + 8u * cp[1];
-            } else {       // value pair (kt, nt, rho): coordinate 8 nt + gr, tokens 16 kt + 8 rho + 2 tc (+1)
-              const int kt = slot >> 5, nt = (slot >> 1) & 15, rho = slot & 1;
-              const uint8_t* cp = ct + (16 * kt + 8 * rho + 2 * tc) * kCodeRow + 8 * nt + gr;
-              idx = cp[0] + 8u * cp[kCodeRow];
+          for (int f = 0; f < 5; ++f) word |= (uint32_t)((v >> (8 * f)) & 0x3Fu) << (6 * f);
+          if (w == 12) word &= 0x00FFFFFFu;   // slots 60..63 only
+        } else {
+          // value pair (kt, nt, rho) of slot s: coordinate 8 nt + gr, token pair 8 kt + 4 rho + tc
+          const int gr = ln >> 2, tc = ln & 3;
+#pragma unroll
+          for (int f = 0; f < 5; ++f) {
+            const int sl = 5 * w + f;
+            if (sl < 64) {
+              const int kt = sl >> 5, nt = (sl >> 1) & 15, rho = sl & 1;
+              word |= (uint32_t)sIV[(16 * tb + 8 * kt + 4 * rho + tc) * 128 + 8 * nt + gr] << (6 * f);
             }
-            word |= idx << (6 * f);
           }
         }
-        out[(vblk ? kTqVCodes : kTqKCodes) / 4 + q] = word;
+        out[(vblk ? kTqVCodes : kTqKCodes) / 4 + i] = word;
       }
-      asm volatile("bar.sync 1, 256;\n" ::: "memory");   // the code tiles are free for the next tile
+      asm volatile("bar.sync 9, %0;\n" ::"r"(kTokThreads) : "memory");   // index tiles free for the next tile
     }
   }
 
@@ -364,14 +440,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
 void launch_tq_quantize_tc(const QuantArgs& a, cudaStream_t st) {
   const int64_t tasks = (int64_t)a.geom.B * a.geom.Hkv * a.n_groups;
   if (tasks <= 0) return;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(tq_quantize_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSmem::BYTES);
-    attr_set = true;
+  auto kern = a.geom.dtype == KVQ_BF16 ? tq_quantize_tc_kernel<true> : tq_quantize_tc_kernel<false>;
+  static bool attr_set[2] = {false, false};
+  const int di = a.geom.dtype == KVQ_BF16;
+  if (!attr_set[di]) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSmem::BYTES);
+    attr_set[di] = true;
   }
   const int64_t tiles = (tasks + 3) / 4;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  tq_quantize_tc_kernel<<<grid, kTcThreads, TcSmem::BYTES, st>>>(a);
+  kern<<<grid, kTcThreads, TcSmem::BYTES, st>>>(a);
   count_launch(1);
 }
 
