@@ -60,8 +60,10 @@ struct TcSmem {
   static constexpr int NP = IV + 64 * 128;             // double [2 kinds][2 halves][128] partial sums of squares
   static constexpr int EP = NP + 2 * 2 * 128 * 8;      // float [128] partial ||64 e||^2 of the low half
   static constexpr int SW = EP + 128 * 4;              // uint32 [128][4] sign words of the low half
-  static constexpr int BYTES = SW + 128 * 16;
+  static constexpr int XS = SW + 128 * 16;             // [2 kinds][128 tokens][kXRow] staged input rows
+  static constexpr int BYTES = XS + 2 * 128 * 272;
 };
+constexpr int kXRow = 272;   // staged row pitch: 256 bytes + 16, so 8 consecutive rows fall 4 banks apart
 static_assert(TcSmem::BYTES <= 227 * 1024, "TurboQuant tensor-core quantizer exceeds shared memory");
 
 template <bool BF>
@@ -93,6 +95,9 @@ __device__ __forceinline__ bool mbar_wait_nap(uint64_t* b, uint32_t parity, vola
 }
 
 __device__ __forceinline__ void bar_pair(int id) { asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory"); }
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
 
 // The chain D = A_hi B_hi + A_hi B_lo + A_lo B_hi over K = 128.
 __device__ __forceinline__ void issue_product(uint32_t d, uint32_t a_hi, uint32_t a_lo, const unsigned char* b_hi,
@@ -213,6 +218,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
     for (int k = 0; k < 7; ++k) thr[k] = s_t256[k];
     const int entry = 8 * ((tt >> 1) & 3) + 4 * (tt >> 4) + 2 * ((tt >> 3) & 1) + (tt & 1);
     const double rng = recip(a.n_groups);
+    // The thread's half row of a tile is staged with cp.async one tile ahead,
+    // into a shared-memory region only this thread reads.
+    unsigned char* xs = smem + TcSmem::XS + (kind * 128 + m) * kXRow + 128 * h;
+    auto stage_rows = [&](int64_t t) {
+      const int64_t tk = t * 4 + tbm;
+      if (t < n_tiles && tk < n_tasks) {
+        const int rw = (int)div_floor(tk, a.n_groups, rng);
+        const int64_t bk = tk - (int64_t)rw * a.n_groups;
+        const uint16_t* g = (kind ? a.src_v : a.src_k) + (int64_t)rw * a.src_row_stride + (bk * kTB + tt) * kTqD + 64 * h;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cp_async16(xs + 16 * i, g + 8 * i);
+      }
+      asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+    stage_rows(blockIdx.x);
     int64_t it = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       const int64_t task = tile * 4 + tbm;
@@ -230,13 +250,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
       }
 
       // ---------------------------------------------------------- u = x / ||x||, split, into the A operand
-      // the token's 64 coordinates are read twice: for the norm, then (from L1) for the split
-      const uint4* src = reinterpret_cast<const uint4*>((kind ? a.src_v : a.src_k) + (int64_t)row * a.src_row_stride +
-                                                        (blk * kTB + tt) * kTqD + 64 * h);
+      // the staged 64 coordinates are read twice: for the norm, then for the split
+      asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+      const uint4* src = reinterpret_cast<const uint4*>(xs);
       double s0 = 0.0, s1 = 0.0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const uint4 rv = valid ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+        const uint4 rv = valid ? src[i] : make_uint4(0, 0, 0, 0);
         const uint32_t w[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -257,7 +277,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
           uint32_t hi[8], lo[8];
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
-            const uint4 rv = valid ? __ldg(src + 2 * g + i) : make_uint4(0, 0, 0, 0);
+            const uint4 rv = valid ? src[2 * g + i] : make_uint4(0, 0, 0, 0);
             const uint32_t w[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k)
@@ -267,6 +287,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
           tmem_st8(t_lo + 32 * h + 8 * g, lo);
         }
       }
+      stage_rows(tile + gridDim.x);   // this thread's staged rows are consumed
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_a[kind]);
@@ -425,6 +446,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
       }
       asm volatile("bar.sync 9, %0;\n" ::"r"(kTokThreads) : "memory");   // index tiles free for the next tile
     }
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");   // no staging copy outlives the loop
   }
 
   if (flags) atomicOr(&s_flags, flags);
