@@ -28,37 +28,20 @@ __device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bits) {
 }
 
 // Codes are round half to even of (x - z) / s, clamped to [0, levels], with
-// s, z the fp16 scale and zero-point.  The fp32 estimate r = fma(x, 1/s, -z/s)
-// differs from the exact quotient by less than 2^-24 (2 levels + |z| / s) up to
-// second-order terms (one rounding each in 1/s, z/s and the fma; r is only used
-// where it lies in [0, levels]); eb below is four times that.  An estimate more
-// than eb away from every rounding boundary k + 1/2 decides.  Within eb, which
-// takes in the exact ties that 16-bit inputs and fp16 scales often produce, the
-// exact double-precision comparison of 2 (x - z) with (2k + 1) s decides.
-struct CodeParams {
-  float s, z, inv, zinv, eb;
-};
-__device__ __forceinline__ CodeParams code_params(float s, float z, int levels) {
-  CodeParams p;
-  p.s = s;
-  p.z = z;
-  p.inv = s > 0.f ? 1.f / s : 0.f;
-  p.zinv = z * p.inv;
-  p.eb = 2.384185791015625e-7f * (2.f * (float)levels + 2.f + fabsf(p.zinv));   // 2^-22 (...)
-  return p;
-}
+// s, z the fp16 scale and zero-point.  4-bit codes start from the fp32
+// estimate r = fma(x, 1/s, -z/s), which differs from the exact quotient by less
+// than 2^-24 (2 levels + |z| / s) up to second-order terms (one rounding each
+// in 1/s, z/s and the fma); eb = 4 times that.  An estimate more than eb away
+// from every rounding boundary k + 1/2 decides.  Within eb, which takes in the
+// exact ties that 16-bit inputs and fp16 scales often produce, the exact
+// double-precision comparison of 2 (x - z) with (2k + 1) s decides.  (2-bit
+// codes are decided exactly by 16-bit thresholds, below.)
+//
 // The exact decision, out of line: it runs for a small fraction of the
 // elements, and inlining it at every call site bloated the kernel's code
 // (instruction-cache misses were its top stall).
 __device__ __noinline__ uint32_t code_exact(float x, float z, float s, int levels) {
   return (uint32_t)exact_code((double)x, (double)z, (double)s, s > 0.f ? 1.0 / (double)s : 0.0, levels);
-}
-__device__ __forceinline__ uint32_t code_of(float x, const CodeParams& p, int levels) {
-  float r = fmaf(x, p.inv, -p.zinv);
-  r = fminf(fmaxf(r, 0.f), (float)levels);   // also maps NaN to 0
-  const float k = rintf(r);
-  if (fabsf(fabsf(r - k) - 0.5f) > p.eb) return (uint32_t)k;
-  return code_exact(x, p.z, p.s, levels);
 }
 
 // ------------------------------------------------------------------ per-unit parameters
@@ -106,7 +89,7 @@ __device__ __forceinline__ uint16_t threshold16(double X, bool strict) {
 // which is round half to even of (x - z) / s clamped to [0, 3]; X_k is exact
 // in double, so each test becomes "x >= c_k" for one 16-bit constant.  s == 0
 // gives code 0 (thresholds +inf).  4-bit codes use the fp32 estimate described
-// at code_of, with thr = 0.5 - eb, or -1 (every code decided exactly) when z is
+// above, with thr = 0.5 - eb, or -1 (every code decided exactly) when z is
 // far enough from min, or s small enough against max - z, that an estimate
 // could leave [0, 15].
 template <int BITS, bool BF>
@@ -175,6 +158,15 @@ __device__ __forceinline__ void code_pair4(uint32_t x, float inv0, float zinv0, 
   ok = ok && fabsf(r0 - k0) < thr && fabsf(r1 - k1) < thr;
   acc0 = fmaf(k0, kPos, acc0);
   acc1 = fmaf(k1, kPos, acc1);
+}
+
+// One 4-bit code of the fallback path: the estimate when it decides (thr as in
+// code_pair4; thr < 0 decides nothing), else the exact decision with (s, z).
+__device__ __forceinline__ uint32_t estimate_or_exact(float x, float inv, float zinv, float thr, float2 sz, int levels) {
+  constexpr float kRound = 12582912.f;
+  const float r = fmaf(x, inv, -zinv);
+  const float k = (r + kRound) - kRound;
+  return fabsf(r - k) < thr ? (uint32_t)k : code_exact(x, sz.y, sz.x, levels);
 }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -377,13 +369,13 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
           for (int j = 0; j < PAIRS; ++j)
             code_pair4<BF>(x[j], inv[2 * j], zinv[2 * j], inv[2 * j + 1], zinv[2 * j + 1], thr, acc0, acc1, ok, j);
           uint32_t wd = __byte_perm(__float_as_uint(acc0), __float_as_uint(acc1), 0x5410);
-          if (!ok) {
+          if (!ok) {   // redo the word: the estimate where it decides, the exact decision elsewhere
             wd = 0;
             for (int j = 0; j < PAIRS; ++j)
               for (int e = 0; e < 2; ++e) {
                 const int c = cbase + 8 * j + e;
                 const float xv = e ? PT::hi(PT::of(x[j])) : PT::lo(PT::of(x[j]));
-                wd |= code_of(xv, code_params(ksz[c].x, ksz[c].y, L), L) << (16 * e + BITS * j);
+                wd |= estimate_or_exact(xv, inv[2 * j + e], zinv[2 * j + e], thr, ksz[c], L) << (16 * e + BITS * j);
               }
           }
           *word_at(false, tb, nt * WPT + sub) = wd;
@@ -435,13 +427,13 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
           for (int j = 0; j < PAIRS; ++j)
             code_pair4<BF>(x[j], inv[2 * j], zinv[2 * j], inv[2 * j + 1], zinv[2 * j + 1], thr, acc0, acc1, ok, j);
           uint32_t wd = __byte_perm(__float_as_uint(acc0), __float_as_uint(acc1), 0x5410);
-          if (!ok) {
+          if (!ok) {   // redo the word: the estimate where it decides, the exact decision elsewhere
             wd = 0;
             for (int j = 0; j < PAIRS; ++j)
               for (int e = 0; e < 2; ++e) {
                 const int t = tb * kTB + 8 * j + 2 * tc + e;
                 const float xv = e ? PT::hi(PT::of(x[j])) : PT::lo(PT::of(x[j]));
-                wd |= code_of(xv, code_params(vsz[t].x, vsz[t].y, L), L) << (16 * e + BITS * j);
+                wd |= estimate_or_exact(xv, inv[2 * j + e], zinv[2 * j + e], thr, vsz[t], L) << (16 * e + BITS * j);
               }
           }
           *word_at(true, tb, w) = wd;

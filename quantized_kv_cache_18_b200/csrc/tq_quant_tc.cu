@@ -55,15 +55,19 @@ constexpr int kTcCols = 512;
 
 struct TcSmem {
   static constexpr int B = 0;                          // 16 Pi hi, 16 Pi lo, S hi, S lo
-  static constexpr int IK = B + 4 * kTqBImgBytes;      // uint8 [4 blocks][32 lanes][64 slots] key pair indices
-  static constexpr int IV = IK + 4 * 32 * 64;          // uint8 [64 token pairs][128 coordinates] value pair indices
-  static constexpr int NP = IV + 64 * 128;             // double [2 kinds][2 halves][128] partial sums of squares
+  static constexpr int IK = B + 4 * kTqBImgBytes;      // uint8 [4 blocks][32 lanes][kIKRow] key pair indices (64 slots)
+  static constexpr int IV = IK + 4 * 32 * 72;          // uint8 [64 token pairs][kIVRow] value pair indices (128 coordinates)
+  static constexpr int NP = IV + 64 * 144;             // double [2 kinds][2 halves][128] partial sums of squares
   static constexpr int EP = NP + 2 * 2 * 128 * 8;      // float [128] partial ||64 e||^2 of the low half
   static constexpr int SW = EP + 128 * 4;              // uint32 [128][4] sign words of the low half
   static constexpr int XS = SW + 128 * 16;             // [2 kinds][128 tokens][kXRow] staged input rows
   static constexpr int BYTES = XS + 2 * 128 * 272;
 };
 constexpr int kXRow = 272;   // staged row pitch: 256 bytes + 16, so 8 consecutive rows fall 4 banks apart
+// index tile pitches, padded so that the lanes of a packing or index-writing
+// warp spread over the banks instead of hitting one column
+constexpr int kIKRow = 72;
+constexpr int kIVRow = 144;
 static_assert(TcSmem::BYTES <= 227 * 1024, "TurboQuant tensor-core quantizer exceeds shared memory");
 
 template <bool BF>
@@ -324,10 +328,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
             tmem_st8(t_lo + 32 * h + 8 * c, el);
           }
           // key pair indices: lane 4 gr + tc of the block, slots 16 nt + 8 h .. + 7
-          uint8_t* ik = sIK + tbm * 2048 + 16 * (tt >> 3) + 8 * h;
+          uint8_t* ik = sIK + tbm * 32 * kIKRow + 16 * (tt >> 3) + 8 * h;
 #pragma unroll
           for (int tc = 0; tc < 4; ++tc)
-            *reinterpret_cast<uint2*>(ik + (4 * (tt & 7) + tc) * 64) = make_uint2(kx[tc][0], kx[tc][1]);
+            *reinterpret_cast<uint2*>(ik + (4 * (tt & 7) + tc) * kIKRow) = make_uint2(kx[tc][0], kx[tc][1]);
           if (h == 0) sEP[m] = es;
           // S e: the residual into the A operand, then the signs
           tc_wait_st();
@@ -391,7 +395,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
 #pragma unroll
         for (int k = 0; k < 16; ++k) cw[k] += __shfl_down_sync(0xffffffffu, cw[k], 1) << 3;
         if ((lane & 1) == 0) {
-          uint4* iv = reinterpret_cast<uint4*>(sIV + (m >> 1) * 128 + 64 * h);
+          uint4* iv = reinterpret_cast<uint4*>(sIV + (m >> 1) * kIVRow + 64 * h);
 #pragma unroll
           for (int k = 0; k < 4; ++k) iv[k] = make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
         }
@@ -422,7 +426,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
         uint32_t word = 0;
         if (!vblk) {
           // slots 5 w .. 5 w + 4 of the lane's 64 index bytes
-          const uint8_t* ib = sIK + tb * 2048 + ln * 64;
+          const uint8_t* ib = sIK + tb * 32 * kIKRow + ln * kIKRow;
           const int b0 = 5 * w;
           const uint32_t lo = *reinterpret_cast<const uint32_t*>(ib + (b0 & ~3));
           const uint32_t hi = (b0 & ~3) + 4 < 64 ? *reinterpret_cast<const uint32_t*>(ib + (b0 & ~3) + 4) : 0u;
@@ -438,7 +442,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
             const int sl = 5 * w + f;
             if (sl < 64) {
               const int kt = sl >> 5, nt = (sl >> 1) & 15, rho = sl & 1;
-              word |= (uint32_t)sIV[(16 * tb + 8 * kt + 4 * rho + tc) * 128 + 8 * nt + gr] << (6 * f);
+              word |= (uint32_t)sIV[(16 * tb + 8 * kt + 4 * rho + tc) * kIVRow + 8 * nt + gr] << (6 * f);
             }
           }
         }
