@@ -98,14 +98,16 @@ constexpr int kTqThr = kTqLevels + 32;             // float [8] thresholds (7 us
 constexpr int kTqLevels16 = kTqThr + 32;           // fp16 [8] levels
 constexpr int kTqLut = kTqLevels + 128;            // uint32 [64]: fp16x2 (level[lo], level[hi]) of index lo + 8 hi
 constexpr int kTqSPiT = kTqLut + 256;              // float [d][m], transpose of S Pi (the sketch of a rotated query)
-// Tensor-core operand images of the quantizer's products y = Pi u and S e: four
-// fp16 [128][128] matrices B[n][k] (16 Pi hi, 16 Pi lo, S hi, S lo; hi + lo is
-// the fp32 value), each in the no-swizzle K-major layout of tcgen05.mma: the
-// 8 x 8 core matrix (n / 8, k / 8) at byte 2048 (k / 8) + 128 (n / 8), row n % 8
-// at 16-byte steps.
+// Tensor-core operand images of the quantizer's products 16 Pi x and S e: two
+// sets of four [128][128] matrices B[n][k] (16 Pi hi, 16 Pi lo, S hi, S lo; hi
+// + lo approximates the fp32 value), the first in fp16 (for fp16 inputs), the
+// second in bf16 (for bf16 inputs: an mma takes A and B of one type), each in
+// the no-swizzle K-major layout of tcgen05.mma: the 8 x 8 core matrix
+// (n / 8, k / 8) at byte 2048 (k / 8) + 128 (n / 8), row n % 8 at 16-byte steps.
 constexpr int kTqBImg = kTqSPiT + kTqD * kTqM * 4;
 constexpr int kTqBImgBytes = 32768;                // one image
-constexpr int kTqParamBytes = kTqBImg + 4 * kTqBImgBytes;
+constexpr int kTqBImgSet = 4 * kTqBImgBytes;       // one set; the bf16 set follows the fp16 one
+constexpr int kTqParamBytes = kTqBImg + 2 * kTqBImgSet;
 constexpr int kTqQPrepBytes = 2 * (kTqD / 16) * 32 * 16;   // rotated query fragments of one row
 
 __host__ __device__ inline int64_t rec_kscale_off(const Geom& g) { return (int64_t)g.G * g.d * g.bits / 4; }

@@ -66,9 +66,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16 with fp32 accumulation: A
-// and B fp16, both K-major, M x N.
-__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N) {
-  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// and B both fp16 (bf = false) or both bf16, both K-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool bf = false) {
+  return (1u << 4) | ((uint32_t)bf << 7) | ((uint32_t)bf << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
 }
 // Shared-memory matrix descriptor, no swizzle: core matrices of 8 rows x 16
 // bytes; lbo is the byte stride between core matrices along K, sbo between

@@ -2,21 +2,25 @@
 // rotation, 16-bit sources).  The arithmetic and the readings are those of
 // tq_quantize_kernel in tq_quant.cu ("Quantification du KV-Cache : TurboQuant
 // et l'etat de l'art en 2026", "TurboQuant : les cinq innovations", items 1-3):
-// n = ||x|| (fp64 sum), u = x / n, y = Pi u to about fp32 precision, the 3-bit
+// n = ||x|| (fp64 sum), y = Pi x / n to about fp32 precision, the 3-bit
 // Lloyd-Max cell of each coordinate of y (a coordinate equal to a threshold
 // goes to the lower cell), the residual e = y - c_hat in rotated coordinates,
 // the signs of S e (exactly 0 gives bit 1) and gamma = n ||e||.
 //
 // A tile is 128 tokens: four 32-token blocks (tasks) in task order.  Each
 // product is one chain of tcgen05.mma over the whole tile (M = 128 tokens,
-// N = 128 outputs, K = 128 summed coordinates in 8 steps of 16), as three fp16
-// terms hi*hi + hi*lo + lo*hi accumulated in fp32 (the dropped lo*lo term is
-// below 2^-22 of each product):
-//   A  (16 u) or (64 e) split into fp16 hi + lo, in tensor memory, one lane
-//      per token, written by the thread that owns the token;
-//   B  16 Pi and S split the same way, images from the parameter block kept
-//      in shared memory for the whole launch;
-//   D  fp32 in tensor memory: 256 y, then 64 S e.
+// N = 128 outputs, K = 128 summed coordinates in 8 steps of 16), in the
+// input's 16-bit type with fp32 accumulation:
+//   16 Pi x = x (16 Pi hi) + x (16 Pi lo): the input x is exact in its own type,
+//      so A needs no split and y = (16 Pi x) / (16 n) is divided out in the
+//      thresholds and the residual (per-token constants);
+//   64 S e = eh Sh + eh Sl + el Sh with (64 e) split into hi + lo (the dropped
+//      lo*lo term is below 2^-16 of each product in bf16, 2^-22 in fp16).
+//   A  x, or the split 64 e, in tensor memory, one lane per token, written by
+//      the thread that owns the token;
+//   B  images of 16 Pi and S split hi + lo in the input's type, from the
+//      parameter block, kept in shared memory for the whole launch;
+//   D  fp32 in tensor memory.
 // The scalings keep the lo parts clear of fp16 subnormals.
 //
 // Warp roles (544 threads, one persistent CTA per SM):
@@ -27,8 +31,8 @@
 //               token meet in shared memory for its norm, ||e||^2 and sign
 //               words (a 64-thread named barrier per kind and quadrant).
 //   warp 16     lane 0 issues the mma chains and commits them to mbarriers
-// Keys: norm and split u; after y the codes, e, ||e||^2 and split e; after
-// S e the sign bits and (n, gamma).  Values: norm, split u, codes, n.
+// Keys: norm and x into A; after y the codes, e, ||e||^2 and split e; after
+// S e the sign bits and (n, gamma).  Values: norm, x into A, codes, n.
 // Tensor memory (512 columns): keys D 0-127, A hi 128-191, A lo 192-255 (e
 // reuses A, S e reuses D); values D 256-383, A hi 384-447, A lo 448-511.  The
 // value chain runs while the key warps code y, the S e chain while the value
@@ -75,12 +79,21 @@ __device__ __forceinline__ float in16f(uint32_t bits16) {
   return BF ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((uint16_t)bits16));
 }
 
-// fp16 hi + lo split of two fp32 values, packed as fp16x2 pairs
+// hi + lo split of two fp32 values in the 16-bit type (fp16, or bf16), packed as pairs
+template <bool BF>
 __device__ __forceinline__ void split_pair(float v0, float v1, uint32_t& hi, uint32_t& lo) {
-  const __half2 h = __floats2half2_rn(v0, v1);
-  const float2 hf = __half22float2(h);
-  hi = h2_as_u32(h);
-  lo = h2_as_u32(__floats2half2_rn(v0 - hf.x, v1 - hf.y));
+  if constexpr (BF) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+  } else {
+    const __half2 h = __floats2half2_rn(v0, v1);
+    const float2 hf = __half22float2(h);
+    hi = h2_as_u32(h);
+    lo = h2_as_u32(__floats2half2_rn(v0 - hf.x, v1 - hf.y));
+  }
 }
 
 // Bounded wait that sleeps between polls (the waits here last microseconds;
@@ -103,17 +116,18 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
 
-// The chain D = A_hi B_hi + A_hi B_lo + A_lo B_hi over K = 128.
+// The chain D = A_hi B_hi + A_hi B_lo (+ A_lo B_hi when SPLIT_A) over K = 128.
+template <bool BF, bool SPLIT_A>
 __device__ __forceinline__ void issue_product(uint32_t d, uint32_t a_hi, uint32_t a_lo, const unsigned char* b_hi,
                                               const unsigned char* b_lo) {
-  constexpr uint32_t idesc = umma_idesc_f16(kTcTok, kTqD);
+  constexpr uint32_t idesc = umma_idesc_f16(kTcTok, kTqD, BF);
 #pragma unroll
   for (int kk = 0; kk < kTqD / 16; ++kk) {
     const uint64_t bh = umma_sdesc(b_hi + kk * 4096, 2048, 128);
     const uint64_t bl = umma_sdesc(b_lo + kk * 4096, 2048, 128);
     umma_ts(d, a_hi + 8 * kk, bh, idesc, kk > 0);
     umma_ts(d, a_hi + 8 * kk, bl, idesc, true);
-    umma_ts(d, a_lo + 8 * kk, bh, idesc, true);
+    if (SPLIT_A) umma_ts(d, a_lo + 8 * kk, bh, idesc, true);
   }
 }
 
@@ -122,12 +136,16 @@ __device__ __forceinline__ uint32_t gt_mask(float a, float b) {   // 0xFFFFFFFF 
   asm("set.gt.u32.f32 %0, %1, %2;\n" : "=r"(r) : "f"(a), "f"(b));
   return r;
 }
-// code of 256 y against the thresholds scaled by 256 (ascending; the count of
-// thresholds strictly below)
-__device__ __forceinline__ uint32_t cell_of(float acc, const float* t) {
-  const uint32_t s = (gt_mask(acc, t[0]) + gt_mask(acc, t[1]) + gt_mask(acc, t[2])) +
-                     (gt_mask(acc, t[3]) + gt_mask(acc, t[4]) + gt_mask(acc, t[5])) + gt_mask(acc, t[6]);
-  return 0u - s;
+// 3-bit cell of a coordinate from d = 16 n y and the thresholds T4 < T5 < T6
+// of the positive half scaled the same way.  The deployed codebook is
+// symmetric (T_{6-k} = -T_k, T3 = 0; the setup makes it so), so the cell is
+// 4 + #{T_k < d} for d > 0 and 3 - #{T_k < |d|} otherwise.  (A negative d
+// exactly on a threshold would take the upper of the two cells; such a d lies
+// within the rounding error of the exact coordinate, where either is accepted.)
+__device__ __forceinline__ uint32_t cell_sym(float d, float t4, float t5, float t6) {
+  const float ad = fabsf(d);
+  const uint32_t s = gt_mask(ad, t4) + gt_mask(ad, t5) + gt_mask(ad, t6);   // minus the count
+  return d > 0.f ? 4u - s : 3u + s;
 }
 
 template <bool BF>
@@ -180,7 +198,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
       mbar_expect_tx(&bar_b, 4 * kTqBImgBytes);
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        bulk_g2s(sB + i * kTqBImgBytes, gm.params + kTqBImg + i * kTqBImgBytes, kTqBImgBytes, &bar_b);
+        bulk_g2s(sB + i * kTqBImgBytes, gm.params + kTqBImg + (BF ? kTqBImgSet : 0) + i * kTqBImgBytes, kTqBImgBytes,
+                 &bar_b);
       bool ok = mbar_wait_nap(&bar_b, 0, &s_abort);
       if (!ok) mbar_drain(&bar_b, 0);
       const unsigned char *pi_hi = sB, *pi_lo = sB + kTqBImgBytes;
@@ -189,15 +208,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
       for (int64_t tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
         if (!(ok = mbar_wait_nap(&bar_a[0], 0, &s_abort))) break;
         tc_fence_after();
-        issue_product(tbase, tbase + 128, tbase + 192, pi_hi, pi_lo);
+        issue_product<BF, false>(tbase, tbase + 128, tbase + 192, pi_hi, pi_lo);
         umma_commit(&bar_d[0]);
         if (!(ok = mbar_wait_nap(&bar_a[1], (uint32_t)(it & 1), &s_abort))) break;
         tc_fence_after();
-        issue_product(tbase + 256, tbase + 384, tbase + 448, pi_hi, pi_lo);
+        issue_product<BF, false>(tbase + 256, tbase + 384, tbase + 448, pi_hi, pi_lo);
         umma_commit(&bar_d[1]);
         if (!(ok = mbar_wait_nap(&bar_a[0], 1, &s_abort))) break;
         tc_fence_after();
-        issue_product(tbase, tbase + 128, tbase + 192, s_hi, s_lo);
+        issue_product<BF, true>(tbase, tbase + 128, tbase + 192, s_hi, s_lo);
         umma_commit(&bar_d[0]);
       }
       if (!ok) {
@@ -217,9 +236,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
     const int pair_bar = 1 + 4 * kind + q;        // the two halves of these 32 tokens
     const uint32_t t_d = tbase + ((uint32_t)(32 * q) << 16) + (kind ? 256u : 0u);
     const uint32_t t_hi = t_d + 128, t_lo = t_d + 192;
-    float thr[7];
-#pragma unroll
-    for (int k = 0; k < 7; ++k) thr[k] = s_t256[k];
+    const float t4 = s_t256[4], t5 = s_t256[5], t6 = s_t256[6];   // thresholds x 256 (positive half)
     const int entry = 8 * ((tt >> 1) & 3) + 4 * (tt >> 4) + 2 * ((tt >> 3) & 1) + (tt & 1);
     const double rng = recip(a.n_groups);
     // The thread's half row of a tile is staged with cp.async one tile ahead,
@@ -253,8 +270,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
         if (valid && dst == nullptr) flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
       }
 
-      // ---------------------------------------------------------- u = x / ||x||, split, into the A operand
-      // the staged 64 coordinates are read twice: for the norm, then for the split
+      // ---------------------------------------------------------- ||x|| and x into the A operand
       asm volatile("cp.async.wait_group 0;\n" ::: "memory");
       const uint4* src = reinterpret_cast<const uint4*>(xs);
       double s0 = 0.0, s1 = 0.0;
@@ -269,28 +285,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
           s1 = fma(x1, x1, s1);
         }
       }
+      // the raw 16-bit pairs are the A operand as they stand (coordinate pair j = column j)
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        uint32_t xv[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 rv = valid ? src[4 * g + i] : make_uint4(0, 0, 0, 0);
+          xv[4 * i] = rv.x;
+          xv[4 * i + 1] = rv.y;
+          xv[4 * i + 2] = rv.z;
+          xv[4 * i + 3] = rv.w;
+        }
+        tmem_st16(t_hi + 32 * h + 16 * g, xv);
+      }
       sNP[(2 * kind + h) * 128 + m] = s0 + s1;
       bar_pair(pair_bar);
       const double ss = sNP[(2 * kind) * 128 + m] + sNP[(2 * kind + 1) * 128 + m];
       if (h == 0 && !isfinite(ss)) flags |= KVQ_DEV_NONFINITE_INPUT;
       const double n = sqrt(ss);
-      {
-        const float f = n > 0.0 ? (float)(1.0 / n) * 16.f : 0.f;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {   // 16 coordinates = 8 columns at a time
-          uint32_t hi[8], lo[8];
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const uint4 rv = valid ? src[2 * g + i] : make_uint4(0, 0, 0, 0);
-            const uint32_t w[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              split_pair(in16f<BF>(w[k] & 0xFFFFu) * f, in16f<BF>(w[k] >> 16) * f, hi[4 * i + k], lo[4 * i + k]);
-          }
-          tmem_st8(t_hi + 32 * h + 8 * g, hi);
-          tmem_st8(t_lo + 32 * h + 8 * g, lo);
-        }
-      }
+      // D = 16 n y: thresholds 16 n t_k (the table holds 256 t_k), and 64 y = D * 4 / n
+      const float tn = (float)(n * (1.0 / 16.0));
+      const float T4 = tn * t4, T5 = tn * t5, T6 = tn * t6;
+      const float c4 = n > 0.0 ? (float)(4.0 / n) : 0.f;
       stage_rows(tile + gridDim.x);   // this thread's staged rows are consumed
       tc_wait_st();
       tc_fence_before();
@@ -313,16 +330,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
             uint32_t eh[8], el[8];
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-              const float y0 = __uint_as_float(rr[2 * p]), y1 = __uint_as_float(rr[2 * p + 1]);
-              const uint32_t c0 = cell_of(y0, thr), c1 = cell_of(y1, thr);
+              const float y0 = __uint_as_float(rr[2 * p]), y1 = __uint_as_float(rr[2 * p + 1]);   // 16 n y
+              const uint32_t c0 = cell_sym(y0, T4, T5, T6), c1 = cell_sym(y1, T4, T5, T6);
               // pair 32 h + 8 c + p: quad lane p & 3, slot 8 h + 2 c + p / 4
               const uint32_t idx = (c0 + 8u * c1) << (8 * (2 * (c & 1) + (p >> 2)));
               if ((c & 1) == 0 && (p >> 2) == 0) kx[p & 3][c >> 1] = idx;
               else kx[p & 3][c >> 1] |= idx;
-              const float e0 = fmaf(y0, 0.25f, -s_lv64[c0]), e1 = fmaf(y1, 0.25f, -s_lv64[c1]);   // 64 e
+              const float e0 = fmaf(y0, c4, -s_lv64[c0]), e1 = fmaf(y1, c4, -s_lv64[c1]);   // 64 e
               es = fmaf(e0, e0, es);
               es = fmaf(e1, e1, es);
-              split_pair(e0, e1, eh[p], el[p]);
+              split_pair<BF>(e0, e1, eh[p], el[p]);
             }
             tmem_st8(t_hi + 32 * h + 8 * c, eh);
             tmem_st8(t_lo + 32 * h + 8 * c, el);
@@ -385,8 +402,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
           tc_wait_ld();
 #pragma unroll
           for (int p = 0; p < 8; ++p) {
-            const uint32_t pr =
-                cell_of(__uint_as_float(rr[2 * p]), thr) | (cell_of(__uint_as_float(rr[2 * p + 1]), thr) << 8);
+            const uint32_t pr = cell_sym(__uint_as_float(rr[2 * p]), T4, T5, T6) |
+                                (cell_sym(__uint_as_float(rr[2 * p + 1]), T4, T5, T6) << 8);
             if (p & 1) cw[4 * c + (p >> 1)] |= pr << 16;
             else cw[4 * c + (p >> 1)] = pr;
           }

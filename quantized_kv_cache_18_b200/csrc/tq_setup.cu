@@ -17,6 +17,7 @@
 //                      q'' = (S Pi) q for the row's query heads, split into
 //                      fp16 hi + lo and stored in the A-fragment order of the
 //                      decode kernel.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "kvq_internal.cuh"
@@ -168,8 +169,13 @@ __global__ void __launch_bounds__(kSetupThreads, 1)
       c = nc;
       if (diff < 1e-15) break;
     }
-    // deployed: fp16 levels of N(0, 1/d); midpoints are exact in fp32
-    const __half h = __double2half(c / sqrt((double)D));
+    // deployed: fp16 levels of N(0, 1/d); midpoints are exact in fp32.  The
+    // quantizer is odd-symmetric; the lower four levels are taken as the
+    // negatives of the upper four, so the deployed thresholds are exactly
+    // symmetric with the middle one 0 (the tensor-core quantizer relies on it).
+    const uint16_t hu = __half_as_ushort(__double2half(c / sqrt((double)D)));
+    const uint16_t hm = __shfl_sync(0xffffffffu, hu, 7 - l, 8);
+    const __half h = __ushort_as_half(l < 4 ? (uint16_t)(hm ^ 0x8000u) : hu);
     const float lv = __half2float(h);
     const float lv_next = __shfl_down_sync(0xffffffffu, lv, 1, 8);
     float* levels = reinterpret_cast<float*>(params + kTqLevels);
@@ -204,6 +210,7 @@ __global__ void __launch_bounds__(kSetupThreads, 1)
     // (the quantizer scales u by 16 as well, so the lo parts of both stay
     // clear of fp16 subnormals)
     __half* img = reinterpret_cast<__half*>(params + kTqBImg);
+    __nv_bfloat16* imb = reinterpret_cast<__nv_bfloat16*>(params + kTqBImg + kTqBImgSet);
     constexpr int kHalves = kTqBImgBytes / 2;
     for (int e = tid; e < D * D; e += kSetupThreads) {
       const int n = e / D, k = e - n * D;
@@ -215,6 +222,11 @@ __global__ void __launch_bounds__(kSetupThreads, 1)
       img[kHalves + off] = __float2half_rn(p - __half2float(ph));
       img[2 * kHalves + off] = qh;
       img[3 * kHalves + off] = __float2half_rn(q - __half2float(qh));
+      const __nv_bfloat16 pb = __float2bfloat16_rn(p), qb = __float2bfloat16_rn(q);
+      imb[off] = pb;
+      imb[kHalves + off] = __float2bfloat16_rn(p - __bfloat162float(pb));
+      imb[2 * kHalves + off] = qb;
+      imb[3 * kHalves + off] = __float2bfloat16_rn(q - __bfloat162float(qb));
     }
   }
   if (flags) atomicOr(&s_flags, flags);

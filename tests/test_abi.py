@@ -116,8 +116,8 @@ def test_turbo_layout(lib):
     rows = w.batch * w.num_kv_heads
     assert lay.record_bytes == 4032 == 2 * 1664 + 512 + 128 + 64
     assert lay.groups_per_row == (w.max_seq - w.residual) // 32
-    # Pi, Pi^T, S^T, tables, (S Pi)^T, then four fp16 tensor-core operand images
-    assert lay.params_bytes == 4 * 128 * 128 * 4 + 128 + 256 + 4 * 128 * 128 * 2
+    # Pi, Pi^T, S^T, tables, (S Pi)^T, then the fp16 and the bf16 sets of four tensor-core operand images
+    assert lay.params_bytes == 4 * 128 * 128 * 4 + 128 + 256 + 2 * 4 * 128 * 128 * 2
     assert lay.params_offset % 256 == 0 and lay.params_offset >= lay.window_offset + rows * 2 * lay.ring_tokens * 256
     assert lay.status_offset >= lay.params_offset + lay.params_bytes
     assert lib.kvq_cache_bytes(ctypes.byref(cfg)) == lay.total_bytes

@@ -239,6 +239,37 @@ def test_setup_tables_match_the_oracle():
     # (S Pi)^T: fp64 sums of the fp32 tables, then fp32 -- within a few fp32 ulps of the oracle's S Pi
     spit = p[off + 384:off + 384 + d * d * 4].view(np.float32).reshape(d, d)
     assert np.abs(spit.T.astype(np.float64) - S @ Pi).max() < 2e-5
+    # tensor-core operand images: 16 Pi and S split hi + lo, fp16 set then bf16 set, in the
+    # no-swizzle K-major layout (core matrix (n/8, k/8) at 2048 (k/8) + 128 (n/8), row n%8 at 16 B)
+    img0 = off + 384 + d * d * 4
+    n_i, k_i = np.meshgrid(np.arange(d), np.arange(d), indexing="ij")
+    pos = ((k_i >> 3) * 2048 + (n_i >> 3) * 128 + (n_i & 7) * 16 + (k_i & 7) * 2) // 2
+    for kind, (rn, widen) in enumerate(((_rn_fp16_bits, _fp16_bits_value), (_rn_bf16_bits, _bf16_bits_value))):
+        imgs = p[img0 + kind * 4 * 32768: img0 + (kind + 1) * 4 * 32768].view(np.uint16).reshape(4, d * d)
+        for j, mat in enumerate((16.0 * gpi, gst.T)):   # B[n][k] = 16 Pi[n][k], S[n][k]
+            mat = mat.astype(np.float32)
+            hi = rn(mat)
+            lo = rn((mat - widen(hi)).astype(np.float32))
+            assert np.array_equal(imgs[2 * j][pos], hi), (kind, j, "hi")
+            assert np.array_equal(imgs[2 * j + 1][pos], lo), (kind, j, "lo")
+
+
+def _rn_fp16_bits(x32):
+    return x32.astype(np.float16).view(np.uint16)
+
+
+def _fp16_bits_value(b):
+    return b.view(np.float16).astype(np.float32)
+
+
+def _rn_bf16_bits(x32):
+    # round to nearest even on the upper 16 bits of the fp32 pattern (finite inputs)
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def _bf16_bits_value(b):
+    return (b.astype(np.uint32) << 16).view(np.float32)
 
 
 # ------------------------------------------------------------------ Walsh-Hadamard rotation
