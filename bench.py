@@ -591,8 +591,7 @@ def main():
         "prefill": {"us": round(res["prefill_ms"] * 1e3, 1), "bytes": res["prefill_bytes"],
                     "achieved": round(res["prefill_bytes"] / (res["prefill_ms"] * 1e-3) / 1e9, 1), "unit": "GB/s",
                     "frac": round(res["prefill_bytes"] / (res["prefill_ms"] * 1e-3) / 1e9 / hbm, 4),
-                    "kernel": ("kivi_quantize_kernel" if w.scheme != "turbo" else
-                               "tq_quantize_kernel" if w.rotation == "wht" else "tq_quantize_tc_kernel")},
+                    "kernel": "kivi_quantize_kernel" if w.scheme != "turbo" else "tq_quantize_tc_kernel"},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_obj(oracle_sample(w, args.cpu_budget), w)

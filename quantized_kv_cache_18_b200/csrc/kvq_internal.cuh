@@ -281,7 +281,7 @@ void launch_kivi_attention(const AttnArgs& a, cudaStream_t st);
 void launch_clear_words(uint32_t* words, int n, cudaStream_t st);
 void launch_turbo_setup(const Geom& g, const float* rot_gauss, const float* qjl_gauss, bool wht, cudaStream_t st);
 void launch_tq_quantize(const QuantArgs& a, cudaStream_t st);
-// the tensor-core quantizer (dense rotation, 16-bit sources); launch_tq_quantize routes to it
+// the tensor-core quantizer (16-bit sources, either rotation); launch_tq_quantize routes to it
 void launch_tq_quantize_tc(const QuantArgs& a, cudaStream_t st);
 void launch_tq_query_prep(const Geom& g, const uint16_t* q, unsigned char* qprep, cudaStream_t st);
 void launch_tq_attention(const AttnArgs& a, cudaStream_t st);

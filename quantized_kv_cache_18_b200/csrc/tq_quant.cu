@@ -1,4 +1,6 @@
-// TurboQuant-style quantization of 32-token blocks (prefill and window flush).
+// TurboQuant-style quantization of 32-token blocks from FP8 window rows (the
+// mixed cache's flushes); 16-bit sources go to tq_quantize_tc_kernel
+// (tq_quant_tc.cu), which launch_tq_quantize below routes them to.
 //
 // Per token vector x (one kv head): n = ||x||, u = x / n, y = Pi u; each
 // coordinate of y gets the 3-bit index of its Lloyd-Max cell ("Quantification du
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(kQThreads, 1) tq_quantize_kernel(QuantArgs a) 
 void launch_tq_quantize(const QuantArgs& a, cudaStream_t st) {
   const int64_t tasks = (int64_t)a.geom.B * a.geom.Hkv * a.n_groups;
   if (tasks <= 0) return;
-  if (!a.geom.rot_wht && a.src_fp8 == nullptr) {   // dense rotation, 16-bit rows: the tensor-core kernel
+  if (a.src_fp8 == nullptr) {   // 16-bit rows, either rotation (Pi as a dense table): the tensor-core kernel
     launch_tq_quantize_tc(a, st);
     return;
   }

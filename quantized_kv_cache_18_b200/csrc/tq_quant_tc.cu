@@ -1,5 +1,5 @@
-// TurboQuant-style quantization on the 5th-generation tensor cores (dense QR
-// rotation, 16-bit sources).  The arithmetic and the readings are those of
+// TurboQuant-style quantization on the 5th-generation tensor cores (16-bit
+// sources; either rotation, Pi taken as its dense table).  The arithmetic and the readings are those of
 // tq_quantize_kernel in tq_quant.cu ("Quantification du KV-Cache : TurboQuant
 // et l'etat de l'art en 2026", "TurboQuant : les cinq innovations", items 1-3):
 // n = ||x|| (fp64 sum), y = Pi x / n to about fp32 precision, the 3-bit
