@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
   __shared__ uint32_t s_tmem, s_flags;
   __shared__ int s_abort;
   __shared__ float s_t256[8], s_lv64[8];
-  __shared__ uint32_t* s_rec[4];   // records of the tile's four tasks (null: none or outside the pool)
+  __shared__ uint32_t* s_rec[2][4];   // records of a tile's four tasks (null: none or outside the pool), by tile parity
 
   const Geom& gm = a.geom;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -253,24 +253,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
       }
       asm volatile("cp.async.commit_group;\n" ::: "memory");
     };
-    stage_rows(blockIdx.x);
-    int64_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
-      const int64_t task = tile * 4 + tbm;
-      const bool valid = task < n_tasks;
+    // The A stage of a tile: its records, the norm, x into the A operand, the
+    // per-token constants; then the next tile's rows are staged and the A
+    // operand is signalled.  It runs for tile i + 1 before tile i's words are
+    // packed, so the tensor core computes the next y while the warps pack.
+    bool valid = false;
+    unsigned char* dst = nullptr;
+    double ss = 0.0;
+    float T4 = 0.f, T5 = 0.f, T6 = 0.f, c4 = 0.f;
+    auto stage_a = [&](int64_t t, int par) {
+      const int64_t task = t * 4 + tbm;
+      valid = task < n_tasks;
       int row = 0;
       int64_t blk = 0;
       if (valid) {
         row = (int)div_floor(task, a.n_groups, rng);
         blk = task - (int64_t)row * a.n_groups;
       }
-      unsigned char* dst = valid ? reinterpret_cast<unsigned char*>(record_ptr(gm, row, a.dst_group0 + blk)) : nullptr;
+      dst = valid ? reinterpret_cast<unsigned char*>(record_ptr(gm, row, a.dst_group0 + blk)) : nullptr;
       if (kind == 0 && h == 0 && tt == 0) {
-        s_rec[tbm] = reinterpret_cast<uint32_t*>(dst);
+        s_rec[par][tbm] = reinterpret_cast<uint32_t*>(dst);
         if (valid && dst == nullptr) flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
       }
-
-      // ---------------------------------------------------------- ||x|| and x into the A operand
       asm volatile("cp.async.wait_group 0;\n" ::: "memory");
       const uint4* src = reinterpret_cast<const uint4*>(xs);
       double s0 = 0.0, s1 = 0.0;
@@ -299,20 +303,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
         }
         tmem_st16(t_hi + 32 * h + 16 * g, xv);
       }
+      stage_rows(t + gridDim.x);   // this thread's staged rows are consumed
       sNP[(2 * kind + h) * 128 + m] = s0 + s1;
       bar_pair(pair_bar);
-      const double ss = sNP[(2 * kind) * 128 + m] + sNP[(2 * kind + 1) * 128 + m];
+      ss = sNP[(2 * kind) * 128 + m] + sNP[(2 * kind + 1) * 128 + m];
       if (h == 0 && !isfinite(ss)) flags |= KVQ_DEV_NONFINITE_INPUT;
       const double n = sqrt(ss);
       // D = 16 n y: thresholds 16 n t_k (the table holds 256 t_k), and 64 y = D * 4 / n
       const float tn = (float)(n * (1.0 / 16.0));
-      const float T4 = tn * t4, T5 = tn * t5, T6 = tn * t6;
-      const float c4 = n > 0.0 ? (float)(4.0 / n) : 0.f;
-      stage_rows(tile + gridDim.x);   // this thread's staged rows are consumed
+      T4 = tn * t4;
+      T5 = tn * t5;
+      T6 = tn * t6;
+      c4 = n > 0.0 ? (float)(4.0 / n) : 0.f;
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_a[kind]);
-
+    };
+    stage_rows(blockIdx.x);
+    if (blockIdx.x < n_tiles) stage_a(blockIdx.x, 0);
+    int64_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       // ---------------------------------------------------------- y: codes (keys also e)
       // (ok is made warp-uniform: tcgen05.ld / st and the shuffle below are warp-collective)
       bool ok = __all_sync(0xffffffffu, mbar_wait_nap(&bar_d[kind], kind ? (uint32_t)(it & 1) : 0u, &s_abort));
@@ -379,6 +389,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
         const bool both = ok && !s_abort;
         if (both && h == 1) {
           const uint4 o = *reinterpret_cast<const uint4*>(sSW + 4 * m);
+          const double n = sqrt(ss);
           const __half hn = __double2half(n);
           const __half hg = __double2half(n * sqrt((double)(sEP[m] + es) * (1.0 / 4096.0)));
           if (isinf(__half2float(hn)) || isinf(__half2float(hg))) flags |= KVQ_DEV_PARAM_OVERFLOW;
@@ -417,7 +428,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
           for (int k = 0; k < 4; ++k) iv[k] = make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]);
         }
         if (h == 0) {
-          const __half hv = __double2half(n);
+          const __half hv = __double2half(sqrt(ss));
           if (isinf(__half2float(hv))) flags |= KVQ_DEV_PARAM_OVERFLOW;
           if (dst != nullptr) reinterpret_cast<uint16_t*>(dst + kTqVMeta)[entry] = __half_as_ushort(hv);
         }
@@ -428,13 +439,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
         break;
       }
 
+      // the next tile's A stage: its y is computed while this tile is packed
+      if (tile + gridDim.x < n_tiles) stage_a(tile + gridDim.x, (int)((it + 1) & 1));
+
       // ---------------------------------------------------------- pack the tile's code words
       // word i of a block's key (value) codes: i < 384 is word 4 (i / 128) + i % 4
       // of lane (i / 4) % 32, i >= 384 word 12 of lane i - 384
 #pragma unroll 1
       for (int item = tid; item < 4 * 2 * 416; item += kTokThreads) {
         const int tb = item / 832, rest = item - 832 * tb;
-        uint32_t* out = s_rec[tb];
+        uint32_t* out = s_rec[it & 1][tb];
         if (out == nullptr) continue;
         const int vblk = rest >= 416;
         const int i = rest - 416 * vblk;
