@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
   __shared__ uint32_t s_tmem, s_flags;
   __shared__ int s_abort;
   __shared__ float s_t256[8], s_lv64[8];
-  __shared__ uint32_t* s_rec[2][4];   // records of a tile's four tasks (null: none or outside the pool), by tile parity
+  __shared__ uint32_t* s_rec[2][2][4];   // [kind][tile parity]: records of a tile's four tasks (null: none or outside the pool)
 
   const Geom& gm = a.geom;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -271,9 +271,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
         blk = task - (int64_t)row * a.n_groups;
       }
       dst = valid ? reinterpret_cast<unsigned char*>(record_ptr(gm, row, a.dst_group0 + blk)) : nullptr;
-      if (kind == 0 && h == 0 && tt == 0) {
-        s_rec[par][tbm] = reinterpret_cast<uint32_t*>(dst);
-        if (valid && dst == nullptr) flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
+      if (h == 0 && tt == 0) {   // each kind's group keeps its own copy
+        s_rec[kind][par][tbm] = reinterpret_cast<uint32_t*>(dst);
+        if (kind == 0 && valid && dst == nullptr) flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
       }
       asm volatile("cp.async.wait_group 0;\n" ::: "memory");
       const uint4* src = reinterpret_cast<const uint4*>(xs);
@@ -433,29 +433,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
           if (dst != nullptr) reinterpret_cast<uint16_t*>(dst + kTqVMeta)[entry] = __half_as_ushort(hv);
         }
       }
-      // all token threads agree on stopping before the tile's words are packed
-      if (bar_red_or(9, kTokThreads, !ok)) {
+      // The key and value warps (256 each) run as two groups from here: each
+      // agrees on stopping, packs the code words of its own kind from its own
+      // index tile, and frees that tile with its own barrier.  Keys start the
+      // next tile's A stage before packing (the next y then runs meanwhile);
+      // values pack first, while the key warps wait for S e and take signs.
+      const int grp_bar = 9 + kind;
+      if (bar_red_or(grp_bar, kTokThreads / 2, !ok)) {
         flags |= KVQ_DEV_WAIT_TIMEOUT;
         break;
       }
+      const bool more = tile + gridDim.x < n_tiles;
+      if (kind == 0 && more) stage_a(tile + gridDim.x, (int)((it + 1) & 1));
 
-      // the next tile's A stage: its y is computed while this tile is packed
-      if (tile + gridDim.x < n_tiles) stage_a(tile + gridDim.x, (int)((it + 1) & 1));
-
-      // ---------------------------------------------------------- pack the tile's code words
+      // ---------------------------------------------------------- pack this kind's code words of the tile
       // word i of a block's key (value) codes: i < 384 is word 4 (i / 128) + i % 4
       // of lane (i / 4) % 32, i >= 384 word 12 of lane i - 384
+      const int gtid = tid - kind * (kTokThreads / 2);
 #pragma unroll 1
-      for (int item = tid; item < 4 * 2 * 416; item += kTokThreads) {
-        const int tb = item / 832, rest = item - 832 * tb;
-        uint32_t* out = s_rec[it & 1][tb];
+      for (int item = gtid; item < 4 * 416; item += kTokThreads / 2) {
+        const int tb = item / 416, i = item - 416 * tb;
+        uint32_t* out = s_rec[kind][it & 1][tb];
         if (out == nullptr) continue;
-        const int vblk = rest >= 416;
-        const int i = rest - 416 * vblk;
         const int ln = i < 384 ? (i >> 2) & 31 : i - 384;
         const int w = i < 384 ? 4 * (i >> 7) + (i & 3) : 12;
         uint32_t word = 0;
-        if (!vblk) {
+        if (kind == 0) {
           // slots 5 w .. 5 w + 4 of the lane's 64 index bytes
           const uint8_t* ib = sIK + tb * 32 * kIKRow + ln * kIKRow;
           const int b0 = 5 * w;
@@ -477,9 +480,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
             }
           }
         }
-        out[(vblk ? kTqVCodes : kTqKCodes) / 4 + i] = word;
+        out[(kind ? kTqVCodes : kTqKCodes) / 4 + i] = word;
       }
-      asm volatile("bar.sync 9, %0;\n" ::"r"(kTokThreads) : "memory");   // index tiles free for the next tile
+      if (kind == 1 && more) stage_a(tile + gridDim.x, (int)((it + 1) & 1));
+      asm volatile("bar.sync %0, %1;\n" ::"r"(grp_bar), "r"(kTokThreads / 2) : "memory");   // index tile free
     }
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");   // no staging copy outlives the loop
   }
