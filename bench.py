@@ -21,7 +21,9 @@ and again: the warm-L2 median), and the launch overhead is reported apart:
 the host cost of one library call and the device gap a separately launched
 graph adds.  The e2e figure calls the public API step by step with host
 buffers: one pinned host-to-device copy of the step's inputs and one
-device-to-host copy of its output per step.
+device-to-host copy of its output per step, each on its own stream into
+double-buffered device rows, so a step's copies overlap its neighbours'
+kernels as in a serving loop (events keep every buffer's reuse in order).
 """
 from __future__ import annotations
 
@@ -58,6 +60,82 @@ def _profiled_traffic(kernel: str, source: str, workload: str):
         return None
     src = open(os.path.join(ROOT, "quantized_kv_cache_18_b200", "csrc", source), "rb").read()
     return int(m.group(1)) if hashlib.sha256(src).hexdigest()[:16] == m.group(2) else None
+
+
+class CudaRt:
+    """The e2e loop's copies and stream orderings, issued as plain CUDA runtime
+    calls (the system libcudart through ctypes): the torch equivalents cost
+    several microseconds of host time each, which bounds a ~40 us step.
+    Events per buffer b: in[b] (inputs on the device), done[b] (the kernel that
+    read row b ended), read[b] (output buffer b copied back)."""
+
+    H2D, D2H, NO_TIMING = 1, 2, 2
+
+    def __init__(self, compute, s_h2d, s_d2h):
+        self.lib = None
+        for name in ("libcudart.so.12", "/usr/local/cuda/lib64/libcudart.so.12"):
+            try:
+                self.lib = ctypes.CDLL(name)
+                break
+            except OSError:
+                continue
+        if self.lib is None:
+            raise RuntimeError("the CUDA runtime library (libcudart.so.12) is needed for the e2e copies")
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        self.lib.cudaMemcpyAsync.argtypes = [vp, vp, sz, ctypes.c_int, vp]
+        self.lib.cudaEventRecord.argtypes = [vp, vp]
+        self.lib.cudaStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
+        self.lib.cudaEventCreateWithFlags.argtypes = [ctypes.POINTER(vp), ctypes.c_uint]
+        self.lib.cudaEventDestroy.argtypes = [vp]
+
+        def make():
+            e = vp()
+            self._chk(self.lib.cudaEventCreateWithFlags(ctypes.byref(e), self.NO_TIMING), "cudaEventCreateWithFlags")
+            return e
+        self.ev = {k: [make(), make()] for k in ("in", "done", "read")}
+        self.sp = {k: vp(st.cuda_stream) for k, st in (("c", compute), ("h", s_h2d), ("d", s_d2h))}
+
+    @staticmethod
+    def _chk(r, what):
+        if r != 0:
+            raise RuntimeError(f"{what} failed ({r})")
+
+    def _wait(self, stream_key, ev):
+        self._chk(self.lib.cudaStreamWaitEvent(self.sp[stream_key], ev, 0), "cudaStreamWaitEvent")
+
+    def _record(self, ev, stream_key):
+        self._chk(self.lib.cudaEventRecord(ev, self.sp[stream_key]), "cudaEventRecord")
+
+    def _copy(self, dst, src, n, kind, stream_key):
+        self._chk(self.lib.cudaMemcpyAsync(ctypes.c_void_p(dst), ctypes.c_void_p(src), n, kind, self.sp[stream_key]),
+                  "cudaMemcpyAsync")
+
+    def h2d(self, dst, src, n, b, wait_done):
+        if wait_done:
+            self._wait("h", self.ev["done"][b])
+        self._copy(dst, src, n, self.H2D, "h")
+        self._record(self.ev["in"][b], "h")
+
+    def before_kernel(self, b, wait_read):
+        self._wait("c", self.ev["in"][b])
+        if wait_read:
+            self._wait("c", self.ev["read"][b])
+
+    def after_kernel(self, b):
+        self._record(self.ev["done"][b], "c")
+
+    def d2h(self, dst, src, n, b):
+        self._wait("d", self.ev["done"][b])
+        self._copy(dst, src, n, self.D2H, "d")
+        self._record(self.ev["read"][b], "d")
+
+    def finish(self, b):
+        self._wait("c", self.ev["read"][b])
+
+    def close(self):
+        for evs in self.ev.values():
+            for e in evs:
+                self.lib.cudaEventDestroy(e)
 
 
 def _peaks():
@@ -370,10 +448,14 @@ def run_gpu(args, w, rank, world):
         h_in[j, nq:nq + nk].copy_(kn[i].reshape(-1))
         h_in[j, nq + nk:].copy_(vn[i].reshape(-1))
     h_out = torch.empty((args.steps,) + tuple(out.shape), dtype=torch.float32).pin_memory()
-    d_in = torch.empty(row_elems, dtype=q.dtype, device=device)
-    esz = d_in.element_size()
-    d_q, d_kn, d_vn = (ctypes.c_void_p(d_in.data_ptr()), ctypes.c_void_p(d_in.data_ptr() + nq * esz),
-                       ctypes.c_void_p(d_in.data_ptr() + (nq + nk) * esz))
+    # two device input rows and two output buffers: step j uses buffer j % 2, so
+    # the copy of step j + 1's inputs and the read of step j's output can run
+    # on their own streams while step j + 1 (or j) computes
+    d_in = [torch.empty(row_elems, dtype=q.dtype, device=device) for _ in range(2)]
+    d_out = [torch.empty_like(out) for _ in range(2)]
+    esz = d_in[0].element_size()
+    d_ptrs = [(ctypes.c_void_p(t.data_ptr()), ctypes.c_void_p(t.data_ptr() + nq * esz),
+               ctypes.c_void_p(t.data_ptr() + (nq + nk) * esz)) for t in d_in]
     e_caches = [new_cache() for _ in range(n_rep)]
     K, V, _, _, _ = device_inputs(w, device, 1, rank)
     if turbo:
@@ -394,16 +476,27 @@ def run_gpu(args, w, rank, world):
     e_args = [(c.handle, ptr(c.ws), c.ws.numel()) for c in e_caches]
     e_bytes = 0
     torch.cuda.synchronize()
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    rt = CudaRt(stream, s_h2d, s_d2h)
+    in_bytes, out_bytes = int(row_elems * esz), int(out.numel() * 4)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    s_h2d.wait_event(e0)
     for j in range(args.steps):
+        b = j % 2
         hnd, wsp, wsn = e_args[j % n_rep]
-        d_in.copy_(h_in[j], non_blocking=True)
-        L.check(lib.kvq_append_decode(hnd, d_kn, d_vn, d_q, outp, scale, wsp, wsn, sp), "append_decode")
-        h_out[j].copy_(out, non_blocking=True)
+        # inputs of step j into row b once the kernel that last read it (step j - 2) is done
+        rt.h2d(d_in[b].data_ptr(), h_in[j].data_ptr(), in_bytes, b, wait_done=j >= 2)
+        d_q, d_kn, d_vn = d_ptrs[b]
+        rt.before_kernel(b, wait_read=j >= 2)
+        L.check(lib.kvq_append_decode(hnd, d_kn, d_vn, d_q, ptr(d_out[b]), scale, wsp, wsn, sp), "append_decode")
+        rt.after_kernel(b)
+        rt.d2h(h_out[j].data_ptr(), d_out[b].data_ptr(), out_bytes, b)
         e_bytes += step_bytes(e_caches[j % n_rep])
+    rt.finish((args.steps - 1) % 2)
     e1.record(stream)
     torch.cuda.synchronize()
+    rt.close()
     e_ms = e0.elapsed_time(e1)
     e_ms, e_bytes = combine_ranks(e_ms, e_bytes, world, device)
 
