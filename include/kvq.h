@@ -332,18 +332,22 @@ const char* kvq_cuda_error_string(void);
 uint64_t kvq_launch_count(void);
 
 /*
- * Test hook for the decode kernels' bounded waits (no counterpart on the
- * pages).  Every pipeline wait inside a decode launch gives up after a bound
- * (default: about 1 s of SM clock cycles); a wait that gives up sets
- * KVQ_DEV_WAIT_TIMEOUT and the launch finishes without writing outputs it
- * cannot trust, leaving the GPU context usable.  This call lets a test reach
- * that path without a GPU fault:
- *   wait_cycles           the bound in SM clock cycles for later decode
- *                         launches of this process (0 restores the default;
- *                         values above the default are rejected);
+ * Test hook for the bounded waits of the decode kernels and of the
+ * tensor-core TurboQuant quantizer (no counterpart on the pages).  Every
+ * pipeline wait inside such a launch gives up after a bound (default: about
+ * 1 s of SM clock cycles); a wait that gives up sets KVQ_DEV_WAIT_TIMEOUT and
+ * the launch finishes without writing outputs it cannot trust (a quantizer
+ * CTA stops at a tile boundary: its remaining records are unspecified),
+ * leaving the GPU context usable.  This call lets a test reach that path
+ * without a GPU fault:
+ *   wait_cycles           the bound in SM clock cycles for later launches of
+ *                         these kernels in this process (0 restores the
+ *                         default; values above the default are rejected);
  *   withhold_first_stage  nonzero: CTA 0 of later decode launches does not
- *                         issue the copy of its first pipeline stage, so the
- *                         waits on that stage run out after `wait_cycles`.
+ *                         issue the copy of its first pipeline stage, and CTA
+ *                         0 of later tensor-core quantizer launches not the
+ *                         copy of its operand images, so the waits on them
+ *                         run out after `wait_cycles`.
  * Waits for copies already in flight before a CTA exits keep the default
  * bound.  Process-wide, not thread-safe against concurrent launches; for
  * tests only.  Returns KVQ_ERR_INVALID_ARG for a bound above the default.

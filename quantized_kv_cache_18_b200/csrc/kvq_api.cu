@@ -32,6 +32,12 @@ static thread_local const char* g_cuda_error = "no error";
 // Test hook of the decode kernels' bounded waits (kvq_debug_set_wait_test).
 static std::atomic<long long> g_wait_cycles{0};   // 0: the default bound
 static std::atomic<int> g_withhold{0};
+// the hook's values for a quantizer launch
+static void quant_wait_args(QuantArgs& a) {
+  const long long wc = g_wait_cycles.load(std::memory_order_relaxed);
+  a.wait_cycles = wc > 0 ? wc : kWaitCyclesDefault;
+  a.withhold_first_stage = g_withhold.load(std::memory_order_relaxed);
+}
 
 // Records the failing CUDA call's message for kvq_cuda_error_string.
 static kvq_status cuda_failed(cudaError_t e) {
@@ -327,6 +333,7 @@ kvq_status kvq_quantize_prefill(kvq_cache* h, const void* k, const void* v, int3
   a.src_fp8 = nullptr;
   a.dst_group0 = 0;
   a.n_groups = tq / G;
+  quant_wait_args(a);
   if (c.scheme == KVQ_TURBO) launch_tq_quantize(a, st);
   else launch_kivi_quantize(a, st);
   if (c.fp8_recent) {
@@ -377,6 +384,7 @@ kvq_status kvq_append_token(kvq_cache* h, const void* k_new, const void* v_new, 
                              : nullptr;
     a.dst_group0 = tq / G;
     a.n_groups = 1;
+    quant_wait_args(a);
     if (c.scheme == KVQ_TURBO) launch_tq_quantize(a, st);
     else launch_kivi_quantize(a, st);
     head = (head + G) % cap;

@@ -236,6 +236,8 @@ struct QuantArgs {
   const unsigned char* src_fp8;   // TURBO mixed flush: FP8 window rows of the first token (ring layout), or null
   int64_t dst_group0;      // first record index written
   int n_groups;            // groups per row handled by this launch
+  long long wait_cycles;   // bound of the tensor-core quantizer's waits (SM cycles)
+  int withhold_first_stage;   // test hook: CTA 0 of the tensor-core quantizer skips its operand-image copy
 };
 
 struct AttnArgs {

@@ -98,7 +98,7 @@ __device__ __forceinline__ void split_pair(float v0, float v1, uint32_t& hi, uin
 
 // Bounded wait that sleeps between polls (the waits here last microseconds;
 // polling would take issue slots from the warps that work meanwhile).
-__device__ __forceinline__ bool mbar_wait_nap(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_nap(uint64_t* b, uint32_t parity, volatile int* abort_flag, long long limit) {
   if (mbar_try_wait(b, parity)) return true;
   const long long t0 = clock64();
   uint32_t ns = 32;
@@ -106,7 +106,7 @@ __device__ __forceinline__ bool mbar_wait_nap(uint64_t* b, uint32_t parity, vola
     __nanosleep(ns);
     if (mbar_try_wait(b, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
     if (ns < 256) ns <<= 1;
   }
 }
@@ -195,26 +195,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
   if (warp == kTokWarps) {
     // ------------------------------------------------------------ mma issue
     if (lane == 0) {
-      mbar_expect_tx(&bar_b, 4 * kTqBImgBytes);
+      // (test hook: CTA 0 may withhold the copy, so that the wait below runs out)
+      const bool withheld = a.withhold_first_stage && blockIdx.x == 0;
+      if (!withheld) {
+        mbar_expect_tx(&bar_b, 4 * kTqBImgBytes);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        bulk_g2s(sB + i * kTqBImgBytes, gm.params + kTqBImg + (BF ? kTqBImgSet : 0) + i * kTqBImgBytes, kTqBImgBytes,
-                 &bar_b);
-      bool ok = mbar_wait_nap(&bar_b, 0, &s_abort);
-      if (!ok) mbar_drain(&bar_b, 0);
+        for (int i = 0; i < 4; ++i)
+          bulk_g2s(sB + i * kTqBImgBytes, gm.params + kTqBImg + (BF ? kTqBImgSet : 0) + i * kTqBImgBytes, kTqBImgBytes,
+                   &bar_b);
+      }
+      bool ok = mbar_wait_nap(&bar_b, 0, &s_abort, a.wait_cycles);
+      if (!ok && !withheld) mbar_drain(&bar_b, 0);   // the copy in flight lands before the CTA exits
       const unsigned char *pi_hi = sB, *pi_lo = sB + kTqBImgBytes;
       const unsigned char *s_hi = sB + 2 * kTqBImgBytes, *s_lo = sB + 3 * kTqBImgBytes;
       int64_t it = 0;
       for (int64_t tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
-        if (!(ok = mbar_wait_nap(&bar_a[0], 0, &s_abort))) break;
+        if (!(ok = mbar_wait_nap(&bar_a[0], 0, &s_abort, a.wait_cycles))) break;
         tc_fence_after();
         issue_product<BF, false>(tbase, tbase + 128, tbase + 192, pi_hi, pi_lo);
         umma_commit(&bar_d[0]);
-        if (!(ok = mbar_wait_nap(&bar_a[1], (uint32_t)(it & 1), &s_abort))) break;
+        if (!(ok = mbar_wait_nap(&bar_a[1], (uint32_t)(it & 1), &s_abort, a.wait_cycles))) break;
         tc_fence_after();
         issue_product<BF, false>(tbase + 256, tbase + 384, tbase + 448, pi_hi, pi_lo);
         umma_commit(&bar_d[1]);
-        if (!(ok = mbar_wait_nap(&bar_a[0], 1, &s_abort))) break;
+        if (!(ok = mbar_wait_nap(&bar_a[0], 1, &s_abort, a.wait_cycles))) break;
         tc_fence_after();
         issue_product<BF, true>(tbase, tbase + 128, tbase + 192, s_hi, s_lo);
         umma_commit(&bar_d[0]);
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
       // ---------------------------------------------------------- y: codes (keys also e)
       // (ok is made warp-uniform: tcgen05.ld / st and the shuffle below are warp-collective)
-      bool ok = __all_sync(0xffffffffu, mbar_wait_nap(&bar_d[kind], kind ? (uint32_t)(it & 1) : 0u, &s_abort));
+      bool ok = __all_sync(0xffffffffu, mbar_wait_nap(&bar_d[kind], kind ? (uint32_t)(it & 1) : 0u, &s_abort, a.wait_cycles));
       if (!ok) s_abort = 1;
       if (kind == 0) {
         float es = 0.f;
@@ -364,7 +368,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tq_quantize_tc_kernel(QuantArgs
           tc_wait_st();
           tc_fence_before();
           mbar_arrive(&bar_a[0]);
-          ok = __all_sync(0xffffffffu, mbar_wait_nap(&bar_d[0], 1u, &s_abort));
+          ok = __all_sync(0xffffffffu, mbar_wait_nap(&bar_d[0], 1u, &s_abort, a.wait_cycles));
           if (!ok) s_abort = 1;
         }
         uint32_t sw[4] = {0u, 0u, 0u, 0u};

@@ -1,4 +1,5 @@
-"""The decode kernels' bounded waits, exercised without a GPU fault.
+"""The bounded waits of the decode kernels and of the tensor-core TurboQuant
+quantizer, exercised without a GPU fault.
 
 Every pipeline wait inside a decode launch gives up after a bound; the
 launch then sets KVQ_DEV_WAIT_TIMEOUT and finishes without the outputs it
@@ -84,6 +85,40 @@ def test_turbo_wait_timeout_sets_status_and_recovers():
             check_attention(out[b, h * g:(h + 1) * g], row.attention(q[b, h * g:(h + 1) * g], w.scale))
 
     _timed_out_then_recovers(cache, lambda: cache.attention(qd), check)
+
+
+def test_turbo_quantizer_wait_timeout_sets_status_and_recovers():
+    """The tensor-core TurboQuant quantizer: CTA 0 withholds its operand-image
+    copy, its mma thread's wait runs out, the CTA stops at a tile boundary and
+    sets the status bit; the other CTAs finish.  After a clear, a fresh prefill
+    quantizes every block like the oracle."""
+    from test_gpu_turbo import SMALL, check_blocks, gpu_cache, oracle_params
+    lib = L.load()
+    w = W.with_sizes(SMALL, batch=2, seq_len=3000)
+    K, V = W.prefill(w, seq_len=3000)
+    cache = gpu_cache(w)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    L.check(lib.kvq_debug_set_wait_test(SHORT_WAIT, 1), "kvq_debug_set_wait_test")
+    try:
+        cache.prefill(to_dev(K), to_dev(V))
+        torch.cuda.synchronize()
+    finally:
+        L.check(lib.kvq_debug_set_wait_test(0, 0), "kvq_debug_set_wait_test")
+    assert cache.status(clear=True) & L.KVQ_DEV_WAIT_TIMEOUT
+    assert cache.status() == 0
+    params = oracle_params(w)
+    fresh = gpu_cache(w)
+    fresh.prefill(to_dev(K), to_dev(V))
+    torch.cuda.synchronize()
+    assert fresh.status() == 0
+    n_tb = fresh.quantized_len // 32
+    assert n_tb > 0
+    rec = fresh.records_view()
+    for b in range(w.batch):
+        for h in range(w.num_kv_heads):
+            check_blocks(rec[b * w.num_kv_heads + h, :n_tb].cpu().numpy(), w, params,
+                         K[b, h][:32 * n_tb], V[b, h][:32 * n_tb])
 
 
 def test_wait_bound_above_default_is_rejected():
