@@ -365,7 +365,7 @@ int32_t kvq_decode_splits(const kvq_cache* cache);
  * CTA c of the decode launch owns the global items item0[c] .. item0[c+1]-1
  * (global item = row x n_items + item); item0[0] = 0, item0[n] = rows x
  * n_items, strictly increasing.  The ranges balance stages (a stage carries
- * up to 12 KIVI groups for G = 32, 6 for G = 64, or 8 TURBO blocks;
+ * up to 12 KIVI groups for G = 32, 6 for G = 64, or 11 TURBO blocks;
  * a window chunk's stage weighs 1.5 of them) and quantized ranges start at a
  * stage boundary of their row.  Fills item0[0 .. n] (caller-owned, `cap`
  * entries) and returns n, or 0 for a null pointer, an unsupported

@@ -41,7 +41,7 @@ constexpr int kMaxDecodeCtas = 160;   // decode launches use at most this many C
 constexpr int kDecodeWinTok = 32;     // window tokens per decode work item
 constexpr int kKiviConsumersTM = 12;  // KIVI decode consumer warps, token-major formulation (GQA groups <= 4)
 constexpr int kKiviConsumersHM = 12;  // KIVI decode consumer warps, hybrid formulation (GQA groups of 8)
-constexpr int kTqDecodeConsumers = 8; // TurboQuant decode consumer warps
+constexpr int kTqDecodeConsumers = 11; // TurboQuant decode consumer warps
 constexpr long long kWaitCyclesDefault = 2000000000ll;   // decode wait bound: about 1 s of SM cycles
 
 struct Geom {

@@ -47,7 +47,7 @@ struct TL {
   static constexpr int WROW = D * 2;
   static constexpr int WINB = kTqWin * WROW * 2;
   static constexpr int STAGE = ((SG * kTqTbBytes > WINB ? SG * kTqTbBytes : WINB) + 127) / 128 * 128;
-  static constexpr int NST = 3;
+  static constexpr int NST = 2;
   static constexpr int QRAW = 8 * D * 2;                          // raw 16-bit q of up to 8 heads
   static constexpr int QSLOT = kTqQPrepBytes + QRAW;
   static constexpr int OFF_PI = NST * STAGE;                      // float [D][D], Pi[j][c]

@@ -11,9 +11,9 @@ WS, WW = 2, 3   # weights of a stage of quantized items and of a window chunk
 
 def stage_items(cfg):
     """Quantized items per stage: the decode kernels' consumer warps take one
-    32-token block each (12 KIVI warps in either formulation, 8 TURBO)."""
+    32-token block each (12 KIVI warps in either formulation, 11 TURBO)."""
     if cfg.scheme != 0:
-        return 8
+        return 11
     return 12 // (cfg.group // 32)
 
 
