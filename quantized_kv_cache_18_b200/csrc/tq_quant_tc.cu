@@ -38,7 +38,11 @@
 // value chain runs while the key warps code y, the S e chain while the value
 // warps code theirs.  Key threads write their 6-bit pair indices in record
 // slot order; value threads combine their codes with the next token's (the
-// next lane) into pair indices; the token warps then pack the tile's words.
+// next lane) into pair indices.  The key warps and the value warps (256
+// threads each) then run as two groups: each packs the words of its own kind
+// from its own index tile.  The values pack while the keys wait for S e; the
+// keys run the next tile's A stage before packing, so that its y chain runs
+// meanwhile (the value warps run theirs after packing).
 // Every wait is bounded and idles with a short sleep instead of spinning; a
 // wait that gives up sets KVQ_DEV_WAIT_TIMEOUT and the CTA stops at the next
 // tile boundary, after its issued chains complete.
