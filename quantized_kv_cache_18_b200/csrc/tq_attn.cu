@@ -13,7 +13,7 @@
 // shared memory, and +-1 built from the sign bits with one LOP3.
 //
 // Structure as the KIVI decode kernel: one CTA per SM, a producer warp feeding
-// a ring of shared-memory stages with 1-D bulk copies (no multicast), eight
+// a ring of shared-memory stages with 1-D bulk copies (no multicast), eleven
 // consumer warps each taking one 32-token block of a stage.  A row's items are
 // its token blocks, then its 32-token window chunks; the two kinds form
 // separate segments because their partial outputs live in different bases
