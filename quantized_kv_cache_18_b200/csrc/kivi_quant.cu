@@ -21,7 +21,11 @@ namespace kvq {
 
 namespace {
 
-constexpr int kQuantThreads = 128;
+// Threads of a quantizer CTA: 128 (key warps 0-1, value warps 2-3), or 256
+// for 4-bit records of 64 tokens and d = 128, whose longer code phase is split
+// over four key and four value warps.
+template <int BITS, int D, int G>
+__host__ __device__ constexpr int quant_threads() { return BITS == 4 && D == 128 && G == 64 ? 256 : 128; }
 
 __device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bits) {
   if (bits) atomicOr(status, bits);
@@ -188,7 +192,9 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 //    token blocks), warps 2-3 values (a thread keeps its eight tokens').
 // 4. The record, assembled in shared memory, is stored in 16-byte pieces.
 template <int BITS, int D, int G, bool BF>
-__global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(quant_threads<BITS, D, G>()) kivi_quantize_kernel(QuantArgs a) {
+  constexpr int NT = quant_threads<BITS, D, G>();
+  constexpr int KW = NT / 64;                   // key warps, then as many value warps
   constexpr int L = (1 << BITS) - 1;
   constexpr int NTB = G / kTB;
   constexpr int PAIRS = 16 / BITS;              // pairs per word
@@ -198,9 +204,10 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
   constexpr int TBB = kTB * D * BITS / 8;       // code bytes of one TB
   constexpr int REC = 2 * NTB * TBB + 4 * D + NTB * kTB * 4;
   constexpr int PITCH = D + 8;                  // staged row pitch (halves)
-  constexpr int KS = 128 / D;                   // key parameter threads per channel pair
-  constexpr int VS = 64 / G;                    // value parameter threads per token
-  static_assert(REC % 16 == 0 && PAIRS % 4 == 0 && (D / 2) * KS == 64 && VS >= 1, "shape");
+  constexpr int KS = NT / D;                    // key parameter threads per channel pair
+  constexpr int VS = NT / 2 / G;                // value parameter threads per token
+  static_assert(REC % 16 == 0 && PAIRS % 4 == 0 && (D / 2) * KS == NT / 2 && VS >= 1, "shape");
+  static_assert(KS <= 2 && VS <= 2, "parameter threads per unit");
   extern __shared__ __align__(16) unsigned char smem[];
   uint16_t* sk = reinterpret_cast<uint16_t*>(smem);           // [G][PITCH]
   uint16_t* sv = sk + G * PITCH;                              // [G][PITCH]
@@ -223,7 +230,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
     const uint16_t* gk = a.src_k + (int64_t)row * a.src_row_stride + (int64_t)grp * G * D;
     const uint16_t* gv = a.src_v + (int64_t)row * a.src_row_stride + (int64_t)grp * G * D;
 #pragma unroll 4
-    for (int i = tid; i < G * D / 8; i += kQuantThreads) {
+    for (int i = tid; i < G * D / 8; i += NT) {
       const int t = i / (D / 8), c8 = i - t * (D / 8);
       cp_async16(sk + t * PITCH + 8 * c8, gk + 8 * i);
       cp_async16(sv + t * PITCH + 8 * c8, gv + 8 * i);
@@ -266,7 +273,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
   };
 
   // 2. parameters
-  if (tid < 64) {
+  if (tid < NT / 2) {
     // channel pair pc over tokens ks, ks + KS, ... (rows 1 apart: 4 banks apart)
     const int pc = tid / KS, ks = tid % KS;
     T2 mn = PT::of(BF ? 0x7F807F80u : 0x7C007C00u), mx = PT::of(BF ? 0xFF80FF80u : 0xFC00FC00u);
@@ -289,7 +296,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
     }
   } else {
     // token t over channel pairs [v D/(2 VS), (v + 1) D/(2 VS)), four at a time
-    const int u = tid - 64, t = u / VS, v = u % VS;
+    const int u = tid - NT / 2, t = u / VS, v = u % VS;
     constexpr int PPV = D / (2 * VS);
     T2 mn = PT::of(BF ? 0x7F807F80u : 0x7C007C00u), mx = PT::of(BF ? 0xFF80FF80u : 0xFC00FC00u);
 #pragma unroll 4
@@ -319,11 +326,15 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
   auto word_at = [&](bool is_v, int tb, int w) -> uint32_t* {
     return reinterpret_cast<uint32_t*>(srec + (is_v ? NTB + tb : tb) * TBB + 16 * (32 * (w >> 2) + lane) + 4 * (w & 3));
   };
-  if (warp < 2) {
-    // keys: word (nt, sub) of token 8 nt + gr holds channels 8 PAIRS sub + 8 j + 2 tc (+1)
-    constexpr int SUBS_PER_WARP = WPT >= 2 ? WPT / 2 : 1;
+  if (warp < KW) {
+    // keys: word (nt, sub) of token 8 nt + gr holds channels 8 PAIRS sub + 8 j + 2 tc (+1);
+    // a warp takes subs warp, warp + KW, ... of every 8-token block, or (fewer
+    // subs than key warps) one sub of every (KW / WPT)-th block
+    constexpr int SUBS_PER_WARP = WPT >= KW ? WPT / KW : 1;
+    constexpr int IT_STEP = WPT >= KW ? 1 : KW / WPT;
+    const int it0 = WPT >= KW ? 0 : warp / WPT;
     for (int si = 0; si < SUBS_PER_WARP; ++si) {
-      const int sub = WPT >= 2 ? 2 * si + warp : 0;
+      const int sub = WPT >= KW ? KW * si + warp : warp % WPT;
       const int cbase = 8 * PAIRS * sub + 2 * tc;
       if constexpr (BITS == 2) {
         uint32_t c0[PAIRS], c1[PAIRS], c2[PAIRS];
@@ -334,7 +345,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
           c2[j] = *reinterpret_cast<const uint32_t*>(&kc[2][cbase + 8 * j]);
         }
 #pragma unroll 1
-        for (int it = (WPT >= 2 ? 0 : warp); it < NTB * 4; it += (WPT >= 2 ? 1 : 2)) {
+        for (int it = it0; it < NTB * 4; it += IT_STEP) {
           const int tb = it >> 2, nt = it & 3;
           const uint16_t* rowp = sk + (tb * kTB + 8 * nt + (lane & 7)) * PITCH + 8 * PAIRS * sub + 8 * (lane >> 3);
           uint32_t x[PAIRS];
@@ -357,7 +368,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
             thr = fminf(thr, q.z);
           }
 #pragma unroll 1
-        for (int it = (WPT >= 2 ? 0 : warp); it < NTB * 4; it += (WPT >= 2 ? 1 : 2)) {
+        for (int it = it0; it < NTB * 4; it += IT_STEP) {
           const int tb = it >> 2, nt = it & 3;
           const uint16_t* rowp = sk + (tb * kTB + 8 * nt + (lane & 7)) * PITCH + 8 * PAIRS * sub + 8 * (lane >> 3);
           uint32_t x[PAIRS];
@@ -384,7 +395,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
     }
   } else {
     // values: word w holds channels 8 (CPW w + j / 4) + gr, tokens 8 (j % 4) + 2 tc (+1)
-    const int vw = warp - 2;
+    const int vw = warp - KW;
     for (int tb = 0; tb < NTB; ++tb) {
       if constexpr (BITS == 2) {
         uint32_t c0[4], c1[4], c2[4];
@@ -396,7 +407,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
           c2[m] = *reinterpret_cast<const uint32_t*>(&vc[2][t]);
         }
 #pragma unroll 1
-        for (int w = vw; w < P; w += 2) {
+        for (int w = vw; w < P; w += KW) {
           uint32_t x[PAIRS];
 #pragma unroll
           for (int i = 0; i < PAIRS / 4; ++i)
@@ -418,7 +429,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
             thr = fminf(thr, q.z);
           }
 #pragma unroll 1
-        for (int w = vw; w < P; w += 2) {
+        for (int w = vw; w < P; w += KW) {
           uint32_t x[PAIRS];
           ldsm_x4_t(x, sv + (tb * kTB + 8 * (lane >> 3) + (lane & 7)) * PITCH + 8 * w);
           float acc0 = 8388608.f, acc1 = 8388608.f;
@@ -448,7 +459,7 @@ __global__ void __launch_bounds__(kQuantThreads) kivi_quantize_kernel(QuantArgs 
   // 4. store the record
   char* rec = record_ptr(a.geom, row, a.dst_group0 + grp);
   if (rec != nullptr) {
-    for (int i = tid; i < REC / 16; i += kQuantThreads)
+    for (int i = tid; i < REC / 16; i += NT)
       reinterpret_cast<uint4*>(rec)[i] = reinterpret_cast<const uint4*>(srec)[i];
   } else if (tid == 0) {
     s_flags |= KVQ_DEV_BAD_PAGE;   // page outside the pool: nothing is written
@@ -498,7 +509,7 @@ void launch_q_dtype(const QuantArgs& a, cudaStream_t st) {
     attr_set = true;
   }
   dim3 grid(a.n_groups, a.geom.B * a.geom.Hkv);
-  kern<<<grid, kQuantThreads, smem, st>>>(a);
+  kern<<<grid, quant_threads<BITS, D, G>(), smem, st>>>(a);
 }
 template <int BITS, int D, int G>
 void launch_q(const QuantArgs& a, cudaStream_t st) {
