@@ -138,6 +138,31 @@ def test_code_decisions_on_tiny_inputs(dtype, bits):
     _run_prefill_bits(w, k, v)
 
 
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_code_decisions_d128_g64_4bit(dtype):
+    """The 4-bit quantizer instance of 64-token records at d = 128 (eight warps
+    a CTA), on the inputs of the two tests above: large zero-points against
+    the scale and exact ties (even heads: offsets, odd heads: the half-step
+    grid), then inputs around 1e-6.  Bit-exact like the oracle."""
+    w = W.with_sizes(W.WORKLOADS["8b4"], batch=1, dtype=dtype)
+    assert (w.bits, w.group, w.head_dim) == (4, 64, 128)
+    rng = np.random.default_rng(11)
+    S, H, levels = 400, w.num_kv_heads, 15
+    x = np.empty((1, H, S, 128), np.float32)
+    for h in range(H):
+        if h % 2 == 0:
+            for t0, off in ((0, 512.0), (128, -300.0), (256, 1000.0)):
+                x[0, h, t0:t0 + 144] = off + rng.normal(0.0, 1.5, (min(144, S - t0), 128))
+        else:
+            x[0, h] = 512.0 + rng.integers(0, 2 * levels + 1, (S, 128)) / 2.0
+            x[0, h, :, 0] = 512.0
+            x[0, h, :, 1] = 512.0 + levels
+    _run_prefill_bits(w, W.to_bits(x, dtype), W.to_bits(x[..., ::-1].copy(), dtype))
+    y = rng.normal(0.0, 1.5e-6, (1, H, S, 128))
+    y[0, 1::2] += 4e-6
+    _run_prefill_bits(w, W.to_bits(y, dtype), W.to_bits(y[..., ::-1].copy(), dtype))
+
+
 def _run_prefill_bits(w, K, V):
     cache = gpu_prefill(w, K, V)
     for b in range(w.batch):
