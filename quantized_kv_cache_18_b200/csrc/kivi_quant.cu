@@ -182,14 +182,14 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 //
 // 1. The key and value tiles are copied to shared memory (rows padded by 16
 //    bytes, so the 8 rows of an 8x8 ldmatrix tile fall in distinct banks).
-// 2. Parameters: warps 0-1 reduce key channel pairs over the G tokens, warps
-//    2-3 value tokens over the d channels, with 16-bit pair min/max.
+// 2. Parameters: the first half of the threads reduce key channel pairs over
+//    the G tokens, the second half value tokens over d, with 16-bit min/max.
 // 3. Codes: a thread builds whole 32-bit words of the packed format for its own
 //    lane.  ldmatrix hands lane (gr, tc) exactly a word's pairs: a key tile
 //    (tokens x channels) gives token gr, channels 2tc and 2tc + 1; the same
 //    tile transposed gives channel gr, tokens 2tc and 2tc + 1 for the values.
-//    Warps 0-1 code keys (a thread keeps the thresholds of its channels across
-//    token blocks), warps 2-3 values (a thread keeps its eight tokens').
+//    The first half of the warps code keys (a thread keeps the thresholds of its
+//    channels across token blocks), the rest values (its eight tokens').
 // 4. The record, assembled in shared memory, is stored in 16-byte pieces.
 template <int BITS, int D, int G, bool BF>
 __global__ void __launch_bounds__(quant_threads<BITS, D, G>()) kivi_quantize_kernel(QuantArgs a) {
