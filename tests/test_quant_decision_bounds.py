@@ -102,3 +102,47 @@ def test_exact_ties_go_to_the_exact_rule():
     assert not decided[tie].any()
     assert decided[~tie].all()
     _check(x, mn, mx, 0.45)
+
+
+# ------------------------------------------------------------------ 2-bit thresholds
+def _all_finite16(dtype):
+    """Every finite value of the 16-bit format, ascending (each value once)."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    if dtype == "fp16":
+        v = bits.astype(np.uint16).view(np.float16).astype(np.float64)
+    else:
+        with np.errstate(invalid="ignore"):   # the nan patterns
+            v = (bits << 16).view(np.float32).astype(np.float64)
+    return np.unique(v[np.isfinite(v)])
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_2bit_threshold_counts_give_the_exact_codes(dtype):
+    """The 2-bit rule: with X_k = z + (k + 1/2) s (exact in float64), c_k is the
+    smallest 16-bit value v with v >= X_k (v > X_k for even k, so that a tie
+    goes to the even code), and the code of x is the number of c_k that x
+    reaches.  Here c_k is found by searching the sorted set of all 16-bit
+    values; for every 16-bit input of each unit the count must equal the
+    oracle's exact round-half-even code."""
+    vals = _all_finite16(dtype)
+    rng = np.random.default_rng(17 if dtype == "fp16" else 18)
+    checked = 0
+    for _ in range(400):
+        scale = float(np.exp(rng.uniform(np.log(1e-6), np.log(300.0))))
+        lo, hi = np.sort(rng.normal(0.0, 1.0, 2)) * scale + rng.normal(0.0, 3.0) * scale
+        lo_i = np.searchsorted(vals, lo)
+        hi_i = max(np.searchsorted(vals, hi, side="right") - 1, lo_i)
+        xs = vals[lo_i:hi_i + 1]
+        mn, mx = xs[0], xs[-1]
+        s, z = kivi.params(np.float64(mn), np.float64(mx), 2)
+        if s == 0:
+            continue
+        count = np.zeros(xs.shape, np.int64)
+        for k in range(3):
+            X = z + (k + 0.5) * s
+            i = np.searchsorted(vals, X, side="right" if k % 2 == 0 else "left")
+            c = vals[i] if i < vals.size else np.inf
+            count += xs >= c
+        assert np.array_equal(count, kivi.codes(xs, s, z, 2)), (mn, mx, s, z)
+        checked += xs.size
+    assert checked > 100000
