@@ -157,8 +157,9 @@ typedef struct kvq_cache kvq_cache; /* opaque host handle */
  * config is invalid or unsupported. */
 size_t kvq_cache_bytes(const kvq_config* cfg);
 
-/* Device scratch bytes kvq_decode_attention needs (split-K partial states);
- * 0 if the config is invalid. */
+/* Device scratch bytes kvq_decode_attention needs: the split-K partial states
+ * and, for TURBO, the rotated query of every (batch, kv head) row; 0 if the
+ * config is invalid. */
 size_t kvq_workspace_bytes(const kvq_config* cfg);
 
 /* Fills *out with the buffer layout of a config. */
