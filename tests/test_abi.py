@@ -132,3 +132,12 @@ def test_unsupported_turbo_configs_are_rejected(lib, field, value):
     cfg = config_from_workload(WORKLOADS["tq"])
     setattr(cfg, field, value)
     assert lib.kvq_cache_bytes(ctypes.byref(cfg)) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """No fallback: without libkvq.so every call path raises."""
+    from quantized_kv_cache_18_b200 import _lib as L
+    monkeypatch.setattr(L, "_lib", None)
+    monkeypatch.setattr(L, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libkvq.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        L.load()
